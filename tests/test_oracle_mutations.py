@@ -1,0 +1,92 @@
+"""Plants plausible mistakes into a copy of the oracle's C source (on the CPU, in a temporary
+directory) and checks that at least one pin of test_oracle_pins.py fails for each of them.
+This shows the pins constrain every part of the oracle, not just the parts they name."""
+import ctypes
+import json
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
+
+# (name, text in ssm_oracle.c, replacement): one plausible slip each.
+MUTATIONS = [
+    ("euler_bbar", "expm1(delta * A) / A * B;", "delta * B;"),
+    ("dropped_D_skip", "y += (D ? D[d] : 0.0) * u[t];", "y += 0.0 * u[t];"),
+    ("reversed_taps", "acc += w[k] * x[t - k];", "acc += w[K - 1 - k] * x[t - k];"),
+    ("gate_sigmoid_not_silu", "y * ssm_oracle_silu(z[off + t])", "y * ssm_oracle_sigmoid(z[off + t])"),
+    ("softplus_dropped_max", "log1p(exp(-fabs(v))) + (v > 0.0 ? v : 0.0)", "log1p(exp(-fabs(v)))"),
+    ("input_inside_decay", "h[n] = Abar * h[n] + Bbar * u[t];", "h[n] = Abar * (h[n] + Bbar * u[t]);"),
+    ("A_sign", "const double A = -exp(A_log[d * N + n]);", "const double A = -exp(-A_log[d * N + n]);"),
+    ("dropped_conv_bias", "double acc = b;", "double acc = 0.0 * b;"),
+    ("bwd_lambda_same_step", "lam[n] = dy[t] * Cb[n * L + t] + anext * lam[n];",
+     "lam[n] = dy[t] * Cb[n * L + t] + a[i] * lam[n];"),
+    ("bwd_dA_dropped_input_term", "u[t] * Bt_n * (xx * a[i] - em1[i]) / (A[n] * A[n]));", "0.0);"),
+    ("bwd_dB_euler", "dBb[n * L + t] += lam[n] * u[t] * em1[i] / A[n];",
+     "dBb[n * L + t] += lam[n] * u[t] * dl[t];"),
+    ("bwd_gate_derivative", "s * (1.0 + zz * (1.0 - s))", "s"),
+    ("bwd_conv_dx_taps", "acc += w[k] * dc[j + k];", "acc += w[K - 1 - k] * dc[j + k];"),
+    ("bwd_dAlog_chain", "= dA[n] * A[n];", "= dA[n];"),
+]
+
+
+def _pin_functions():
+    return [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _run_pins(gold):
+    failed = []
+    for fn in _pin_functions():
+        try:
+            if "gold" in fn.__code__.co_varnames[:fn.__code__.co_argcount]:
+                fn(gold)
+            else:
+                fn()
+        except AssertionError:
+            failed.append(fn.__name__)
+        except Exception:
+            failed.append(fn.__name__ + "(error)")
+    return failed
+
+
+@pytest.fixture(scope="module")
+def gold():
+    with open(pins.GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.fixture(scope="module")
+def workdir():
+    d = tempfile.mkdtemp(prefix="oracle_mut_")
+    yield d
+    shutil.rmtree(d, ignore_errors=True)
+
+
+def test_unmutated_oracle_passes_every_pin(gold):
+    assert _run_pins(gold) == []
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_mutation_is_caught(name, old, new, gold, workdir):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found: " + name
+    mutated = src.replace(old, new)
+    cpath = os.path.join(workdir, name + ".c")
+    sopath = os.path.join(workdir, "lib" + name + ".so")
+    with open(cpath, "w") as f:
+        f.write(mutated)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-w", "-o", sopath,
+                    cpath, "-lm"], check=True)
+    saved = oracle._lib
+    oracle._lib = oracle.bind(ctypes.CDLL(sopath))
+    try:
+        failed = _run_pins(gold)
+    finally:
+        oracle._lib = saved
+    assert failed, "no pin caught mutation " + name
