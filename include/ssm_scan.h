@@ -1,0 +1,170 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective-scan library (Mamba-1 S6).
+ *
+ * The operation (per batch element b, channel d, state n, time t):
+ *
+ *   u_t      = SiLU(conv_b[d] + sum_{k<K} conv_w[d][k] * x_{t-k})      (x_{t<0} = 0)
+ *   Delta_t  = softplus(dt_t + dt_bias[d])          (or dt_t + dt_bias[d] when delta_softplus = 0)
+ *   A        = -exp(A_log[d][n])
+ *   A_bar    = exp(Delta_t * A),   B_bar = (A_bar - 1) / A * B_t[n]      (exact zero-order hold)
+ *   h_t[n]   = A_bar * h_{t-1}[n] + B_bar * u_t,                         h_{-1} = 0
+ *   y_t      = sum_n C_t[n] * h_t[n] + D[d] * u_t
+ *   out_t    = y_t * SiLU(z_t)
+ *
+ * Sources (page title, section):
+ *  - "Sequence and state-space models" (docs.algenta.ai), `state_space_models`: the exact ZOH
+ *    pair ssm_discretize_zoh / ssm_discretize_b, ssm_recurrence_step, ssm_output_step and
+ *    mamba_delta_softplus.
+ *  - "state-space models" (aarnphm.xyz): "From continuous time to tokens", "One recurrence, one
+ *    convolution" (h_{-1} = 0), "Mamba" (token-dependent Delta_t, B_t, C_t; fixed diagonal A).
+ *  - "State-Space Models & Long-Context Sequence Architectures (Mamba)" (glossary),
+ *    "Mathematical Formulation" (the D feed-through) and Lab 3 (associative scan).
+ *  - "Selective Mamba" (TorchLean Runtime.Autograd.Model.Mamba): Parameters (convKernel rows
+ *    newest-first, convBias before the SiLU, logA, dSkip on the activated feature, the SiLU
+ *    gate; B and C shared by the expanded channels), Options.validate (empty axes rejected),
+ *    runArray (an empty chunk changes nothing).
+ *  - rustytorch commit log: the real S6 forward order and the hand-written VJP (reverse-time
+ *    recurrence; dA_log = dA * A).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named "device" are CUDA device (or managed) memory on the current device. The
+ *    caller owns every buffer; the library allocates nothing on the device and keeps no global
+ *    mutable state, so calls from several host threads on different streams are safe.
+ *  - Layouts are dense, row-major, innermost axis last: activations (Bt, Dn, L) with L
+ *    contiguous; B and C (Bt, N, L) with L contiguous; per-channel parameters fp32.
+ *    conv_w is [Dn, K] (each channel's taps contiguous, tap 0 = the current token), i.e. the
+ *    transpose of the page's [kernelWidth, innerWidth] orientation.
+ *  - Validation is synchronous on the host and happens before any launch; on an error nothing
+ *    is launched. Execution is asynchronous on `stream` (a cudaStream_t passed as void*; NULL =
+ *    the legacy default stream). A returned SSM_OK means the launches were enqueued; later
+ *    device faults surface on the stream as usual.
+ *  - Sizes: Dn, N and (with a conv) K must be >= 1 (SSM_ERR_SHAPE otherwise); Bt = 0 or L = 0 is
+ *    a valid empty problem and returns SSM_OK without launching anything.
+ *  - Alignment: every tensor pointer must be aligned to its element size (SSM_ERR_ALIGN).
+ *    Inputs whose rows are also 16-byte aligned (L * element size a multiple of 16 and 16-byte
+ *    aligned bases) take the 128-bit cp.async path; others take a scalar-load path.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ssm_status {
+  SSM_OK = 0,
+  SSM_ERR_NULL = 1,        /* a required pointer is NULL */
+  SSM_ERR_SHAPE = 2,       /* negative size, empty internal axis, or size overflow */
+  SSM_ERR_ALIGN = 3,       /* a pointer is not aligned to its element type */
+  SSM_ERR_DTYPE = 4,       /* unknown dtype code */
+  SSM_ERR_UNSUPPORTED = 5, /* d_state > 64 or K > 4 */
+  SSM_ERR_CUDA = 6,        /* a CUDA call or launch failed; see ssm_last_cuda_error() */
+  SSM_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssm_*_workspace_size() */
+  SSM_ERR_TIMEOUT = 8      /* reserved for bounded device-side waits; not returned today */
+} ssm_status;
+
+typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+/* Time steps between saved states (chunk_states) and of the backward's recompute blocks. */
+#define SSM_STATE_CHUNK 16
+
+/* Number of saved states per channel for a sequence of length L: ceil(L / SSM_STATE_CHUNK). */
+int64_t ssm_num_state_chunks(int64_t L);
+
+/*
+ * Forward arguments. The activations x, dt, z, B, C share one dtype (in_dtype); out and u_out
+ * share out_dtype. fp32 inputs select the accurate math path (library expf/expm1f/log1pf);
+ * bf16 inputs select the fast path (hardware ex2/lg2/rcp approximations).
+ */
+typedef struct ssm_fwd_args {
+  const void *x;         /* device (Bt, Dn, L): pre-conv input when conv_w != NULL, else u itself */
+  const void *dt;        /* device (Bt, Dn, L): time-step input before dt_bias / softplus */
+  const float *dt_bias;  /* device [Dn] or NULL (= 0) */
+  const float *A_log;    /* device [Dn, N]: A = -exp(A_log) */
+  const void *B;         /* device (Bt, N, L): input state vectors, shared by all channels */
+  const void *C;         /* device (Bt, N, L): readout state vectors, shared by all channels */
+  const float *D;        /* device [Dn] or NULL (= 0): skip coefficient on u */
+  const void *z;         /* device (Bt, Dn, L) or NULL: no SiLU(z) gate */
+  const float *conv_w;   /* device [Dn, K] newest-first taps, or NULL: no conv (x is u) */
+  const float *conv_b;   /* device [Dn] or NULL (= 0); ignored without conv_w */
+  void *out;             /* device (Bt, Dn, L), out_dtype: the gated output */
+  float *chunk_states;   /* device (Bt, Dn, ssm_num_state_chunks(L), N) fp32 or NULL: h after
+                            every SSM_STATE_CHUNK-th step (the last entry after step L-1);
+                            ssm_scan_bwd consumes them */
+  void *u_out;           /* device (Bt, Dn, L), out_dtype, or NULL: the scan input u */
+  int64_t Bt, Dn, N, L;  /* batch, channels (d_inner), states (d_state), sequence length */
+  int32_t K;             /* conv taps, 1..4 (ignored without conv_w) */
+  int32_t in_dtype;      /* ssm_dtype of x, dt, z, B, C */
+  int32_t out_dtype;     /* ssm_dtype of out and u_out */
+  int32_t delta_softplus;/* 1: Delta = softplus(dt + dt_bias); 0: Delta = dt + dt_bias */
+} ssm_fwd_args;
+
+/*
+ * Forward selective scan with the causal depthwise conv1d + SiLU fused in front and the SiLU(z)
+ * gate fused behind: computes every output listed in ssm_fwd_args on `stream`.
+ * Errors: SSM_ERR_NULL (x, dt, A_log, B, C or out NULL), SSM_ERR_SHAPE, SSM_ERR_ALIGN,
+ * SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED (N > 64, K outside 1..4), SSM_ERR_CUDA.
+ */
+ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream);
+
+/*
+ * Backward arguments: the forward's inputs (same meaning and dtypes; out/u_out unused) plus the
+ * upstream gradient and the gradient outputs. Every gradient output is fp32, caller-allocated,
+ * OVERWRITTEN (never accumulated into) and may be NULL when not wanted.
+ */
+typedef struct ssm_bwd_args {
+  ssm_fwd_args fwd;            /* forward inputs; fwd.out and fwd.u_out are ignored */
+  const void *dout;            /* device (Bt, Dn, L), fwd.in_dtype: dLoss/dout */
+  const float *chunk_states;   /* device states saved by ssm_scan_fwd, or NULL: recomputed into
+                                  the workspace */
+  float *dx;      /* (Bt, Dn, L): w.r.t. the pre-conv x, or w.r.t. u when there is no conv */
+  float *ddt;     /* (Bt, Dn, L): w.r.t. dt (before dt_bias / softplus) */
+  float *dz;      /* (Bt, Dn, L): w.r.t. z (ignored without a gate) */
+  float *dA_log;  /* [Dn, N] */
+  float *dB;      /* (Bt, N, L) */
+  float *dC;      /* (Bt, N, L) */
+  float *dD;      /* [Dn] */
+  float *ddt_bias;/* [Dn] */
+  float *dconv_w; /* [Dn, K] (ignored without a conv) */
+  float *dconv_b; /* [Dn]    (ignored without a conv) */
+  void *workspace;          /* device scratch of at least ssm_bwd_workspace_size() bytes,
+                               256-byte aligned; contents need not be initialised */
+  size_t workspace_bytes;
+} ssm_bwd_args;
+
+/* Bytes of device scratch ssm_scan_bwd needs for these arguments (0 for an empty problem). */
+size_t ssm_bwd_workspace_size(const ssm_bwd_args *args);
+
+/*
+ * Backward (vector-Jacobian product) of ssm_scan_fwd against `dout`: the reverse-time adjoint
+ * recurrence lambda_t = C_t * dy_t + A_bar_{t+1} * lambda_{t+1} over the states recomputed from
+ * chunk_states, with all parameter gradients. Deterministic: cross-channel and cross-batch sums
+ * are reduced in a fixed order. Errors as ssm_scan_fwd, plus SSM_ERR_WORKSPACE.
+ */
+ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream);
+
+/*
+ * Standalone causal depthwise conv1d + SiLU: u = SiLU(b + sum_k w[k] * x_{t-k}).
+ * x: device (Bt, Dn, L) in_dtype; u: device (Bt, Dn, L) out_dtype; w: device [Dn, K] fp32,
+ * newest-first; b: device [Dn] fp32 or NULL. K in 1..4.
+ * Errors: SSM_ERR_NULL, SSM_ERR_SHAPE, SSM_ERR_ALIGN, SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED,
+ * SSM_ERR_CUDA.
+ */
+ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
+                           int64_t Dn, int64_t L, int32_t K, int32_t in_dtype, int32_t out_dtype,
+                           void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *ssm_status_string(ssm_status s);
+
+/* The cudaError_t (as int) behind the calling thread's most recent SSM_ERR_CUDA, or 0. */
+int ssm_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

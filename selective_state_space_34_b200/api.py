@@ -1,0 +1,199 @@
+"""PyTorch-facing marshalling for the C ABI (include/ssm_scan.h).
+
+Each function validates tensor devices/dtypes/contiguity, allocates outputs (and the backward's
+scratch) with torch on the inputs' device, fills the C argument struct with raw device pointers
+and calls the library on torch's current CUDA stream. Nothing is computed here.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, Optional
+
+import torch
+
+from . import _abi
+
+_DT = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(name: str, t: torch.Tensor) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (the library has no CPU path)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _opt(name, t, dtype=None):
+    if t is None:
+        return None
+    _need_cuda(name, t)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    return t
+
+
+def _stream_handle(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def ssm_num_state_chunks(L: int) -> int:
+    return int(_abi.load().ssm_num_state_chunks(int(L)))
+
+
+def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype):
+    for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
+        _need_cuda(n, t)
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    act = x.dtype
+    for n, t in (("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != act:
+            raise TypeError("%s must have the activation dtype %s" % (n, act))
+    _opt("z", z, act)
+    for n, t in (("A_log", A_log), ("D", D), ("dt_bias", dt_bias), ("conv_w", conv_w),
+                 ("conv_b", conv_b)):
+        _opt(n, t, torch.float32)
+    if x.dim() != 3 or B.dim() != 3 or A_log.dim() != 2:
+        raise ValueError("x must be (Bt, Dn, L), B/C (Bt, N, L), A_log (Dn, N)")
+    Bt, Dn, L = x.shape
+    N = A_log.shape[1]
+    if tuple(dt.shape) != (Bt, Dn, L) or (z is not None and tuple(z.shape) != (Bt, Dn, L)):
+        raise ValueError("dt and z must have the shape of x")
+    if tuple(B.shape) != (Bt, N, L) or tuple(C.shape) != (Bt, N, L) or A_log.shape[0] != Dn:
+        raise ValueError("B, C must be (Bt, N, L) and A_log (Dn, N)")
+    for n, t in (("D", D), ("dt_bias", dt_bias), ("conv_b", conv_b)):
+        if t is not None and tuple(t.shape) != (Dn,):
+            raise ValueError("%s must be (Dn,)" % n)
+    K = 0
+    if conv_w is not None:
+        if conv_w.dim() != 2 or conv_w.shape[0] != Dn:
+            raise ValueError("conv_w must be (Dn, K)")
+        K = conv_w.shape[1]
+    od = act if out_dtype is None else out_dtype
+    if od not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    a = _abi.FwdArgs()
+    a.x, a.dt, a.dt_bias, a.A_log = _ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log)
+    a.B, a.C, a.D, a.z = _ptr(B), _ptr(C), _ptr(D), _ptr(z)
+    a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
+    a.Bt, a.Dn, a.N, a.L, a.K = Bt, Dn, N, L, K
+    a.in_dtype, a.out_dtype = _DT[act], _DT[od]
+    a.delta_softplus = 1 if delta_softplus else 0
+    return a, od
+
+
+def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, conv_b=None,
+                 delta_softplus: bool = True, out_dtype=None, save_states: bool = False,
+                 return_u: bool = False, out: Optional[torch.Tensor] = None):
+    """Fused forward. Returns ``out`` or a dict with ``out`` and, when asked, ``chunk_states``
+    ((Bt, Dn, ceil(L/16), N) fp32, for ssm_scan_bwd) and ``u`` (the scan input)."""
+    a, od = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype)
+    Bt, Dn, L = x.shape
+    N = A_log.shape[1]
+    if out is None:
+        out = torch.empty((Bt, Dn, L), dtype=od, device=x.device)
+    else:
+        _opt("out", out, od)
+    a.out = _ptr(out)
+    res: Dict[str, torch.Tensor] = {"out": out}
+    if save_states:
+        st = torch.empty((Bt, Dn, ssm_num_state_chunks(L), N), dtype=torch.float32, device=x.device)
+        a.chunk_states = _ptr(st)
+        res["chunk_states"] = st
+    if return_u:
+        u = torch.empty((Bt, Dn, L), dtype=od, device=x.device)
+        a.u_out = _ptr(u)
+        res["u"] = u
+    lib = _abi.load()
+    _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(a), _stream_handle(x.device)))
+    return res if (save_states or return_u) else out
+
+
+def _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
+                chunk_states):
+    a, _ = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, None)
+    _need_cuda("dout", dout)
+    if dout.dtype != x.dtype or dout.shape != x.shape:
+        raise ValueError("dout must match x in shape and dtype")
+    _opt("chunk_states", chunk_states, torch.float32)
+    bw = _abi.BwdArgs()
+    bw.fwd = a
+    bw.dout = _ptr(dout)
+    bw.chunk_states = _ptr(chunk_states)
+    return bw
+
+
+def ssm_bwd_workspace_size(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None,
+                           conv_b=None, delta_softplus=True, chunk_states=None) -> int:
+    bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
+                     chunk_states)
+    return int(_abi.load().ssm_bwd_workspace_size(ctypes.byref(bw)))
+
+
+def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None,
+                 conv_b=None, delta_softplus: bool = True, chunk_states=None,
+                 workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None):
+    """Backward. Returns a dict of fp32 gradients: dx, ddt, dA_log, dB, dC, and dD / ddt_bias /
+    dz / dconv_w / dconv_b where the corresponding input exists. ``workspace`` (uint8, at least
+    ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call."""
+    bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
+                     chunk_states)
+    Bt, Dn, L = x.shape
+    N = A_log.shape[1]
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    if grads is None:
+        grads = {"dx": torch.empty((Bt, Dn, L), **f32), "ddt": torch.empty((Bt, Dn, L), **f32),
+                 "dA_log": torch.empty((Dn, N), **f32), "dB": torch.empty((Bt, N, L), **f32),
+                 "dC": torch.empty((Bt, N, L), **f32)}
+        if D is not None:
+            grads["dD"] = torch.empty((Dn,), **f32)
+        if dt_bias is not None:
+            grads["ddt_bias"] = torch.empty((Dn,), **f32)
+        if z is not None:
+            grads["dz"] = torch.empty((Bt, Dn, L), **f32)
+        if conv_w is not None:
+            grads["dconv_w"] = torch.empty(tuple(conv_w.shape), **f32)
+            grads["dconv_b"] = torch.empty((Dn,), **f32)
+    for k, v in grads.items():
+        _opt(k, v, torch.float32)
+        setattr(bw, k, _ptr(v))
+    lib = _abi.load()
+    need = int(lib.ssm_bwd_workspace_size(ctypes.byref(bw)))
+    if need > 0:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+        base = workspace.data_ptr()
+        aligned = (base + 255) & ~255
+        if aligned + need > base + workspace.numel() * workspace.element_size():
+            workspace = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+            base = workspace.data_ptr()
+            aligned = (base + 255) & ~255
+        bw.workspace = aligned
+        bw.workspace_bytes = need
+    _abi.check("ssm_scan_bwd", lib.ssm_scan_bwd(ctypes.byref(bw), _stream_handle(dev)))
+    return grads
+
+
+def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = None):
+    """Standalone causal depthwise conv1d + SiLU: x (Bt, Dn, L), w (Dn, K) newest-first."""
+    _need_cuda("x", x)
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    _opt("w", w, torch.float32)
+    _opt("b", b, torch.float32)
+    Bt, Dn, L = x.shape
+    od = x.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((Bt, Dn, L), dtype=od, device=x.device)
+    lib = _abi.load()
+    _abi.check("ssm_conv1d_silu", lib.ssm_conv1d_silu(
+        _ptr(x), _ptr(out), _ptr(w), _ptr(b), Bt, Dn, L, int(w.shape[1]), _DT[x.dtype], _DT[od],
+        _stream_handle(x.device)))
+    return out

@@ -1,0 +1,218 @@
+// ssm_api.cu -- the extern "C" boundary declared in include/ssm_scan.h: host-side validation
+// (synchronous, before any launch) and dispatch to the kernel launchers. No exception crosses the
+// ABI and the library allocates no device memory.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/ssm_scan.h"
+#include "ssm_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+ssm_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SSM_OK;
+  g_last_cuda_error = (int)e;
+  return SSM_ERR_CUDA;
+}
+
+size_t dtype_size(int32_t dt) { return dt == SSM_BF16 ? 2 : 4; }
+bool dtype_ok(int32_t dt) { return dt == SSM_F32 || dt == SSM_BF16; }
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > INT64_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+// Shape, dtype and pointer checks shared by forward and backward. Sets *empty for Bt = 0 or L = 0.
+ssm_status check_fwd(const ssm_fwd_args *a, bool need_out, bool *empty) {
+  if (!a) return SSM_ERR_NULL;
+  if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
+  if (a->Bt < 0 || a->Dn < 0 || a->N < 0 || a->L < 0) return SSM_ERR_SHAPE;
+  if (a->Dn == 0 || a->N == 0) return SSM_ERR_SHAPE;  // empty internal axes are rejected
+  if (a->conv_w && a->K <= 0) return SSM_ERR_SHAPE;
+  if (a->N > 64) return SSM_ERR_UNSUPPORTED;
+  if (a->conv_w && a->K > 4) return SSM_ERR_UNSUPPORTED;
+  int64_t rows, elems, bc;
+  if (!mul_ok(a->Bt, a->Dn, &rows) || !mul_ok(rows, a->L, &elems) || !mul_ok(a->Bt, a->N, &bc) ||
+      !mul_ok(bc, a->L, &bc) || elems > (INT64_C(1) << 50))
+    return SSM_ERR_SHAPE;
+  *empty = (a->Bt == 0 || a->L == 0);
+  if (*empty) return SSM_OK;
+  if (!a->x || !a->dt || !a->A_log || !a->B || !a->C || (need_out && !a->out)) return SSM_ERR_NULL;
+  const size_t ei = dtype_size(a->in_dtype), eo = dtype_size(a->out_dtype);
+  const void *in_ptrs[5] = {a->x, a->dt, a->z, a->B, a->C};
+  for (const void *p : in_ptrs)
+    if (p && !aligned(p, ei)) return SSM_ERR_ALIGN;
+  if ((a->out && !aligned(a->out, eo)) || (a->u_out && !aligned(a->u_out, eo))) return SSM_ERR_ALIGN;
+  const void *f32_ptrs[6] = {a->dt_bias, a->A_log, a->D, a->conv_w, a->conv_b, a->chunk_states};
+  for (const void *p : f32_ptrs)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  return SSM_OK;
+}
+
+// 16-byte staging / vector stores are allowed when every row starts on a 16-byte boundary.
+int vec_ok(const ssm_fwd_args *a, const void *const *extra, int n_extra) {
+  if (a->L % 8 != 0) return 0;
+  const void *ptrs[7] = {a->x, a->dt, a->z, a->B, a->C, a->out, a->u_out};
+  for (const void *p : ptrs)
+    if (p && !aligned(p, 16)) return 0;
+  for (int i = 0; i < n_extra; i++)
+    if (extra[i] && !aligned(extra[i], 16)) return 0;
+  return 1;
+}
+
+ssm::FwdParams make_fwd_params(const ssm_fwd_args *a, int vec) {
+  ssm::FwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.B = a->B;
+  p.C = a->C;
+  p.dt_bias = a->dt_bias;
+  p.A_log = a->A_log;
+  p.D = a->D;
+  p.conv_w = a->conv_w;
+  p.conv_b = a->conv_w ? a->conv_b : nullptr;
+  p.out = a->out;
+  p.u_out = a->u_out;
+  p.chunk_states = a->chunk_states;
+  p.Bt = a->Bt;
+  p.Dn = a->Dn;
+  p.N = a->N;
+  p.L = a->L;
+  p.n_ck = ssm_num_state_chunks(a->L);
+  p.K = a->conv_w ? a->K : 0;
+  p.delta_softplus = a->delta_softplus ? 1 : 0;
+  p.vec = vec;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t ssm_num_state_chunks(int64_t L) {
+  return L <= 0 ? 0 : (L + SSM_STATE_CHUNK - 1) / SSM_STATE_CHUNK;
+}
+
+const char *ssm_status_string(ssm_status s) {
+  switch (s) {
+    case SSM_OK: return "SSM_OK: success";
+    case SSM_ERR_NULL: return "SSM_ERR_NULL: a required pointer is NULL";
+    case SSM_ERR_SHAPE: return "SSM_ERR_SHAPE: negative size, empty internal axis or size overflow";
+    case SSM_ERR_ALIGN: return "SSM_ERR_ALIGN: a pointer is not aligned to its element type";
+    case SSM_ERR_DTYPE: return "SSM_ERR_DTYPE: unknown dtype code";
+    case SSM_ERR_UNSUPPORTED: return "SSM_ERR_UNSUPPORTED: d_state > 64 or conv taps > 4";
+    case SSM_ERR_CUDA: return "SSM_ERR_CUDA: a CUDA call or launch failed";
+    case SSM_ERR_WORKSPACE: return "SSM_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case SSM_ERR_TIMEOUT: return "SSM_ERR_TIMEOUT: a bounded device wait ran out";
+  }
+  return "unknown ssm_status";
+}
+
+int ssm_last_cuda_error(void) { return g_last_cuda_error; }
+
+ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream) {
+  bool empty = false;
+  ssm_status st = check_fwd(args, true, &empty);
+  if (st != SSM_OK || empty) return st;
+  const ssm::FwdParams p = make_fwd_params(args, vec_ok(args, nullptr, 0));
+  return cuda_status(ssm::launch_fwd(p, args->in_dtype == SSM_BF16, args->out_dtype == SSM_BF16,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
+                           int64_t Dn, int64_t L, int32_t K, int32_t in_dtype, int32_t out_dtype,
+                           void *stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return SSM_ERR_DTYPE;
+  if (Bt < 0 || Dn < 0 || L < 0) return SSM_ERR_SHAPE;
+  if (Dn == 0 || K <= 0) return SSM_ERR_SHAPE;
+  if (K > 4) return SSM_ERR_UNSUPPORTED;
+  int64_t rows, elems;
+  if (!mul_ok(Bt, Dn, &rows) || !mul_ok(rows, L, &elems) || elems > (INT64_C(1) << 50))
+    return SSM_ERR_SHAPE;
+  if (Bt == 0 || L == 0) return SSM_OK;
+  if (!x || !u || !w) return SSM_ERR_NULL;
+  if (!aligned(x, dtype_size(in_dtype)) || !aligned(u, dtype_size(out_dtype)) || !aligned(w, 4) ||
+      (b && !aligned(b, 4)))
+    return SSM_ERR_ALIGN;
+  return cuda_status(ssm::launch_conv1d_silu(x, u, w, b, Bt, Dn, L, K, in_dtype == SSM_BF16,
+                                             out_dtype == SSM_BF16, 0,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {
+  if (!args) return 0;
+  const ssm_fwd_args *a = &args->fwd;
+  if (a->Bt <= 0 || a->L <= 0 || a->Dn <= 0 || a->N <= 0) return 0;
+  return ssm::bwd_workspace_bytes(a->Bt, a->Dn, a->N, a->L, args->chunk_states == nullptr);
+}
+
+ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
+  if (!args) return SSM_ERR_NULL;
+  bool empty = false;
+  ssm_status st = check_fwd(&args->fwd, false, &empty);
+  if (st != SSM_OK) return st;
+  const ssm_fwd_args *a = &args->fwd;
+  if (empty) return SSM_OK;
+  if (!args->dout) return SSM_ERR_NULL;
+  if (!aligned(args->dout, dtype_size(a->in_dtype))) return SSM_ERR_ALIGN;
+  const void *g32[12] = {args->chunk_states, args->dx, args->ddt, args->dz, args->dA_log, args->dB,
+                         args->dC, args->dD, args->ddt_bias, args->dconv_w, args->dconv_b,
+                         nullptr};
+  for (const void *p : g32)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  const size_t need = ssm_bwd_workspace_size(args);
+  if (need > 0 && (!args->workspace || args->workspace_bytes < need || !aligned(args->workspace, 256)))
+    return SSM_ERR_WORKSPACE;
+
+  const void *extra[5] = {args->dout, args->dx, args->ddt, args->dz, nullptr};
+  ssm_fwd_args fa = *a;
+  fa.out = nullptr;
+  fa.u_out = nullptr;
+  fa.chunk_states = nullptr;
+  ssm::BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.f = make_fwd_params(&fa, vec_ok(&fa, extra, 4));
+  p.dout = args->dout;
+  p.chunk_states = args->chunk_states;
+  p.dx = args->dx;
+  p.ddt = args->ddt;
+  p.dz = a->z ? args->dz : nullptr;
+  p.dB = args->dB;
+  p.dC = args->dC;
+  p.dA_log = args->dA_log;
+  p.dD = args->dD;
+  p.ddt_bias = args->ddt_bias;
+  p.dconv_w = a->conv_w ? args->dconv_w : nullptr;
+  p.dconv_b = a->conv_w ? args->dconv_b : nullptr;
+  // carve the workspace (layout mirrored by ssm::bwd_workspace_bytes)
+  char *ws = static_cast<char *>(args->workspace);
+  auto take = [&](size_t bytes) {
+    char *r = ws;
+    ws += (bytes + 255) & ~size_t(255);
+    return r;
+  };
+  const ssm::LaneLayout lay = ssm::choose_layout(a->N, a->Bt * a->Dn);
+  const int64_t ch = ssm::channels_per_cta(lay);
+  p.n_dtiles = (a->Dn + ch - 1) / ch;
+  const int64_t BD = a->Bt * a->Dn;
+  p.p_dA_log = reinterpret_cast<float *>(take(sizeof(float) * BD * a->N));
+  p.p_dD = reinterpret_cast<float *>(take(sizeof(float) * BD));
+  p.p_ddt_bias = reinterpret_cast<float *>(take(sizeof(float) * BD));
+  p.p_dconv_w = reinterpret_cast<float *>(take(sizeof(float) * BD * 4));
+  p.p_dconv_b = reinterpret_cast<float *>(take(sizeof(float) * BD));
+  p.p_dB = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
+  p.p_dC = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
+  if (!args->chunk_states)
+    p.f.chunk_states = reinterpret_cast<float *>(take(sizeof(float) * BD * p.f.n_ck * a->N));
+  return cuda_status(ssm::launch_bwd(p, a->in_dtype == SSM_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,537 @@
+// ssm_bwd.cu -- selective-scan backward (vector-Jacobian product) for sm_100a.
+//
+// The analytic VJP of the fused forward, run as a reverse-time recurrence over the states that
+// are recomputed block by block from the saved chunk states (rustytorch commit log, "Hand-written
+// VJP": reverse-time recurrence over the cached h trajectory; dA_log = dA * A). With
+// x = Delta*A, a = exp(x), lambda_t = dL/dh_t:
+//
+//   lambda_t   = dy_t C_t + a_{t+1} lambda_{t+1}
+//   dC_t[n]   += dy_t h_t[n]                        (summed over channels)
+//   dB_t[n]   += lambda_t[n] u_t (a - 1) / A        (summed over channels)
+//   dDelta_t   = sum_n lambda_t[n] (A h_t[n] + B_t[n] u_t)      [= a (A h_{t-1} + B u)]
+//   du_t       = D dy_t + sum_n lambda_t[n] B_bar_t[n]
+//   dA_log[n] += Delta_t * lambda (A h_t + B u) - u_t lambda B_bar
+//
+// The last line is A * dA (the chain rule through A = -exp(A_log)); it uses the identity
+// A * d(h-update)/dA = Delta * d(h-update)/dDelta - u * B_bar, which avoids the cancelling
+// difference x a - (a - 1) for small x.
+//
+// Decomposition mirrors the forward: a CTA owns CH = 128/G channels of one batch element, lanes
+// hold NS states each, and the sequence is walked backwards in stages of kT steps, each split in
+// blocks of kSub = 16 steps: recompute the block forward from its saved start state (a_t and h_t
+// kept in registers), then run the adjoint backwards through it. dB and dC are summed over the
+// CTA's channels in shared memory and written as per-tile partials; a second kernel adds the
+// tiles (and the per-batch partials of the per-channel parameter gradients) in a fixed order, so
+// the result is deterministic.
+#include "ssm_common.cuh"
+#include "ssm_internal.h"
+
+namespace ssm {
+
+template <typename T> __device__ __forceinline__ T bzero() { return from_f32<T>(0.0f); }
+
+// dst[r][i] = src[r][t0 + i] for r < rows_valid and 0 <= t0 + i < L, else 0, i in [0, LEN).
+template <typename T, int ROWS, int LEN>
+__device__ __forceinline__ void stage_rows_b(T *dst, int dst_stride, const T *src, int64_t src_stride,
+                                             int rows_valid, int64_t t0, int64_t L, bool vec) {
+  constexpr int EPV = 16 / sizeof(T);
+  constexpr int VPR = LEN / EPV;
+  if (vec) {
+    for (int idx = threadIdx.x; idx < ROWS * VPR; idx += kThreads) {
+      const int r = idx / VPR, v = idx % VPR;
+      const int64_t t = t0 + (int64_t)v * EPV;
+      T *d = dst + r * dst_stride + v * EPV;
+      if (r < rows_valid && t >= 0 && t < L)
+        cp_async16(d, src + (int64_t)r * src_stride + t);
+      else
+        *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
+    for (int idx = threadIdx.x; idx < ROWS * LEN; idx += kThreads) {
+      const int r = idx / LEN, i = idx % LEN;
+      const int64_t t = t0 + i;
+      dst[r * dst_stride + i] =
+          (r < rows_valid && t >= 0 && t < L) ? src[(int64_t)r * src_stride + t] : bzero<T>();
+    }
+  }
+}
+
+template <int G, int NS, typename Tin> struct BwdSmem {
+  static constexpr int CH = kThreads / G;
+  static constexpr int NP = G * NS;
+  static constexpr int XS = kPre + kT;
+  static constexpr int BS = NP + 4;
+  static constexpr int US = kT + 4;
+  static constexpr int YG = kSub + 8;
+  static constexpr int YC = G * YG + 4;
+  static constexpr int DCS = kT + 8;            // dc row: this stage, then the next stage's 3
+  static constexpr int RBS = CH + 2;            // reduction buffer: stride between steps
+  static constexpr int RBN = kSub * RBS + 2;    // reduction buffer: stride between states
+  static constexpr size_t x_off = 0;
+  static constexpr size_t dt_off = x_off + sizeof(Tin) * 2 * CH * XS;
+  static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * kT;
+  static constexpr size_t do_off = z_off + sizeof(Tin) * 2 * CH * kT;
+  static constexpr size_t braw_off = do_off + sizeof(Tin) * 2 * CH * kT;
+  static constexpr size_t craw_off = braw_off + sizeof(Tin) * 2 * NP * kT;
+  static constexpr size_t bs_off = craw_off + sizeof(Tin) * 2 * NP * kT;
+  static constexpr size_t cs_off = bs_off + sizeof(float) * kT * BS;
+  static constexpr size_t us_off = cs_off + sizeof(float) * kT * BS;
+  static constexpr size_t dls_off = us_off + sizeof(float) * CH * US;
+  static constexpr size_t dys_off = dls_off + sizeof(float) * CH * US;
+  static constexpr size_t yb0_off = dys_off + sizeof(float) * CH * US;
+  static constexpr size_t yb1_off = yb0_off + sizeof(float) * CH * YC;
+  static constexpr size_t dcs_off = yb1_off + sizeof(float) * CH * YC;
+  static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
+  static constexpr size_t bytes = rb_off + ((sizeof(float) * NP * RBN + 15) / 16) * 16;
+};
+
+template <int G, int NS, typename Tin>
+__global__ void __launch_bounds__(kThreads)
+ssm_bwd_kernel(const BwdParams P) {
+  using S = BwdSmem<G, NS, Tin>;
+  constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G;
+  constexpr bool PRECISE = sizeof(Tin) == 4;
+  const FwdParams &p = P.f;
+  extern __shared__ __align__(16) unsigned char smem[];
+  Tin *xs = reinterpret_cast<Tin *>(smem + S::x_off);
+  Tin *dts = reinterpret_cast<Tin *>(smem + S::dt_off);
+  Tin *zs = reinterpret_cast<Tin *>(smem + S::z_off);
+  Tin *dos = reinterpret_cast<Tin *>(smem + S::do_off);
+  Tin *braw = reinterpret_cast<Tin *>(smem + S::braw_off);
+  Tin *craw = reinterpret_cast<Tin *>(smem + S::craw_off);
+  float *Bs = reinterpret_cast<float *>(smem + S::bs_off);
+  float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
+  float *us = reinterpret_cast<float *>(smem + S::us_off);
+  float *dls = reinterpret_cast<float *>(smem + S::dls_off);
+  float *dys = reinterpret_cast<float *>(smem + S::dys_off);
+  float *yb0 = reinterpret_cast<float *>(smem + S::yb0_off);
+  float *yb1 = reinterpret_cast<float *>(smem + S::yb1_off);
+  float *dcs = reinterpret_cast<float *>(smem + S::dcs_off);
+  float *rb = reinterpret_cast<float *>(smem + S::rb_off);
+
+  const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
+  const int64_t tile = blockIdx.x % n_dtiles;
+  const int64_t b = blockIdx.x / n_dtiles;
+  const int64_t d0 = tile * CH;
+  const int rows_valid = (int)imin64(CH, p.Dn - d0);
+  const int tid = threadIdx.x, c = tid / G, g = tid % G;
+  const int64_t d = d0 + c;
+  const bool live = d < p.Dn;
+  const bool has_conv = p.conv_w != nullptr, has_z = p.z != nullptr;
+  const bool vec = p.vec != 0;
+  const int64_t L = p.L, N = p.N;
+
+  float A[NS], Acoef[NS], invA[NS], lam[NS], aN[NS], dAl[NS];
+#pragma unroll
+  for (int j = 0; j < NS; j++) {
+    const int n = g * NS + j;
+    lam[j] = 0.f;
+    aN[j] = 0.f;
+    dAl[j] = 0.f;
+    if (live && n < N) {
+      A[j] = -expf(p.A_log[d * N + n]);
+      Acoef[j] = PRECISE ? A[j] : A[j] * kLog2e;
+      invA[j] = 1.0f / A[j];
+    } else {
+      A[j] = 0.f;
+      Acoef[j] = 0.f;
+      invA[j] = 0.f;
+    }
+  }
+  float w4[4] = {0.f, 0.f, 0.f, 0.f};
+  float cbias = 0.f, Dd = 0.f, dtb = 0.f;
+  if (live) {
+    if (has_conv) {
+      for (int k = 0; k < p.K; k++) w4[k] = p.conv_w[d * p.K + k];
+      cbias = p.conv_b ? p.conv_b[d] : 0.f;
+    }
+    Dd = p.D ? p.D[d] : 0.f;
+    dtb = p.dt_bias ? p.dt_bias[d] : 0.f;
+  }
+  float accD = 0.f, accDtb = 0.f, accCb = 0.f, accW[4] = {0.f, 0.f, 0.f, 0.f};
+
+  const int64_t row0 = (b * p.Dn + d0) * L;
+  const Tin *gx = static_cast<const Tin *>(p.x) + row0;
+  const Tin *gdt = static_cast<const Tin *>(p.dt) + row0;
+  const Tin *gz = has_z ? static_cast<const Tin *>(p.z) + row0 : nullptr;
+  const Tin *gdo = static_cast<const Tin *>(P.dout) + row0;
+  const Tin *gB = static_cast<const Tin *>(p.B) + b * N * L;
+  const Tin *gC = static_cast<const Tin *>(p.C) + b * N * L;
+  const int n_rows = (int)imin64(NP, N);
+  const float *states = P.chunk_states ? P.chunk_states : p.chunk_states;
+
+  // dc halo of the (non-existent) stage after the sequence end is zero
+  for (int i = tid; i < CH * S::DCS; i += kThreads) dcs[i] = 0.f;
+
+  const int64_t n_stages = (L + kT - 1) / kT;
+  auto issue = [&](int64_t stage, int buf) {
+    const int64_t t0 = stage * kT;
+    stage_rows_b<Tin, CH, kPre + kT>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
+    stage_rows_b<Tin, CH, kT>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
+    if (has_z) stage_rows_b<Tin, CH, kT>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
+    stage_rows_b<Tin, CH, kT>(dos + buf * CH * kT, kT, gdo, L, rows_valid, t0, L, vec);
+    stage_rows_b<Tin, NP, kT>(braw + buf * NP * kT, kT, gB, L, n_rows, t0, L, vec);
+    stage_rows_b<Tin, NP, kT>(craw + buf * NP * kT, kT, gC, L, n_rows, t0, L, vec);
+    cp_async_commit();
+  };
+
+  if (n_stages > 0) issue(n_stages - 1, (int)((n_stages - 1) & 1));
+  for (int64_t st = n_stages - 1; st >= 0; st--) {
+    const int buf = (int)(st & 1);
+    const int64_t t0 = st * kT;
+    cp_async_wait<0>();
+    __syncthreads();
+    if (st > 0) issue(st - 1, buf ^ 1);
+
+    for (int i = tid; i < NP * kT; i += kThreads) {
+      const int n = i / kT, t = i % kT;
+      Bs[t * S::BS + n] = to_f32(braw[buf * NP * kT + i]);
+      Cs[t * S::BS + n] = to_f32(craw[buf * NP * kT + i]);
+    }
+    const Tin *xrow = xs + (buf * CH + c) * S::XS + kPre;
+    const Tin *dtrow = dts + (buf * CH + c) * kT;
+    const Tin *zrow = zs + (buf * CH + c) * kT;
+    const Tin *dorow = dos + (buf * CH + c) * kT;
+
+    // per-element phase A: u, Delta, dy for the steps this lane owns
+#pragma unroll
+    for (int sb = 0; sb < kT / kSub; sb++) {
+#pragma unroll
+      for (int j = 0; j < EPL; j++) {
+        const int t = sb * kSub + g * EPL + j;
+        float u;
+        if (has_conv) {
+          float acc = cbias;
+#pragma unroll
+          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], to_f32(xrow[t - k]), acc);
+          u = acc * sigmoid<PRECISE>(acc);
+        } else {
+          u = to_f32(xrow[t]);
+        }
+        const float v = to_f32(dtrow[t]) + dtb;
+        float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
+        float dy = to_f32(dorow[t]);
+        if (has_z) {
+          const float zz = to_f32(zrow[t]);
+          dy *= zz * sigmoid<PRECISE>(zz);
+        }
+        if (t0 + t >= L) {
+          u = 0.f;
+          dl = 0.f;
+          dy = 0.f;
+        }
+        us[c * S::US + t] = u;
+        dls[c * S::US + t] = dl;
+        dys[c * S::US + t] = dy;
+      }
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int sb = kT / kSub - 1; sb >= 0; sb--) {
+      const int64_t tb = t0 + sb * kSub;  // first step of this block
+      // (a) start state of the block
+      float h0[NS];
+      {
+        const int64_t kk = tb / kSub;
+#pragma unroll
+        for (int j = 0; j < NS; j++) {
+          const int n = g * NS + j;
+          h0[j] = (kk > 0 && live && n < N) ? states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n] : 0.f;
+        }
+      }
+      // (b) forward recompute: e = A_bar (fast) or A_bar - 1 (precise), and h, kept in registers
+      float ea[kSub][NS], hh[kSub][NS];
+      float *my0 = yb0 + c * S::YC + g * S::YG;
+      float *my1 = yb1 + c * S::YC + g * S::YG;
+      {
+        float h[NS];
+#pragma unroll
+        for (int j = 0; j < NS; j++) h[j] = h0[j];
+#pragma unroll
+        for (int tt = 0; tt < kSub; tt++) {
+          const int t = sb * kSub + tt;
+          const float u = us[c * S::US + t], dl = dls[c * S::US + t], dy = dys[c * S::US + t];
+          const float *brow = Bs + t * S::BS + g * NS;
+          const float *crow = Cs + t * S::BS + g * NS;
+          float y = 0.f;
+#pragma unroll
+          for (int j = 0; j < NS; j++) {
+            const float w = brow[j] * u * invA[j];
+            if (PRECISE) {
+              const float em1 = expm1f(dl * Acoef[j]);
+              h[j] = fmaf(em1, h[j] + w, h[j]);
+              ea[tt][j] = em1;
+            } else {
+              const float a = ex2_approx(dl * Acoef[j]);
+              h[j] = fmaf(a, h[j] + w, -w);
+              ea[tt][j] = a;
+            }
+            hh[tt][j] = h[j];
+            y = fmaf(crow[j], h[j], y);
+            rb[(g * NS + j) * S::RBN + tt * S::RBS + c] = dy * h[j];  // dC partial
+          }
+          my0[tt] = y;
+        }
+      }
+      __syncthreads();
+      // (c) dC partial of this channel tile; y of the steps this lane owns
+      for (int o = tid; o < NP * kSub; o += kThreads) {
+        const int n = o / kSub, tt = o % kSub;
+        const int64_t t = tb + tt;
+        if (n < N && t < L) {
+          float s = 0.f;
+          const float *r = rb + n * S::RBN + tt * S::RBS;
+          for (int cc = 0; cc < CH; cc++) s += r[cc];
+          P.p_dC[((tile * p.Bt + b) * N + n) * L + t] = s;
+        }
+      }
+      float yfin[EPL];
+#pragma unroll
+      for (int j = 0; j < EPL; j++) {
+        const int tl = g * EPL + j;
+        float y = 0.f;
+#pragma unroll
+        for (int gg = 0; gg < G; gg++) y += yb0[c * S::YC + gg * S::YG + tl];
+        yfin[j] = fmaf(Dd, us[c * S::US + sb * kSub + tl], y);
+      }
+      __syncthreads();
+
+      // (d) adjoint backwards through the block
+#pragma unroll
+      for (int tt = kSub - 1; tt >= 0; tt--) {
+        const int t = sb * kSub + tt;
+        const float u = us[c * S::US + t], dl = dls[c * S::US + t], dy = dys[c * S::US + t];
+        const float *brow = Bs + t * S::BS + g * NS;
+        const float *crow = Cs + t * S::BS + g * NS;
+        float du = 0.f, dd = 0.f;
+#pragma unroll
+        for (int j = 0; j < NS; j++) {
+          const float anext = (tt + 1 < kSub) ? (PRECISE ? 1.f + ea[tt + 1][j] : ea[tt + 1][j]) : aN[j];
+          lam[j] = fmaf(anext, lam[j], dy * crow[j]);
+          const float em1 = PRECISE ? ea[tt][j] : ea[tt][j] - 1.0f;
+          const float bbar = em1 * brow[j] * invA[j];
+          const float lb = lam[j] * bbar;
+          du += lb;
+          rb[(g * NS + j) * S::RBN + tt * S::RBS + c] = lam[j] * u * em1 * invA[j];  // dB partial
+          const float dterm = lam[j] * fmaf(A[j], hh[tt][j], brow[j] * u);
+          dd += dterm;
+          dAl[j] = fmaf(dl, dterm, fmaf(-u, lb, dAl[j]));
+        }
+        my0[tt] = du;
+        my1[tt] = dd;
+      }
+#pragma unroll
+      for (int j = 0; j < NS; j++) aN[j] = PRECISE ? 1.f + ea[0][j] : ea[0][j];
+      __syncthreads();
+      // (e) dB partial of this channel tile
+      for (int o = tid; o < NP * kSub; o += kThreads) {
+        const int n = o / kSub, tt = o % kSub;
+        const int64_t t = tb + tt;
+        if (n < N && t < L) {
+          float s = 0.f;
+          const float *r = rb + n * S::RBN + tt * S::RBS;
+          for (int cc = 0; cc < CH; cc++) s += r[cc];
+          P.p_dB[((tile * p.Bt + b) * N + n) * L + t] = s;
+        }
+      }
+      // (f) per-element phase C for the steps this lane owns
+#pragma unroll
+      for (int j = 0; j < EPL; j++) {
+        const int tl = g * EPL + j, t = sb * kSub + tl;
+        const int64_t tg = t0 + t;
+        float du = 0.f, ddl = 0.f;
+#pragma unroll
+        for (int gg = 0; gg < G; gg++) {
+          du += yb0[c * S::YC + gg * S::YG + tl];
+          ddl += yb1[c * S::YC + gg * S::YG + tl];
+        }
+        const float u = us[c * S::US + t], dy = dys[c * S::US + t];
+        du = fmaf(Dd, dy, du);
+        const bool in = live && tg < L;
+        if (in) accD = fmaf(dy, u, accD);
+        // gate
+        if (has_z && in) {
+          const float zz = to_f32(zrow[t]);
+          const float sg = sigmoid<PRECISE>(zz);
+          const float dz = to_f32(dorow[t]) * yfin[j] * sg * fmaf(zz, 1.f - sg, 1.f);
+          if (P.dz) P.dz[(b * p.Dn + d) * L + tg] = dz;
+        }
+        // Delta -> dt
+        const float v = to_f32(dtrow[t]) + dtb;
+        const float dv = p.delta_softplus ? ddl * sigmoid<PRECISE>(v) : ddl;
+        if (in) {
+          if (P.ddt) P.ddt[(b * p.Dn + d) * L + tg] = dv;
+          accDtb += dv;
+        }
+        // u -> conv pre-activation
+        if (has_conv) {
+          float acc = cbias;
+#pragma unroll
+          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], to_f32(xrow[t - k]), acc);
+          const float sg = sigmoid<PRECISE>(acc);
+          const float dc = in ? du * sg * fmaf(acc, 1.f - sg, 1.f) : 0.f;
+          dcs[c * S::DCS + t] = dc;
+          accCb += dc;
+#pragma unroll
+          for (int k = 0; k < 4; k++) accW[k] = fmaf(dc, to_f32(xrow[t - k]), accW[k]);
+        } else if (in && P.dx) {
+          P.dx[(b * p.Dn + d) * L + tg] = du;
+        }
+      }
+      __syncthreads();
+    }
+
+    // conv backward for the stage: dx_t = sum_k w[k] dc_{t+k} (dc beyond the stage = halo)
+    if (has_conv) {
+#pragma unroll
+      for (int sb = 0; sb < kT / kSub; sb++) {
+#pragma unroll
+        for (int j = 0; j < EPL; j++) {
+          const int t = sb * kSub + g * EPL + j;
+          const int64_t tg = t0 + t;
+          float acc = 0.f;
+#pragma unroll
+          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
+          if (live && tg < L && P.dx) P.dx[(b * p.Dn + d) * L + tg] = acc;
+        }
+      }
+      __syncthreads();
+      // this stage's first 3 dc values become the halo of the stage before it
+      if (g == 0) {
+        for (int k = 0; k < 3; k++) dcs[c * S::DCS + kT + k] = dcs[c * S::DCS + k];
+      }
+      // (visible to the next stage after its top-of-loop barrier)
+    }
+  }
+
+  // per-channel parameter partials for this batch element
+  if (live) {
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+      const int n = g * NS + j;
+      if (n < N) P.p_dA_log[(b * p.Dn + d) * N + n] = dAl[j];
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < G; off <<= 1) {
+    accD += __shfl_xor_sync(0xffffffffu, accD, off);
+    accDtb += __shfl_xor_sync(0xffffffffu, accDtb, off);
+    accCb += __shfl_xor_sync(0xffffffffu, accCb, off);
+#pragma unroll
+    for (int k = 0; k < 4; k++) accW[k] += __shfl_xor_sync(0xffffffffu, accW[k], off);
+  }
+  if (live && g == 0) {
+    const int64_t bd = b * p.Dn + d;
+    P.p_dD[bd] = accD;
+    P.p_ddt_bias[bd] = accDtb;
+    P.p_dconv_b[bd] = accCb;
+    for (int k = 0; k < 4; k++) P.p_dconv_w[bd * 4 + k] = accW[k];
+  }
+}
+
+// dB/dC: add the channel-tile partials in tile order.
+__global__ void reduce_tiles_kernel(const float *__restrict__ pdB, const float *__restrict__ pdC,
+                                    float *dB, float *dC, int64_t n_tiles, int64_t per_tile) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= per_tile) return;
+  float sb = 0.f, sc = 0.f;
+  for (int64_t k = 0; k < n_tiles; k++) {
+    sb += pdB[k * per_tile + i];
+    sc += pdC[k * per_tile + i];
+  }
+  if (dB) dB[i] = sb;
+  if (dC) dC[i] = sc;
+}
+
+// per-channel parameters: add the batch partials in batch order.
+__global__ void reduce_params_kernel(const BwdParams P) {
+  const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t Dn = P.f.Dn, N = P.f.N, Bt = P.f.Bt;
+  if (d >= Dn) return;
+  float sD = 0.f, sT = 0.f, sCb = 0.f, sW[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t b = 0; b < Bt; b++) {
+    sD += P.p_dD[b * Dn + d];
+    sT += P.p_ddt_bias[b * Dn + d];
+    sCb += P.p_dconv_b[b * Dn + d];
+    for (int k = 0; k < 4; k++) sW[k] += P.p_dconv_w[(b * Dn + d) * 4 + k];
+  }
+  if (P.dD) P.dD[d] = sD;
+  if (P.ddt_bias) P.ddt_bias[d] = sT;
+  if (P.dconv_b) P.dconv_b[d] = sCb;
+  if (P.dconv_w)
+    for (int k = 0; k < P.f.K; k++) P.dconv_w[d * P.f.K + k] = sW[k];
+  if (P.dA_log)
+    for (int64_t n = 0; n < N; n++) {
+      float s = 0.f;
+      for (int64_t b = 0; b < Bt; b++) s += P.p_dA_log[(b * Dn + d) * N + n];
+      P.dA_log[d * N + n] = s;
+    }
+}
+
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states) {
+  auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const LaneLayout lay = choose_layout(N, Bt * Dn);
+  const int64_t ch = channels_per_cta(lay);
+  const int64_t n_tiles = (Dn + ch - 1) / ch;
+  const int64_t BD = Bt * Dn;
+  size_t s = 0;
+  s += rnd(sizeof(float) * BD * N);
+  s += rnd(sizeof(float) * BD);
+  s += rnd(sizeof(float) * BD);
+  s += rnd(sizeof(float) * BD * 4);
+  s += rnd(sizeof(float) * BD);
+  s += rnd(sizeof(float) * n_tiles * Bt * N * L);
+  s += rnd(sizeof(float) * n_tiles * Bt * N * L);
+  if (need_states) s += rnd(sizeof(float) * BD * ((L + kSub - 1) / kSub) * N);
+  return s;
+}
+
+template <int G, int NS, typename Tin>
+static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
+  using S = BwdSmem<G, NS, Tin>;
+  auto kern = ssm_bwd_kernel<G, NS, Tin>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = P.n_dtiles * P.f.Bt;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<(unsigned)grid, kThreads, S::bytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t bwd_dispatch(const LaneLayout &lay, const BwdParams &P, cudaStream_t s) {
+#define SSM_BWD_CASE(G_, NS_) \
+  if (lay.G == G_ && lay.NS == NS_) return launch_bwd_t<G_, NS_, Tin>(P, s);
+  SSM_BWD_CASE(4, 1) SSM_BWD_CASE(4, 2) SSM_BWD_CASE(4, 4)
+  SSM_BWD_CASE(8, 1) SSM_BWD_CASE(8, 2) SSM_BWD_CASE(8, 4)
+  SSM_BWD_CASE(16, 1) SSM_BWD_CASE(16, 2) SSM_BWD_CASE(16, 4)
+#undef SSM_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
+  cudaError_t e;
+  if (!P.chunk_states) {
+    // states were not saved by the forward: recompute them (no outputs) into the workspace
+    FwdParams f = P.f;
+    f.out = nullptr;
+    f.u_out = nullptr;
+    e = launch_fwd(f, in_bf16, 0, stream);
+    if (e != cudaSuccess) return e;
+  }
+  const LaneLayout lay = choose_layout(P.f.N, P.f.Bt * P.f.Dn);
+  e = in_bf16 ? bwd_dispatch<__nv_bfloat16>(lay, P, stream) : bwd_dispatch<float>(lay, P, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t per_tile = P.f.Bt * P.f.N * P.f.L;
+  if (P.dB || P.dC) {
+    const int64_t blocks = (per_tile + 255) / 256;
+    reduce_tiles_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P.p_dB, P.p_dC, P.dB, P.dC, P.n_dtiles, per_tile);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  reduce_params_kernel<<<(unsigned)((P.f.Dn + 127) / 128), 128, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace ssm

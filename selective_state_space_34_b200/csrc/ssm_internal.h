@@ -1,0 +1,61 @@
+// ssm_internal.h -- launch parameters and launcher declarations shared by the kernel files and
+// the C-ABI layer. Host/device plain data only; no torch types anywhere in the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssm {
+
+constexpr int kThreads = 128;  // threads per CTA for the scan kernels
+constexpr int kT = 32;         // time steps staged per CTA pipeline stage
+constexpr int kSub = 16;       // recompute / state-save block (SSM_STATE_CHUNK)
+constexpr int kPre = 8;        // conv halo prefix kept in front of each staged x row
+
+// Lane layout of the scan kernels: a channel's N states are spread over G adjacent lanes of one
+// warp, NS states per lane (G * NS >= N, padded states are inert).
+struct LaneLayout {
+  int G;
+  int NS;
+};
+
+struct FwdParams {
+  const void *x, *dt, *z, *B, *C;
+  const float *dt_bias, *A_log, *D, *conv_w, *conv_b;
+  void *out, *u_out;
+  float *chunk_states;
+  int64_t Bt, Dn, N, L, n_ck;
+  int K;
+  int delta_softplus;
+  int vec;  // 1: rows are 16-byte aligned, stage with cp.async and store with vector stores
+};
+
+struct BwdParams {
+  FwdParams f;
+  const void *dout;
+  const float *chunk_states;
+  float *dx, *ddt, *dz, *dB, *dC;
+  // per-(b, d) partial sums of the per-channel parameter gradients, reduced over b afterwards
+  float *p_dA_log;   // (Bt, Dn, N)
+  float *p_dD;       // (Bt, Dn)
+  float *p_ddt_bias; // (Bt, Dn)
+  float *p_dconv_w;  // (Bt, Dn, 4)
+  float *p_dconv_b;  // (Bt, Dn)
+  // per-channel-tile partial sums of dB / dC: (n_dtiles, Bt, N, L) each
+  float *p_dB, *p_dC;
+  int64_t n_dtiles;
+  float *dA_log, *dD, *ddt_bias, *dconv_w, *dconv_b;
+};
+
+LaneLayout choose_layout(int64_t N, int64_t channels);
+int channels_per_cta(const LaneLayout &lay);
+
+cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states);
+cudaError_t launch_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
+                               int64_t Dn, int64_t L, int K, int in_bf16, int out_bf16, int vec,
+                               cudaStream_t stream);
+
+}  // namespace ssm

@@ -1,0 +1,151 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function that
+include/ssm_scan.h declares, and the synchronous argument validation returns the documented
+status codes before anything is launched (only invalid or empty arguments are passed here, so
+no CUDA call is ever reached)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_34_b200 import _abi, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ssm_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ssm_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = _declared_functions()
+    assert {"ssm_scan_fwd", "ssm_scan_bwd", "ssm_conv1d_silu"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(n for n, _, _ in _abi.SIGNATURES) == names
+
+
+def test_struct_layout_matches_header_field_order():
+    src = open(HEADER).read()
+    body = src[src.index("typedef struct ssm_fwd_args"):src.index("} ssm_fwd_args;")]
+    fields = re.findall(r"\b(\w+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
+    flat = []
+    for line in re.sub(r"/\*.*?\*/", "", body, flags=re.S).split(";"):
+        names = re.findall(r"[\*\s](\w+)\s*(?:,|$)", line.strip() + " ")
+        if names:
+            flat.extend(re.findall(r"(\w+)\s*(?=,|$)", line.split("{")[-1].strip()))
+    ct = [f[0] for f in _abi.FwdArgs._fields_]
+    assert [f for f in flat if f in ct] == ct
+    assert ctypes.sizeof(_abi.FwdArgs) == 13 * 8 + 4 * 8 + 4 * 4
+
+
+def test_status_strings(lib):
+    for code, name in _abi.STATUS.items():
+        assert lib.ssm_status_string(code).decode().startswith(name)
+    assert lib.ssm_status_string(99) == b"unknown ssm_status"
+
+
+def test_state_chunk_count(lib):
+    assert lib.ssm_num_state_chunks(0) == 0
+    assert lib.ssm_num_state_chunks(1) == 1
+    assert lib.ssm_num_state_chunks(16) == 1
+    assert lib.ssm_num_state_chunks(17) == 2
+    assert lib.ssm_num_state_chunks(65536) == 4096
+
+
+def _args(**kw):
+    a = _abi.FwdArgs()
+    a.x, a.dt, a.A_log, a.B, a.C, a.out = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000
+    a.Bt, a.Dn, a.N, a.L, a.K = 2, 8, 4, 32, 4
+    a.in_dtype, a.out_dtype, a.delta_softplus = 0, 0, 1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _fwd(lib, a):
+    return lib.ssm_scan_fwd(ctypes.byref(a), None)
+
+
+def test_fwd_validation_codes(lib):
+    assert lib.ssm_scan_fwd(None, None) == 1
+    assert _fwd(lib, _args(x=None)) == 1
+    assert _fwd(lib, _args(out=None)) == 1
+    assert _fwd(lib, _args(in_dtype=7)) == 4
+    assert _fwd(lib, _args(out_dtype=-1)) == 4
+    assert _fwd(lib, _args(Dn=0)) == 2          # empty internal axes are rejected
+    assert _fwd(lib, _args(N=0)) == 2
+    assert _fwd(lib, _args(L=-1)) == 2
+    assert _fwd(lib, _args(Bt=-3)) == 2
+    assert _fwd(lib, _args(N=65)) == 5
+    assert _fwd(lib, _args(conv_w=0x7000, K=5)) == 5
+    assert _fwd(lib, _args(conv_w=0x7000, K=0)) == 2
+    assert _fwd(lib, _args(Bt=1 << 40, Dn=1 << 30)) == 2   # size overflow
+    assert _fwd(lib, _args(x=0x1001)) == 3      # fp32 tensor not 4-byte aligned
+    assert _fwd(lib, _args(in_dtype=1, x=0x1001)) == 3
+    assert _fwd(lib, _args(A_log=0x3002)) == 3
+    assert _fwd(lib, _args(out_dtype=1, out=0x6001)) == 3
+
+
+def test_empty_problems_are_noops(lib):
+    # L = 0 or Bt = 0: nothing to do, no pointer is touched (even NULL ones)
+    assert _fwd(lib, _args(L=0, x=None, out=None)) == 0
+    assert _fwd(lib, _args(Bt=0, x=None)) == 0
+
+
+def test_bwd_validation_codes(lib):
+    bw = _abi.BwdArgs()
+    bw.fwd = _args()
+    assert lib.ssm_scan_bwd(None, None) == 1
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 1      # dout missing
+    bw.dout = 0x8000
+    need = lib.ssm_bwd_workspace_size(ctypes.byref(bw))
+    assert need > 0
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 7      # no workspace
+    bw.workspace, bw.workspace_bytes = 0x100000, need - 1
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 7      # too small
+    bw.workspace, bw.workspace_bytes = 0x100010, need
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 7      # not 256-byte aligned
+    bw.dx = 0x9002
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 3
+    bw.dx = 0
+    bw.dout = 0x8001
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 3
+    bw.fwd = _args(L=0)
+    assert lib.ssm_bwd_workspace_size(ctypes.byref(bw)) == 0
+    assert lib.ssm_scan_bwd(ctypes.byref(bw), None) == 0
+    # saved states shrink the workspace (no recompute buffer)
+    bw.fwd = _args()
+    bw.dout = 0x8000
+    bw.chunk_states = 0
+    full = lib.ssm_bwd_workspace_size(ctypes.byref(bw))
+    bw.chunk_states = 0xA000
+    assert lib.ssm_bwd_workspace_size(ctypes.byref(bw)) < full
+
+
+def test_conv_validation_codes(lib):
+    f = lib.ssm_conv1d_silu
+    assert f(0x1000, 0x2000, 0x3000, None, 2, 4, 8, 4, 9, 0, None) == 4
+    assert f(0x1000, 0x2000, 0x3000, None, 2, 0, 8, 4, 0, 0, None) == 2
+    assert f(0x1000, 0x2000, 0x3000, None, 2, 4, 8, 0, 0, 0, None) == 2
+    assert f(0x1000, 0x2000, 0x3000, None, 2, 4, 8, 5, 0, 0, None) == 5
+    assert f(None, 0x2000, 0x3000, None, 2, 4, 8, 4, 0, 0, None) == 1
+    assert f(0x1001, 0x2000, 0x3000, None, 2, 4, 8, 4, 0, 0, None) == 3
+    assert f(None, None, None, None, 2, 4, 0, 4, 0, 0, None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import selective_state_space_34_b200 as ssm
+    x = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        ssm.ssm_scan_fwd(x, x, torch.zeros(2, 4), torch.zeros(1, 4, 8), torch.zeros(1, 4, 8))
