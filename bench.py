@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the fused selective scan (Mamba-1 S6) on B200: one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic input: the fused forward
+(conv1d + SiLU -> softplus Delta -> exact-ZOH scan -> D skip -> SiLU(z) gate, saving the chunk
+states) followed by the backward (all gradients), on the 4 x 4096 x 16 x 4096 Mamba-1.4B-shaped
+workload with bf16 activations, fp32 state and fp32 gradients. The forward alone on the same shape
+(the HBM-headline case) is timed in the same run and reported under "forward".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (launched with torch.distributed.run): every rank runs its own batch (weak scaling);
+the data path has no collective. Timing is on the device (CUDA events), max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("selective-scan fwd/bwd (batch·d_inner·L·d_state)/s and HBM GB/s vs peak, "
+          "1×B200")
+UNIT = "elem_states/s"
+# Measured on this machine's B200s (copy bandwidth, bf16 GEMM); used when the per-pod file is absent.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+# sm_100a pipe rates per SM per clock (FP32 FMA lanes, MUFU ex2), used for the ALU ceiling.
+FMA_LANES, MUFU_LANES, N_SM = 128, 16, 148
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+# ---- algorithmic bytes (the minimum the method must move; intermediates never touch HBM) -------
+
+def fwd_bytes(Bt, Dn, N, L, s_in, s_out, states=False):
+    elems = Bt * Dn * L
+    b = elems * (3 * s_in + s_out)              # x, dt, z in; out
+    b += Bt * N * L * 2 * s_in                  # B, C (shared by all channels)
+    b += Dn * (N + 4 + 4) * 4                   # A_log, D, dt_bias, conv taps + bias
+    if states:
+        b += Bt * Dn * ((L + 15) // 16) * N * 4  # chunk states for the backward
+    return b
+
+
+def bwd_bytes(Bt, Dn, N, L, s_in, states=True):
+    elems = Bt * Dn * L
+    b = elems * (4 * s_in + 3 * 4)              # x, dt, z, dout in; dx, ddt, dz out (fp32)
+    b += Bt * N * L * (2 * s_in + 2 * 4)        # B, C in; dB, dC out (fp32)
+    b += Dn * (N + 8) * 4 * 2                   # parameters in, parameter grads out
+    if states:
+        b += Bt * Dn * ((L + 15) // 16) * N * 4
+    return b
+
+
+# ---- clocks during the timed region -------------------------------------------------------------
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- CPU baseline: the float64 oracle on a bounded sample of the same workload ------------------
+
+def oracle_sample(w, a, n_channels, threads):
+    """Run the oracle's forward + backward on n_channels channels of the workload, spread over a
+    thread pool (the C oracle releases the GIL); returns (seconds, elem_states)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    per = max(1, min(16, n_channels // max(1, threads)))
+    picks = [(i // w.Dn % w.Bt, i % w.Dn) for i in range(n_channels)]
+    groups = [picks[i:i + per] for i in range(0, len(picks), per)]
+
+    def run(group):
+        b = group[0][0]
+        ds = [d for bb, d in group if bb == b]
+        sl = slice(ds[0], ds[-1] + 1)
+        kw = dict(D=a["D"][sl], z=None if a["z"] is None else a["z"][b:b + 1, sl],
+                  dt_bias=a["dt_bias"][sl], conv_w=None if a["conv_w"] is None else a["conv_w"][sl],
+                  conv_b=None if a["conv_b"] is None else a["conv_b"][sl])
+        x, dt = a["x"][b:b + 1, sl], a["dt"][b:b + 1, sl]
+        B, C, Al = a["B"][b:b + 1], a["C"][b:b + 1], a["A_log"][sl]
+        oracle.fwd(x, dt, Al, B, C, n_threads=1, **kw)
+        if w.backward:
+            oracle.bwd(x, dt, Al, B, C, a["dout"][b:b + 1, sl], n_threads=1, **kw)
+        return len(ds) * w.L * w.N
+
+    oracle.build()
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        done = sum(ex.map(run, groups))
+    return time.perf_counter() - t0, done
+
+
+def reference_arm(args, w):
+    """--impl reference: the float64 oracle timed on the host cores, on bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from selective_state_space_34_b200 import workloads as wl
+    a = wl.generate(w)
+    threads = os.cpu_count() or 1
+    n_ch = max(threads * 4, 64)
+    times, work = [], 0
+    for i in range(args.warmup + args.steps):
+        dt_s, es = oracle_sample(w, a, n_ch, threads)
+        if i >= args.warmup:
+            times.append(dt_s)
+            work += es
+    total = sum(times)
+    value = work / total
+    sample = "%d channels x L=%d x N=%d per step (fwd%s), float64, %d host threads" % (
+        n_ch, w.L, w.N, "+bwd" if w.backward else "", threads)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "Bt": w.Bt, "Dn": w.Dn, "N": w.N, "L": w.L,
+                   "in_dtype": w.in_dtype, "sampled": True},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- our arm ----------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mamba1p4b_fwdbwd")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    from selective_state_space_34_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import selective_state_space_34_b200 as ssm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # each rank draws its own batch (weak scaling)
+    a = wl.generate(w, seed=w.seed + rank)
+    act = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    odt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+
+    def todev(k, dtype):
+        return None if a.get(k) is None else torch.from_numpy(a[k]).to(dev, dtype)
+    T = {k: todev(k, act) for k in ("x", "dt", "z", "B", "C", "dout")}
+    T.update({k: todev(k, torch.float32) for k in ("A_log", "D", "dt_bias", "conv_w", "conv_b")})
+    kw = dict(D=T["D"], z=T["z"], dt_bias=T["dt_bias"], conv_w=T["conv_w"], conv_b=T["conv_b"])
+    Bt, Dn, N, L = w.Bt, w.Dn, w.N, w.L
+    s_in = 2 if act == torch.bfloat16 else 4
+    s_out = 2 if odt == torch.bfloat16 else 4
+    es = w.elem_states
+    backward = w.backward
+
+    out = torch.empty((Bt, Dn, L), dtype=odt, device=dev)
+    states = torch.empty((Bt, Dn, ssm.ssm_num_state_chunks(L), N), dtype=torch.float32, device=dev)
+    grads = None
+    ws = None
+    need = 0
+    if backward:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = {"dx": torch.empty((Bt, Dn, L), **f32), "ddt": torch.empty((Bt, Dn, L), **f32),
+                 "dz": torch.empty((Bt, Dn, L), **f32), "dA_log": torch.empty((Dn, N), **f32),
+                 "dB": torch.empty((Bt, N, L), **f32), "dC": torch.empty((Bt, N, L), **f32),
+                 "dD": torch.empty((Dn,), **f32), "ddt_bias": torch.empty((Dn,), **f32),
+                 "dconv_w": torch.empty(tuple(T["conv_w"].shape), **f32),
+                 "dconv_b": torch.empty((Dn,), **f32)}
+        need = ssm.ssm_bwd_workspace_size(T["dout"], T["x"], T["dt"], T["A_log"], T["B"], T["C"],
+                                          chunk_states=states, **kw)
+        ws = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+
+    import ctypes
+    from selective_state_space_34_b200 import _abi, api
+    lib = _abi.load()
+    s = torch.cuda.current_stream(dev)
+
+    # argument structs built once; each step is then plain C-ABI calls on the current stream
+    fwd_args, _ = api._fwd_args(T["x"], T["dt"], T["A_log"], T["B"], T["C"], kw["D"], kw["z"],
+                                kw["dt_bias"], kw["conv_w"], kw["conv_b"], True, odt)
+    fwd_args.out = out.data_ptr()
+    fwd_args.chunk_states = states.data_ptr() if backward else None
+    fwd_args_fo = _abi.FwdArgs.from_buffer_copy(fwd_args)
+    fwd_args_fo.chunk_states = None
+    if backward:
+        bw_args = api._bwd_struct(T["dout"], T["x"], T["dt"], T["A_log"], T["B"], T["C"], kw["D"],
+                                  kw["z"], kw["dt_bias"], kw["conv_w"], kw["conv_b"], True, states)
+        for k, v in grads.items():
+            setattr(bw_args, k, v.data_ptr())
+        bw_args.workspace = (ws.data_ptr() + 255) & ~255
+        bw_args.workspace_bytes = need
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    n_rec = args.steps
+    ev_f0 = [E() for _ in range(n_rec)]
+    ev_f1 = [E() for _ in range(n_rec)]
+    ev_b = [[E(), E()] for _ in range(n_rec)] if backward else None
+    ev_b1 = [E() for _ in range(n_rec)] if backward else None
+    ev_ptr = []
+    for evs in (ev_b or []):
+        for e in evs:
+            e.record(s)  # creates the underlying cudaEvent_t handles before they are passed down
+        ev_ptr.append((ctypes.c_void_p * 2)(evs[0].cuda_event, evs[1].cuda_event))
+    torch.cuda.synchronize()
+
+    def step(i=None, timed=False):
+        if timed:
+            ev_f0[i].record(s)
+        _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(fwd_args), s.cuda_stream))
+        if timed:
+            ev_f1[i].record(s)
+        if backward:
+            bw_args.timing_events = ctypes.cast(ev_ptr[i], ctypes.c_void_p) if timed else None
+            _abi.check("ssm_scan_bwd", lib.ssm_scan_bwd(ctypes.byref(bw_args), s.cuda_stream))
+            if timed:
+                ev_b1[i].record(s)
+
+    def fwd_only():
+        _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(fwd_args_fo), s.cuda_stream))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # ---- device-resident timing of K steps ----
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = E(), E()
+    t_start.record(s)
+    for i in range(args.steps):
+        step(i, timed=True)
+    t_end.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(el, op=dist.ReduceOp.MAX)
+    max_ms = float(el.item())
+    ms_step = max_ms / args.steps
+    value = es * world * args.steps / (max_ms * 1e-3)
+
+    fwd_ms = float(np.mean([ev_f0[i].elapsed_time(ev_f1[i]) for i in range(args.steps)]))
+    kern = {"ssm_fwd_kernel": fwd_ms}
+    if backward:
+        kern["ssm_bwd_kernel"] = float(np.mean([ev_b[i][0].elapsed_time(ev_b[i][1]) for i in range(args.steps)]))
+        kern["bwd_reductions"] = float(np.mean([ev_b[i][1].elapsed_time(ev_b1[i]) for i in range(args.steps)]))
+
+    # ---- forward alone on the same shape (no state saving): the HBM-headline case ----
+    for _ in range(3):
+        fwd_only()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = E(), E()
+    nf = max(args.steps, 20)
+    f0.record(s)
+    for _ in range(nf):
+        fwd_only()
+    f1.record(s)
+    torch.cuda.synchronize()
+    fo_ms = f0.elapsed_time(f1) / nf
+    fo = torch.tensor([fo_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(fo, op=dist.ReduceOp.MAX)
+    fo_ms = float(fo.item())
+
+    peaks = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fb = fwd_bytes(Bt, Dn, N, L, s_in, s_out, states=False)
+    fwd_roof = {"bound": "hbm", "achieved": fb / (fo_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": fb / (fo_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+                "algorithmic_bytes": fb, "kernel": "ssm_fwd_kernel", "ms": fo_ms,
+                "peak_source": peaks.get("source")}
+    sm_hz = (clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    mufu_peak = MUFU_LANES * N_SM * sm_hz  # ex2 per second at the sampled clock
+    forward = {"ms": fo_ms, "value": es * world / (fo_ms * 1e-3), "unit": UNIT,
+               "out_dtype": args.out_dtype, "roofline": fwd_roof,
+               "alu": {"exp2_per_s": es / (fo_ms * 1e-3), "mufu_peak_per_s": mufu_peak,
+                       "frac_of_one_mufu_exp_per_elem_state": es / (fo_ms * 1e-3) / mufu_peak}}
+
+    if backward:
+        bms = kern["ssm_bwd_kernel"]
+        bb = bwd_bytes(Bt, Dn, N, L, s_in, states=True)
+        roof = {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": bb / (bms * 1e-3) / 1e9 / hbm, "traffic": None, "algorithmic_bytes": bb,
+                "kernel": "ssm_bwd_kernel", "ms": bms, "peak_source": peaks.get("source")}
+    else:
+        roof = dict(fwd_roof)
+    launches_per_step = 1 + (3 if backward else 0)
+
+    # ---- end to end through the C ABI with host buffers: H2D inputs, compute, D2H results ----
+    names_in = ["x", "dt", "z", "B", "C"] + (["dout"] if backward else [])
+    host = {k: torch.empty(T[k].shape, dtype=T[k].dtype, pin_memory=True) for k in names_in}
+    for k in names_in:
+        host[k].copy_(T[k].cpu())
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names_in)
+    res_names = ["dA_log", "dB", "dC", "dD", "ddt_bias", "dconv_w", "dconv_b"] if backward else []
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    host_res = {k: torch.empty(grads[k].shape, dtype=torch.float32, pin_memory=True) for k in res_names}
+    d2h = host_out.numel() * host_out.element_size() + sum(v.numel() * 4 for v in host_res.values())
+
+    def e2e_step():
+        for k in names_in:
+            T[k].copy_(host[k], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        for k in res_names:
+            host_res[k].copy_(grads[k], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = E(), E()
+    e0.record(s)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(et, op=dist.ReduceOp.MAX)
+    e2e = {"value": es * world * args.e2e_steps / (float(et.item()) * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": float(et.item()) / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        n_ch = min(w.Bt * w.Dn, 256 * threads)
+        secs, done = oracle_sample(w, a, n_ch, threads)
+        cpu = {"value": done / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "%d channels x L=%d x N=%d (fwd%s) of the same workload, float64, %.1f s"
+                         % (n_ch, L, N, "+bwd" if backward else "", secs)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "Bt": Bt, "Dn": Dn, "N": N, "L": L,
+                       "in_dtype": w.in_dtype, "out_dtype": args.out_dtype,
+                       "step": "fwd(save states)+bwd" if backward else "fwd",
+                       "l2": "inputs larger than L2 (per-step working set %.2f GB)"
+                             % ((fwd_bytes(Bt, Dn, N, L, s_in, s_out, backward)
+                                 + (bwd_bytes(Bt, Dn, N, L, s_in) if backward else 0)) / 1e9),
+                       "parallelism": "replica per GPU" if world > 1 else "single GPU"},
+            "roofline": roof,
+            "kernels_ms": kern,
+            "forward": forward,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -133,6 +133,10 @@ typedef struct ssm_bwd_args {
   void *workspace;          /* device scratch of at least ssm_bwd_workspace_size() bytes,
                                256-byte aligned; contents need not be initialised */
   size_t workspace_bytes;
+  void *const *timing_events; /* NULL, or 2 caller-created cudaEvent_t: [0] is recorded on
+                                 `stream` just before the main backward kernel, [1] just after it
+                                 (before the cross-tile reductions); lets a caller time the
+                                 kernel alone. Recording does not synchronise. */
 } ssm_bwd_args;
 
 /* Bytes of device scratch ssm_scan_bwd needs for these arguments (0 for an empty problem). */

@@ -37,7 +37,7 @@ class BwdArgs(ctypes.Structure):
         ("dA_log", ctypes.c_void_p), ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p),
         ("dD", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p), ("dconv_w", ctypes.c_void_p),
         ("dconv_b", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("workspace_bytes", ctypes.c_size_t), ("timing_events", ctypes.c_void_p),
     ]
 
 

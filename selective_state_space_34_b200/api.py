@@ -138,10 +138,13 @@ def ssm_bwd_workspace_size(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=Non
 
 def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None,
                  conv_b=None, delta_softplus: bool = True, chunk_states=None,
-                 workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None):
+                 workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None,
+                 timing_events=None):
     """Backward. Returns a dict of fp32 gradients: dx, ddt, dA_log, dB, dC, and dD / ddt_bias /
     dz / dconv_w / dconv_b where the corresponding input exists. ``workspace`` (uint8, at least
-    ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call."""
+    ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call.
+    ``timing_events``: optional pair of recorded-once torch.cuda.Event(enable_timing=True); the
+    library records them just before and just after its main backward kernel."""
     bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
                      chunk_states)
     Bt, Dn, L = x.shape
@@ -177,6 +180,10 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
             aligned = (base + 255) & ~255
         bw.workspace = aligned
         bw.workspace_bytes = need
+    ev_arr = None
+    if timing_events is not None:
+        ev_arr = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in timing_events])
+        bw.timing_events = ctypes.cast(ev_arr, ctypes.c_void_p)
     _abi.check("ssm_scan_bwd", lib.ssm_scan_bwd(ctypes.byref(bw), _stream_handle(dev)))
     return grads
 

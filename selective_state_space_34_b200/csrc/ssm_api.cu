@@ -192,6 +192,7 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   p.ddt_bias = args->ddt_bias;
   p.dconv_w = a->conv_w ? args->dconv_w : nullptr;
   p.dconv_b = a->conv_w ? args->dconv_b : nullptr;
+  p.timing_events = args->timing_events;
   // carve the workspace (layout mirrored by ssm::bwd_workspace_bytes)
   char *ws = static_cast<char *>(args->workspace);
   auto take = [&](size_t bytes) {

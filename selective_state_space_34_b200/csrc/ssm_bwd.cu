@@ -521,8 +521,16 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   const LaneLayout lay = choose_layout(P.f.N, P.f.Bt * P.f.Dn);
+  if (P.timing_events && P.timing_events[0]) {
+    e = cudaEventRecord(static_cast<cudaEvent_t>(P.timing_events[0]), stream);
+    if (e != cudaSuccess) return e;
+  }
   e = in_bf16 ? bwd_dispatch<__nv_bfloat16>(lay, P, stream) : bwd_dispatch<float>(lay, P, stream);
   if (e != cudaSuccess) return e;
+  if (P.timing_events && P.timing_events[1]) {
+    e = cudaEventRecord(static_cast<cudaEvent_t>(P.timing_events[1]), stream);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t per_tile = P.f.Bt * P.f.N * P.f.L;
   if (P.dB || P.dC) {
     const int64_t blocks = (per_tile + 255) / 256;

@@ -76,6 +76,19 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src));
 }
+// Same, asking L2 to fetch the surrounding 256 bytes: rows are streamed in short slices per stage,
+// so the next stages of the same row then hit in L2 instead of reopening a DRAM page.
+__device__ __forceinline__ void cp_async16_l2pf(void *smem_dst, const void *gmem_src) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src));
+}
+// 16-byte global load with the same L2 256-byte prefetch hint (read-only data).
+__device__ __forceinline__ uint4 ld_global_l2pf(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N> __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));

@@ -34,7 +34,7 @@ __device__ __forceinline__ void stage_rows(T *dst, int dst_stride, const T *src,
       const int64_t t = t0 + (int64_t)v * EPV;
       T *d = dst + r * dst_stride + v * EPV;
       if (r < rows_valid && t < L)
-        cp_async16(d, src + (int64_t)r * src_stride + t);
+        cp_async16_l2pf(d, src + (int64_t)r * src_stride + t);
       else
         *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -89,31 +89,127 @@ __device__ __forceinline__ void store_run(T *row, int64_t t, int64_t L, const fl
   }
 }
 
+// n consecutive activations from shared memory as fp32, read with the widest aligned vectors
+// (the callers' offsets are multiples of 4 elements, so 8-byte loads for bf16, 16-byte for fp32).
+template <typename T, int NE> __device__ __forceinline__ void load_window(float *dst, const T *src) {
+  if (sizeof(T) == 2 && NE % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NE; i += 4) {
+      const uint2 v = *reinterpret_cast<const uint2 *>(src + i);
+      const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&v.x);
+      const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&v.y);
+      dst[i] = __low2float(lo);
+      dst[i + 1] = __high2float(lo);
+      dst[i + 2] = __low2float(hi);
+      dst[i + 3] = __high2float(hi);
+    }
+  } else if (sizeof(T) == 4 && NE % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NE; i += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + i);
+      dst[i] = v.x;
+      dst[i + 1] = v.y;
+      dst[i + 2] = v.z;
+      dst[i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < NE; i++) dst[i] = to_f32(src[i]);
+  }
+}
+template <int NE> __device__ __forceinline__ void load_floats(float *dst, const float *src) {
+  if (NE % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NE; i += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + i);
+      dst[i] = v.x;
+      dst[i + 1] = v.y;
+      dst[i + 2] = v.z;
+      dst[i + 3] = v.w;
+    }
+  } else if (NE % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < NE; i += 2) {
+      const float2 v = *reinterpret_cast<const float2 *>(src + i);
+      dst[i] = v.x;
+      dst[i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < NE; i++) dst[i] = src[i];
+  }
+}
+template <int NS> __device__ __forceinline__ void load_states(float *dst, const float *src) {
+  load_floats<NS>(dst, src);
+}
+
 // Shared-memory plan of one CTA (all offsets in bytes, 16-byte aligned).
 template <int G, int NS, typename Tin> struct FwdSmem {
   static constexpr int CH = kThreads / G;    // channels per CTA
   static constexpr int NP = G * NS;          // padded state count
   static constexpr int XS = kPre + kT;       // x row length (elements)
   static constexpr int BS = NP + 4;          // Bs/Cs row stride (floats)
-  static constexpr int US = kT + 4;          // us/dls/ss row stride (floats)
-  static constexpr int YG = kSub + 8;        // y-partial stride between lanes of a channel
+  static constexpr int US = kSub + 2;        // ud row stride (float2 entries: dl, u)
+  static constexpr int YG = kSub + 4;        // y-partial stride between lanes of a channel
   static constexpr int YC = G * YG + 4;      // y-partial stride between channels
   static constexpr size_t x_off = 0;
   static constexpr size_t dt_off = x_off + sizeof(Tin) * 2 * CH * XS;
   static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t braw_off = z_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t craw_off = braw_off + sizeof(Tin) * 2 * NP * kT;
-  static constexpr size_t bs_off = craw_off + sizeof(Tin) * 2 * NP * kT;
-  static constexpr size_t cs_off = bs_off + sizeof(float) * kT * BS;
-  static constexpr size_t us_off = cs_off + sizeof(float) * kT * BS;
-  static constexpr size_t dls_off = us_off + sizeof(float) * CH * US;
-  static constexpr size_t ss_off = dls_off + sizeof(float) * CH * US;
-  static constexpr size_t yp_off = ss_off + sizeof(float) * CH * US;
+  static constexpr size_t bs_off = z_off + sizeof(Tin) * 2 * CH * kT;
+  static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * kT * BS;
+  static constexpr size_t ud_off = cs_off + sizeof(float) * 2 * kT * BS;
+  static constexpr size_t yp_off = ud_off + sizeof(float2) * CH * US;
   static constexpr size_t bytes = yp_off + sizeof(float) * CH * YC;
 };
 
+// B and C of one stage (NP rows x kT steps, row stride L in global memory) go global ->
+// registers -> transposed fp32 rows [t][n] in shared memory, so that the scan reads all of a
+// lane's states at one step with one 16-byte broadcast load. Loads for stage s+1 are issued one
+// stage early into registers; the transposed stores happen after the next barrier-free point.
+template <typename Tin, int NP> struct BCStager {
+  static constexpr int EPV = 16 / sizeof(Tin);               // elements per 16-byte vector
+  static constexpr int VPR = kT / EPV;                       // vectors per row
+  static constexpr int NV = 2 * NP * VPR;                    // B and C vectors per stage
+  static constexpr int PER = (NV + kThreads - 1) / kThreads; // per thread
+  uint4 v[PER];
+
+  __device__ __forceinline__ void load(const Tin *gB, const Tin *gC, int n_rows, int64_t t0,
+                                       int64_t L, bool vec) {
+#pragma unroll
+    for (int k = 0; k < PER; k++) {
+      const int i = threadIdx.x + k * kThreads;
+      v[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (i >= NV) continue;
+      const int which = i / (NP * VPR), r = (i / VPR) % NP, q = i % VPR;
+      const Tin *src = (which ? gC : gB) + (int64_t)r * L;
+      const int64_t t = t0 + (int64_t)q * EPV;
+      if (r >= n_rows) continue;
+      if (vec) {
+        if (t < L) v[k] = ld_global_l2pf(src + t);
+      } else {
+        Tin tmp[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; e++) tmp[e] = (t + e < L) ? src[t + e] : from_f32<Tin>(0.0f);
+        v[k] = *reinterpret_cast<const uint4 *>(tmp);
+      }
+    }
+  }
+  __device__ __forceinline__ void store(float *Bs, float *Cs, int BS) const {
+#pragma unroll
+    for (int k = 0; k < PER; k++) {
+      const int i = threadIdx.x + k * kThreads;
+      if (i >= NV) continue;
+      const int which = i / (NP * VPR), r = (i / VPR) % NP, q = i % VPR;
+      float *dst = (which ? Cs : Bs) + (q * EPV) * BS + r;
+      const Tin *e = reinterpret_cast<const Tin *>(&v[k]);
+#pragma unroll
+      for (int j = 0; j < EPV; j++) dst[j * BS] = to_f32(e[j]);
+    }
+  }
+};
+
 template <int G, int NS, typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 ssm_fwd_kernel(const FwdParams p) {
   using S = FwdSmem<G, NS, Tin>;
   constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G;
@@ -122,13 +218,9 @@ ssm_fwd_kernel(const FwdParams p) {
   Tin *xs = reinterpret_cast<Tin *>(smem + S::x_off);
   Tin *dts = reinterpret_cast<Tin *>(smem + S::dt_off);
   Tin *zs = reinterpret_cast<Tin *>(smem + S::z_off);
-  Tin *braw = reinterpret_cast<Tin *>(smem + S::braw_off);
-  Tin *craw = reinterpret_cast<Tin *>(smem + S::craw_off);
   float *Bs = reinterpret_cast<float *>(smem + S::bs_off);
   float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
-  float *us = reinterpret_cast<float *>(smem + S::us_off);
-  float *dls = reinterpret_cast<float *>(smem + S::dls_off);
-  float *ss = reinterpret_cast<float *>(smem + S::ss_off);
+  float2 *ud = reinterpret_cast<float2 *>(smem + S::ud_off);
   float *yp = reinterpret_cast<float *>(smem + S::yp_off);
 
   const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
@@ -142,8 +234,9 @@ ssm_fwd_kernel(const FwdParams p) {
   const bool vec = p.vec != 0;
   const int64_t L = p.L, N = p.N;
 
-  // per-lane constants
-  float Acoef[NS], invA[NS], h[NS];
+  // per-lane constants: Acoef = A (precise) or A log2(e) (fast), nIA = -1/A; padded states are
+  // inert (A_bar = 1, no input, no readout)
+  float Acoef[NS], nIA[NS], h[NS];
 #pragma unroll
   for (int j = 0; j < NS; j++) {
     const int n = g * NS + j;
@@ -151,17 +244,19 @@ ssm_fwd_kernel(const FwdParams p) {
     if (live && n < N) {
       const float A = -expf(p.A_log[d * N + n]);
       Acoef[j] = PRECISE ? A : A * kLog2e;
-      invA[j] = 1.0f / A;
+      nIA[j] = -1.0f / A;
     } else {
       Acoef[j] = 0.0f;
-      invA[j] = 0.0f;
+      nIA[j] = 0.0f;
     }
   }
   float w4[4] = {0.f, 0.f, 0.f, 0.f};
   float cbias = 0.f, Dd = 0.f, dtb = 0.f;
   if (live) {
     if (has_conv) {
-      for (int k = 0; k < p.K; k++) w4[k] = p.conv_w[d * p.K + k];
+#pragma unroll
+      for (int k = 0; k < 4; k++)
+        if (k < p.K) w4[k] = p.conv_w[d * p.K + k];
       cbias = p.conv_b ? p.conv_b[d] : 0.f;
     }
     Dd = p.D ? p.D[d] : 0.f;
@@ -188,114 +283,166 @@ ssm_fwd_kernel(const FwdParams p) {
     stage_rows<Tin, CH>(xs + buf * CH * S::XS + kPre, S::XS, gx, L, rows_valid, t0, L, vec);
     stage_rows<Tin, CH>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
     if (has_z) stage_rows<Tin, CH>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
-    stage_rows<Tin, NP>(braw + buf * NP * kT, kT, gB, L, n_rows, t0, L, vec);
-    stage_rows<Tin, NP>(craw + buf * NP * kT, kT, gC, L, n_rows, t0, L, vec);
     cp_async_commit();
   };
 
-  if (n_stages > 0) issue(0, 0);
+  BCStager<Tin, NP> bc;
+  if (n_stages > 0) {
+    issue(0, 0);
+    bc.load(gB, gC, n_rows, 0, L, vec);
+    bc.store(Bs, Cs, S::BS);
+    if (n_stages > 1) bc.load(gB, gC, n_rows, kT, L, vec);
+  }
   for (int64_t st = 0; st < n_stages; st++) {
     const int buf = (int)(st & 1), nbuf = buf ^ 1;
     const int64_t t0 = st * kT;
     cp_async_wait<0>();
-    __syncthreads();  // stage st landed; everyone is done with stage st-1's buffers
-    if (st + 1 < n_stages) issue(st + 1, nbuf);
-
-    // B, C: raw (n, t) tile -> fp32 (t, n) rows for broadcast reads
-    for (int i = tid; i < NP * kT; i += kThreads) {
-      const int n = i / kT, t = i % kT;
-      Bs[t * S::BS + n] = to_f32(braw[buf * NP * kT + i]);
-      Cs[t * S::BS + n] = to_f32(craw[buf * NP * kT + i]);
+    __syncthreads();  // stage st landed and Bs/Cs[buf] written; stage st-1's buffers are free
+    if (st + 1 < n_stages) {
+      issue(st + 1, nbuf);
+      bc.store(Bs + nbuf * kT * S::BS, Cs + nbuf * kT * S::BS, S::BS);
+      if (st + 2 < n_stages) bc.load(gB, gC, n_rows, (st + 2) * kT, L, vec);
     }
-
-    // per-element phase: lane g of channel c owns EPL consecutive steps of every sub-block
+    const float *Bst = Bs + buf * kT * S::BS;
+    const float *Cst = Cs + buf * kT * S::BS;
     const Tin *xrow = xs + (buf * CH + c) * S::XS + kPre;
     const Tin *dtrow = dts + (buf * CH + c) * kT;
     const Tin *zrow = zs + (buf * CH + c) * kT;
+
 #pragma unroll
     for (int sb = 0; sb < kT / kSub; sb++) {
-      float uo[EPL];
+      // -- per-element work of this block: lane g owns EPL consecutive steps of its channel.
+      //    Its inputs (x over [t-3, t+EPL), dt, z) are read as one small vector each.
+      const int tb = sb * kSub + g * EPL;  // first owned step (stage-local)
+      float xw[EPL + 4], dtw[EPL], zw[EPL];
+      load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+      load_window<Tin, EPL>(dtw, dtrow + tb);
+      if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
+      float gate[EPL], uown[EPL];
 #pragma unroll
       for (int j = 0; j < EPL; j++) {
-        const int t = sb * kSub + g * EPL + j;
+        const int t = tb + j;
         float u;
         if (has_conv) {
           float acc = cbias;
 #pragma unroll
-          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], to_f32(xrow[t - k]), acc);
+          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
           u = acc * sigmoid<PRECISE>(acc);
         } else {
-          u = to_f32(xrow[t]);
+          u = xw[j + 4];
         }
-        const float v = to_f32(dtrow[t]) + dtb;
+        const float v = dtw[j] + dtb;
         float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
         float s = 1.0f;
-        if (has_z) {
-          const float zz = to_f32(zrow[t]);
-          s = zz * sigmoid<PRECISE>(zz);
-        }
+        if (has_z) s = zw[j] * sigmoid<PRECISE>(zw[j]);
         if (t0 + t >= L) {  // padded tail: an identity step
           u = 0.0f;
           dl = 0.0f;
         }
-        us[c * S::US + t] = u;
-        dls[c * S::US + t] = dl;
-        ss[c * S::US + t] = s;
-        uo[j] = u;
+        ud[c * S::US + g * EPL + j] = make_float2(dl, u);
+        gate[j] = s;
+        uown[j] = u;
         if (t >= kT - 3)  // carry the conv halo into the next stage's prefix
           xs[(nbuf * CH + c) * S::XS + kPre + t - kT] = xrow[t];
       }
       if (p.u_out && live)
         store_run<Tout, EPL>(static_cast<Tout *>(p.u_out) + row0 + (int64_t)c * L,
-                             t0 + sb * kSub + g * EPL, L, uo, vec);
-    }
-    __syncthreads();  // Bs/Cs complete (written by all threads); us/dls/ss visible
+                             t0 + tb, L, uown, vec);
+      __syncwarp();
 
-    // scan phase
-#pragma unroll
-    for (int sb = 0; sb < kT / kSub; sb++) {
-      float ypart[kSub];
-#pragma unroll
-      for (int tt = 0; tt < kSub; tt++) {
-        const int t = sb * kSub + tt;
-        const float u = us[c * S::US + t];
-        const float dl = dls[c * S::US + t];
-        const float *brow = Bs + t * S::BS + g * NS;
-        const float *crow = Cs + t * S::BS + g * NS;
-        float y = 0.0f;
-#pragma unroll
-        for (int j = 0; j < NS; j++) {
-          const float w = brow[j] * u * invA[j];  // B u / A
-          if (PRECISE) {
-            const float em1 = expm1f(dl * Acoef[j]);  // A_bar - 1
-            h[j] = fmaf(em1, h[j] + w, h[j]);         // A_bar h + (A_bar - 1) B u / A
-          } else {
-            const float a = ex2_approx(dl * Acoef[j]);  // A_bar
-            h[j] = fmaf(a, h[j] + w, -w);
-          }
-          y = fmaf(crow[j], h[j], y);
-        }
-        ypart[tt] = y;
-      }
-      // combine the G partial readouts of each step
+      // -- the recurrence over the block's kSub steps, in groups of 4 steps: all shared-memory
+      //    reads of a group are issued together, then the group's exps, then its updates.
       float *myp = yp + c * S::YC + g * S::YG;
 #pragma unroll
-      for (int tt = 0; tt < kSub; tt += 4)
-        *reinterpret_cast<float4 *>(myp + tt) = make_float4(ypart[tt], ypart[tt + 1], ypart[tt + 2], ypart[tt + 3]);
+      for (int tq = 0; tq < kSub; tq += 4) {
+        float dlq[4], uq[4], Bq[4][NS], Cq[4][NS];
+#pragma unroll
+        for (int tt = 0; tt < 4; tt++) {
+          const int t = sb * kSub + tq + tt;
+          const float2 du = ud[c * S::US + tq + tt];
+          dlq[tt] = du.x;
+          uq[tt] = du.y;
+          load_states<NS>(Bq[tt], Bst + t * S::BS + g * NS);
+          load_states<NS>(Cq[tt], Cst + t * S::BS + g * NS);
+        }
+        float yq[4];
+        if (PRECISE) {
+#pragma unroll
+          for (int tt = 0; tt < 4; tt++) {
+            float y = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NS; j++) {
+              const float nw = Bq[tt][j] * uq[tt] * nIA[j];   // -B u / A
+              const float em1 = expm1f(dlq[tt] * Acoef[j]);    // A_bar - 1
+              h[j] = fmaf(em1, h[j] - nw, h[j]);               // A_bar h + (A_bar - 1) B u / A
+              y = fmaf(Cq[tt][j], h[j], y);
+            }
+            yq[tt] = y;
+          }
+        } else {
+          float a[4][NS];
+#pragma unroll
+          for (int tt = 0; tt < 4; tt++) {
+            if (NS % 2 == 0) {
+#pragma unroll
+              for (int j = 0; j < NS; j += 2) {
+                const float2 x = __fmul2_rn(make_float2(dlq[tt], dlq[tt]), make_float2(Acoef[j], Acoef[j + 1]));
+                a[tt][j] = ex2_approx(x.x);
+                a[tt][j + 1] = ex2_approx(x.y);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < NS; j++) a[tt][j] = ex2_approx(dlq[tt] * Acoef[j]);
+            }
+          }
+#pragma unroll
+          for (int tt = 0; tt < 4; tt++) {
+            if (NS % 2 == 0) {
+              float2 y2 = make_float2(0.0f, 0.0f);
+              const float2 u2 = make_float2(uq[tt], uq[tt]);
+#pragma unroll
+              for (int j = 0; j < NS; j += 2) {
+                const float2 nw = __fmul2_rn(__fmul2_rn(make_float2(Bq[tt][j], Bq[tt][j + 1]), u2),
+                                             make_float2(nIA[j], nIA[j + 1]));  // -B u / A
+                float2 hh = make_float2(h[j], h[j + 1]);
+                const float2 sum = __ffma2_rn(nw, make_float2(-1.0f, -1.0f), hh);  // h + w
+                hh = __ffma2_rn(make_float2(a[tt][j], a[tt][j + 1]), sum, nw);     // a (h+w) - w
+                h[j] = hh.x;
+                h[j + 1] = hh.y;
+                y2 = __ffma2_rn(make_float2(Cq[tt][j], Cq[tt][j + 1]), hh, y2);
+              }
+              yq[tt] = y2.x + y2.y;
+            } else {
+              float y = 0.0f;
+#pragma unroll
+              for (int j = 0; j < NS; j++) {
+                const float nw = Bq[tt][j] * uq[tt] * nIA[j];
+                h[j] = fmaf(a[tt][j], h[j] - nw, nw);
+                y = fmaf(Cq[tt][j], h[j], y);
+              }
+              yq[tt] = y;
+            }
+          }
+        }
+        *reinterpret_cast<float4 *>(myp + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
+      }
       __syncwarp();
+
+      // -- combine the G partial readouts of the owned steps, D skip, gate, store
       float o[EPL];
 #pragma unroll
-      for (int j = 0; j < EPL; j++) {
-        const int tl = g * EPL + j, t = sb * kSub + tl;
-        float y = 0.0f;
+      for (int j = 0; j < EPL; j++) o[j] = 0.0f;
 #pragma unroll
-        for (int gg = 0; gg < G; gg++) y += yp[c * S::YC + gg * S::YG + tl];
-        y = fmaf(Dd, us[c * S::US + t], y);
-        o[j] = y * ss[c * S::US + t];
+      for (int gg = 0; gg < G; gg++) {
+        float part[EPL];
+        load_floats<EPL>(part, yp + c * S::YC + gg * S::YG + g * EPL);
+#pragma unroll
+        for (int j = 0; j < EPL; j++) o[j] += part[j];
       }
+#pragma unroll
+      for (int j = 0; j < EPL; j++) o[j] = fmaf(Dd, uown[j], o[j]) * gate[j];
       if (live && p.out)
-        store_run<Tout, EPL>(static_cast<Tout *>(p.out) + row0 + (int64_t)c * L,
-                             t0 + sb * kSub + g * EPL, L, o, vec);
+        store_run<Tout, EPL>(static_cast<Tout *>(p.out) + row0 + (int64_t)c * L, t0 + tb, L, o, vec);
       if (p.chunk_states && live && t0 + sb * kSub < L) {
         const int64_t kk = (t0 + sb * kSub) / kSub;
         float *dst = p.chunk_states + ((b * p.Dn + d) * p.n_ck + kk) * N;
@@ -303,7 +450,7 @@ ssm_fwd_kernel(const FwdParams p) {
         for (int j = 0; j < NS; j++)
           if (g * NS + j < N) dst[g * NS + j] = h[j];
       }
-      __syncwarp();
+      __syncwarp();  // ud / yp are rewritten by the next block
     }
   }
 }

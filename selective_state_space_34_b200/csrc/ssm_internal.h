@@ -46,6 +46,7 @@ struct BwdParams {
   float *p_dB, *p_dC;
   int64_t n_dtiles;
   float *dA_log, *dD, *ddt_bias, *dconv_w, *dconv_b;
+  void *const *timing_events;  // optional: 2 cudaEvent_t around the main backward kernel
 };
 
 LaneLayout choose_layout(int64_t N, int64_t channels);
