@@ -25,87 +25,73 @@
 // the result is deterministic.
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
+#include "ssm_stage.cuh"
 
 namespace ssm {
-
-template <typename T> __device__ __forceinline__ T bzero() { return from_f32<T>(0.0f); }
-
-// dst[r][i] = src[r][t0 + i] for r < rows_valid and 0 <= t0 + i < L, else 0, i in [0, LEN).
-template <typename T, int ROWS, int LEN>
-__device__ __forceinline__ void stage_rows_b(T *dst, int dst_stride, const T *src, int64_t src_stride,
-                                             int rows_valid, int64_t t0, int64_t L, bool vec) {
-  constexpr int EPV = 16 / sizeof(T);
-  constexpr int VPR = LEN / EPV;
-  if (vec) {
-    for (int idx = threadIdx.x; idx < ROWS * VPR; idx += kThreads) {
-      const int r = idx / VPR, v = idx % VPR;
-      const int64_t t = t0 + (int64_t)v * EPV;
-      T *d = dst + r * dst_stride + v * EPV;
-      if (r < rows_valid && t >= 0 && t < L)
-        cp_async16(d, src + (int64_t)r * src_stride + t);
-      else
-        *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
-    }
-  } else {
-    for (int idx = threadIdx.x; idx < ROWS * LEN; idx += kThreads) {
-      const int r = idx / LEN, i = idx % LEN;
-      const int64_t t = t0 + i;
-      dst[r * dst_stride + i] =
-          (r < rows_valid && t >= 0 && t < L) ? src[(int64_t)r * src_stride + t] : bzero<T>();
-    }
-  }
-}
 
 template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr int CH = kThreads / G;
   static constexpr int NP = G * NS;
   static constexpr int XS = kPre + kT;
   static constexpr int BS = NP + 4;
-  static constexpr int US = kT + 4;
-  static constexpr int YG = kSub + 8;
+  static constexpr int ES = kSub + 1;             // e3 row stride (float4: dl, u, dy, -)
+  static constexpr int YG = kSub + 4;
   static constexpr int YC = G * YG + 4;
-  static constexpr int DCS = kT + 8;            // dc row: this stage, then the next stage's 3
-  static constexpr int RBS = CH + 2;            // reduction buffer: stride between steps
-  static constexpr int RBN = kSub * RBS + 2;    // reduction buffer: stride between states
+  static constexpr int DCS = kT + 8;              // dc row: this stage, then the next stage's 3
+  static constexpr int RH = kSub / 2;             // steps per cross-channel reduction
+  static constexpr int CHH = CH / 2;
+  static constexpr int RBC = CHH * NP + 16;       // half-tile of channels (+16 words: banks)
+  static constexpr int RBT = 2 * RBC + 4;         // one step
+  static constexpr int RBW = RH * RBT;            // one quantity (dB or dC)
   static constexpr size_t x_off = 0;
   static constexpr size_t dt_off = x_off + sizeof(Tin) * 2 * CH * XS;
   static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * kT;
   static constexpr size_t do_off = z_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t braw_off = do_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t craw_off = braw_off + sizeof(Tin) * 2 * NP * kT;
-  static constexpr size_t bs_off = craw_off + sizeof(Tin) * 2 * NP * kT;
-  static constexpr size_t cs_off = bs_off + sizeof(float) * kT * BS;
-  static constexpr size_t us_off = cs_off + sizeof(float) * kT * BS;
-  static constexpr size_t dls_off = us_off + sizeof(float) * CH * US;
-  static constexpr size_t dys_off = dls_off + sizeof(float) * CH * US;
-  static constexpr size_t yb0_off = dys_off + sizeof(float) * CH * US;
-  static constexpr size_t yb1_off = yb0_off + sizeof(float) * CH * YC;
-  static constexpr size_t dcs_off = yb1_off + sizeof(float) * CH * YC;
+  static constexpr size_t bs_off = do_off + sizeof(Tin) * 2 * CH * kT;
+  static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * kT * BS;
+  static constexpr size_t e3_off = cs_off + sizeof(float) * 2 * kT * BS;
+  static constexpr size_t y0_off = e3_off + sizeof(float4) * CH * ES;
+  static constexpr size_t y1_off = y0_off + sizeof(float) * CH * YC;
+  static constexpr size_t dcs_off = y1_off + sizeof(float) * CH * YC;
   static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
-  static constexpr size_t bytes = rb_off + ((sizeof(float) * NP * RBN + 15) / 16) * 16;
+  static constexpr size_t bytes = rb_off + sizeof(float) * 2 * RBW;
+  __host__ __device__ static constexpr int rb_index(int which, int tt, int c, int n) {
+    return which * RBW + tt * RBT + (c / CHH) * RBC + (c % CHH) * NP + n;
+  }
 };
 
+template <int NS> __device__ __forceinline__ void store_states(float *dst, const float *v) {
+  if (NS % 4 == 0) {
+#pragma unroll
+    for (int j = 0; j < NS; j += 4)
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  } else if (NS % 2 == 0) {
+#pragma unroll
+    for (int j = 0; j < NS; j += 2) *reinterpret_cast<float2 *>(dst + j) = make_float2(v[j], v[j + 1]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NS; j++) dst[j] = v[j];
+  }
+}
+
 template <int G, int NS, typename Tin>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 ssm_bwd_kernel(const BwdParams P) {
   using S = BwdSmem<G, NS, Tin>;
-  constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G;
+  constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G, RH = S::RH;
   constexpr bool PRECISE = sizeof(Tin) == 4;
+  constexpr bool PAIRS = !PRECISE && (NS % 2 == 0);
   const FwdParams &p = P.f;
   extern __shared__ __align__(16) unsigned char smem[];
   Tin *xs = reinterpret_cast<Tin *>(smem + S::x_off);
   Tin *dts = reinterpret_cast<Tin *>(smem + S::dt_off);
   Tin *zs = reinterpret_cast<Tin *>(smem + S::z_off);
   Tin *dos = reinterpret_cast<Tin *>(smem + S::do_off);
-  Tin *braw = reinterpret_cast<Tin *>(smem + S::braw_off);
-  Tin *craw = reinterpret_cast<Tin *>(smem + S::craw_off);
   float *Bs = reinterpret_cast<float *>(smem + S::bs_off);
   float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
-  float *us = reinterpret_cast<float *>(smem + S::us_off);
-  float *dls = reinterpret_cast<float *>(smem + S::dls_off);
-  float *dys = reinterpret_cast<float *>(smem + S::dys_off);
-  float *yb0 = reinterpret_cast<float *>(smem + S::yb0_off);
-  float *yb1 = reinterpret_cast<float *>(smem + S::yb1_off);
+  float4 *e3 = reinterpret_cast<float4 *>(smem + S::e3_off);
+  float *y0 = reinterpret_cast<float *>(smem + S::y0_off);
+  float *y1 = reinterpret_cast<float *>(smem + S::y1_off);
   float *dcs = reinterpret_cast<float *>(smem + S::dcs_off);
   float *rb = reinterpret_cast<float *>(smem + S::rb_off);
 
@@ -121,28 +107,38 @@ ssm_bwd_kernel(const BwdParams P) {
   const bool vec = p.vec != 0;
   const int64_t L = p.L, N = p.N;
 
-  float A[NS], Acoef[NS], invA[NS], lam[NS], aN[NS], dAl[NS];
+  // A, the exp coefficient (A, or A log2 e on the fast path) and -1/A per owned state
+  constexpr int NH = (NS + 1) / 2;  // state pairs per lane
+  float2 A2[NH], Ac2[NH], nIA2[NH], lam2[NH], aN2[NH], dAl2[NH];
+  float *A = reinterpret_cast<float *>(A2);
+  float *Acoef = reinterpret_cast<float *>(Ac2);
+  float *nIA = reinterpret_cast<float *>(nIA2);
+  float *lam = reinterpret_cast<float *>(lam2);
+  float *aN = reinterpret_cast<float *>(aN2);
+  float *dAl = reinterpret_cast<float *>(dAl2);
 #pragma unroll
-  for (int j = 0; j < NS; j++) {
+  for (int j = 0; j < 2 * NH; j++) {
     const int n = g * NS + j;
     lam[j] = 0.f;
     aN[j] = 0.f;
     dAl[j] = 0.f;
-    if (live && n < N) {
+    if (j < NS && live && n < N) {
       A[j] = -expf(p.A_log[d * N + n]);
       Acoef[j] = PRECISE ? A[j] : A[j] * kLog2e;
-      invA[j] = 1.0f / A[j];
+      nIA[j] = -1.0f / A[j];
     } else {
       A[j] = 0.f;
       Acoef[j] = 0.f;
-      invA[j] = 0.f;
+      nIA[j] = 0.f;
     }
   }
   float w4[4] = {0.f, 0.f, 0.f, 0.f};
   float cbias = 0.f, Dd = 0.f, dtb = 0.f;
   if (live) {
     if (has_conv) {
-      for (int k = 0; k < p.K; k++) w4[k] = p.conv_w[d * p.K + k];
+#pragma unroll
+      for (int k = 0; k < 4; k++)
+        if (k < p.K) w4[k] = p.conv_w[d * p.K + k];
       cbias = p.conv_b ? p.conv_b[d] : 0.f;
     }
     Dd = p.D ? p.D[d] : 0.f;
@@ -160,230 +156,340 @@ ssm_bwd_kernel(const BwdParams P) {
   const int n_rows = (int)imin64(NP, N);
   const float *states = P.chunk_states ? P.chunk_states : p.chunk_states;
 
-  // dc halo of the (non-existent) stage after the sequence end is zero
+  // dc of the (non-existent) steps after the sequence end are zero
   for (int i = tid; i < CH * S::DCS; i += kThreads) dcs[i] = 0.f;
 
   const int64_t n_stages = (L + kT - 1) / kT;
   auto issue = [&](int64_t stage, int buf) {
     const int64_t t0 = stage * kT;
-    stage_rows_b<Tin, CH, kPre + kT>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
-    stage_rows_b<Tin, CH, kT>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
-    if (has_z) stage_rows_b<Tin, CH, kT>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
-    stage_rows_b<Tin, CH, kT>(dos + buf * CH * kT, kT, gdo, L, rows_valid, t0, L, vec);
-    stage_rows_b<Tin, NP, kT>(braw + buf * NP * kT, kT, gB, L, n_rows, t0, L, vec);
-    stage_rows_b<Tin, NP, kT>(craw + buf * NP * kT, kT, gC, L, n_rows, t0, L, vec);
+    stage_rows<Tin, CH, kPre + kT>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
+    stage_rows<Tin, CH>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
+    if (has_z) stage_rows<Tin, CH>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
+    stage_rows<Tin, CH>(dos + buf * CH * kT, kT, gdo, L, rows_valid, t0, L, vec);
     cp_async_commit();
   };
 
-  if (n_stages > 0) issue(n_stages - 1, (int)((n_stages - 1) & 1));
+  BCStager<Tin, NP> bc;
+  if (n_stages > 0) {
+    const int lbuf = (int)((n_stages - 1) & 1);
+    issue(n_stages - 1, lbuf);
+    bc.load(gB, gC, n_rows, (n_stages - 1) * kT, L, vec);
+    bc.store(Bs + lbuf * kT * S::BS, Cs + lbuf * kT * S::BS, S::BS);
+    if (n_stages > 1) bc.load(gB, gC, n_rows, (n_stages - 2) * kT, L, vec);
+  }
   for (int64_t st = n_stages - 1; st >= 0; st--) {
-    const int buf = (int)(st & 1);
+    const int buf = (int)(st & 1), pbuf = buf ^ 1;
     const int64_t t0 = st * kT;
     cp_async_wait<0>();
-    __syncthreads();
-    if (st > 0) issue(st - 1, buf ^ 1);
-
-    for (int i = tid; i < NP * kT; i += kThreads) {
-      const int n = i / kT, t = i % kT;
-      Bs[t * S::BS + n] = to_f32(braw[buf * NP * kT + i]);
-      Cs[t * S::BS + n] = to_f32(craw[buf * NP * kT + i]);
+    __syncthreads();  // stage st landed; B/C rows of stage st written; stage st+1's buffers free
+    if (st > 0) {
+      issue(st - 1, pbuf);
+      bc.store(Bs + pbuf * kT * S::BS, Cs + pbuf * kT * S::BS, S::BS);
+      if (st > 1) bc.load(gB, gC, n_rows, (st - 2) * kT, L, vec);
     }
+    const float *Bst = Bs + buf * kT * S::BS;
+    const float *Cst = Cs + buf * kT * S::BS;
     const Tin *xrow = xs + (buf * CH + c) * S::XS + kPre;
     const Tin *dtrow = dts + (buf * CH + c) * kT;
     const Tin *zrow = zs + (buf * CH + c) * kT;
     const Tin *dorow = dos + (buf * CH + c) * kT;
 
-    // per-element phase A: u, Delta, dy for the steps this lane owns
-#pragma unroll
-    for (int sb = 0; sb < kT / kSub; sb++) {
-#pragma unroll
-      for (int j = 0; j < EPL; j++) {
-        const int t = sb * kSub + g * EPL + j;
-        float u;
-        if (has_conv) {
-          float acc = cbias;
-#pragma unroll
-          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], to_f32(xrow[t - k]), acc);
-          u = acc * sigmoid<PRECISE>(acc);
-        } else {
-          u = to_f32(xrow[t]);
-        }
-        const float v = to_f32(dtrow[t]) + dtb;
-        float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
-        float dy = to_f32(dorow[t]);
-        if (has_z) {
-          const float zz = to_f32(zrow[t]);
-          dy *= zz * sigmoid<PRECISE>(zz);
-        }
-        if (t0 + t >= L) {
-          u = 0.f;
-          dl = 0.f;
-          dy = 0.f;
-        }
-        us[c * S::US + t] = u;
-        dls[c * S::US + t] = dl;
-        dys[c * S::US + t] = dy;
-      }
-    }
-    __syncthreads();
-
 #pragma unroll
     for (int sb = kT / kSub - 1; sb >= 0; sb--) {
-      const int64_t tb = t0 + sb * kSub;  // first step of this block
-      // (a) start state of the block
-      float h0[NS];
+      const int tb = sb * kSub + g * EPL;  // first owned step (stage-local)
+      const int64_t tblk = t0 + sb * kSub;  // first step of the block (global)
+      // (A) per-element values of the owned steps: u, Delta, dy -> e3
       {
-        const int64_t kk = tb / kSub;
+        float xw[EPL + 4], dtw[EPL], zw[EPL], dow[EPL];
+        load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+        load_window<Tin, EPL>(dtw, dtrow + tb);
+        load_window<Tin, EPL>(dow, dorow + tb);
+        if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
 #pragma unroll
-        for (int j = 0; j < NS; j++) {
-          const int n = g * NS + j;
-          h0[j] = (kk > 0 && live && n < N) ? states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n] : 0.f;
-        }
-      }
-      // (b) forward recompute: e = A_bar (fast) or A_bar - 1 (precise), and h, kept in registers
-      float ea[kSub][NS], hh[kSub][NS];
-      float *my0 = yb0 + c * S::YC + g * S::YG;
-      float *my1 = yb1 + c * S::YC + g * S::YG;
-      {
-        float h[NS];
+        for (int j = 0; j < EPL; j++) {
+          float u;
+          if (has_conv) {
+            float acc = cbias;
 #pragma unroll
-        for (int j = 0; j < NS; j++) h[j] = h0[j];
-#pragma unroll
-        for (int tt = 0; tt < kSub; tt++) {
-          const int t = sb * kSub + tt;
-          const float u = us[c * S::US + t], dl = dls[c * S::US + t], dy = dys[c * S::US + t];
-          const float *brow = Bs + t * S::BS + g * NS;
-          const float *crow = Cs + t * S::BS + g * NS;
-          float y = 0.f;
-#pragma unroll
-          for (int j = 0; j < NS; j++) {
-            const float w = brow[j] * u * invA[j];
-            if (PRECISE) {
-              const float em1 = expm1f(dl * Acoef[j]);
-              h[j] = fmaf(em1, h[j] + w, h[j]);
-              ea[tt][j] = em1;
-            } else {
-              const float a = ex2_approx(dl * Acoef[j]);
-              h[j] = fmaf(a, h[j] + w, -w);
-              ea[tt][j] = a;
-            }
-            hh[tt][j] = h[j];
-            y = fmaf(crow[j], h[j], y);
-            rb[(g * NS + j) * S::RBN + tt * S::RBS + c] = dy * h[j];  // dC partial
+            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
+            u = acc * sigmoid<PRECISE>(acc);
+          } else {
+            u = xw[j + 4];
           }
-          my0[tt] = y;
+          const float v = dtw[j] + dtb;
+          float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
+          float dy = dow[j];
+          if (has_z) dy *= zw[j] * sigmoid<PRECISE>(zw[j]);
+          if (t0 + tb + j >= L) {
+            u = 0.f;
+            dl = 0.f;
+            dy = 0.f;
+          }
+          e3[c * S::ES + g * EPL + j] = make_float4(dl, u, dy, 0.f);
         }
       }
-      __syncthreads();
-      // (c) dC partial of this channel tile; y of the steps this lane owns
-      for (int o = tid; o < NP * kSub; o += kThreads) {
-        const int n = o / kSub, tt = o % kSub;
-        const int64_t t = tb + tt;
-        if (n < N && t < L) {
-          float s = 0.f;
-          const float *r = rb + n * S::RBN + tt * S::RBS;
-          for (int cc = 0; cc < CH; cc++) s += r[cc];
-          P.p_dC[((tile * p.Bt + b) * N + n) * L + t] = s;
-        }
-      }
-      float yfin[EPL];
-#pragma unroll
-      for (int j = 0; j < EPL; j++) {
-        const int tl = g * EPL + j;
-        float y = 0.f;
-#pragma unroll
-        for (int gg = 0; gg < G; gg++) y += yb0[c * S::YC + gg * S::YG + tl];
-        yfin[j] = fmaf(Dd, us[c * S::US + sb * kSub + tl], y);
-      }
-      __syncthreads();
+      __syncwarp();
 
-      // (d) adjoint backwards through the block
+      // (B) recompute the block forward from its saved start state; keep A_bar (or A_bar - 1
+      //     on the precise path) and h of every step in registers
+      float2 ea2[kSub][NH], hs2[kSub][NH];
+      {
+        float2 h2[NH];
+        float *h = reinterpret_cast<float *>(h2);
+        const int64_t kk = tblk / kSub;
 #pragma unroll
-      for (int tt = kSub - 1; tt >= 0; tt--) {
-        const int t = sb * kSub + tt;
-        const float u = us[c * S::US + t], dl = dls[c * S::US + t], dy = dys[c * S::US + t];
-        const float *brow = Bs + t * S::BS + g * NS;
-        const float *crow = Cs + t * S::BS + g * NS;
-        float du = 0.f, dd = 0.f;
-#pragma unroll
-        for (int j = 0; j < NS; j++) {
-          const float anext = (tt + 1 < kSub) ? (PRECISE ? 1.f + ea[tt + 1][j] : ea[tt + 1][j]) : aN[j];
-          lam[j] = fmaf(anext, lam[j], dy * crow[j]);
-          const float em1 = PRECISE ? ea[tt][j] : ea[tt][j] - 1.0f;
-          const float bbar = em1 * brow[j] * invA[j];
-          const float lb = lam[j] * bbar;
-          du += lb;
-          rb[(g * NS + j) * S::RBN + tt * S::RBS + c] = lam[j] * u * em1 * invA[j];  // dB partial
-          const float dterm = lam[j] * fmaf(A[j], hh[tt][j], brow[j] * u);
-          dd += dterm;
-          dAl[j] = fmaf(dl, dterm, fmaf(-u, lb, dAl[j]));
+        for (int j = 0; j < 2 * NH; j++) {
+          const int n = g * NS + j;
+          h[j] = (j < NS && kk > 0 && live && n < N) ? states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n] : 0.f;
         }
-        my0[tt] = du;
-        my1[tt] = dd;
-      }
+        float *my0 = y0 + c * S::YC + g * S::YG;
 #pragma unroll
-      for (int j = 0; j < NS; j++) aN[j] = PRECISE ? 1.f + ea[0][j] : ea[0][j];
-      __syncthreads();
-      // (e) dB partial of this channel tile
-      for (int o = tid; o < NP * kSub; o += kThreads) {
-        const int n = o / kSub, tt = o % kSub;
-        const int64_t t = tb + tt;
-        if (n < N && t < L) {
-          float s = 0.f;
-          const float *r = rb + n * S::RBN + tt * S::RBS;
-          for (int cc = 0; cc < CH; cc++) s += r[cc];
-          P.p_dB[((tile * p.Bt + b) * N + n) * L + t] = s;
+        for (int tq = 0; tq < kSub; tq += 4) {
+          float4 eq[4];
+          float2 Bq[4][NH], Cq[4][NH];
+#pragma unroll
+          for (int tt = 0; tt < 4; tt++) {
+            const int t = sb * kSub + tq + tt;
+            eq[tt] = e3[c * S::ES + tq + tt];
+            load_states<NS>(reinterpret_cast<float *>(Bq[tt]), Bst + t * S::BS + g * NS);
+            load_states<NS>(reinterpret_cast<float *>(Cq[tt]), Cst + t * S::BS + g * NS);
+          }
+          float yq[4];
+#pragma unroll
+          for (int tt = 0; tt < 4; tt++) {
+            if (PAIRS) {
+              const float2 dl2 = make_float2(eq[tt].x, eq[tt].x), u2 = make_float2(eq[tt].y, eq[tt].y);
+              float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int q = 0; q < NH; q++) {
+                const float2 x = __fmul2_rn(dl2, Ac2[q]);
+                float2 a;
+                a.x = ex2_approx(x.x);
+                a.y = ex2_approx(x.y);
+                const float2 nw = __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), nIA2[q]);  // -B u / A
+                h2[q] = __ffma2_rn(a, __ffma2_rn(nw, make_float2(-1.f, -1.f), h2[q]), nw);
+                ea2[tq + tt][q] = a;
+                hs2[tq + tt][q] = h2[q];
+                y2 = __ffma2_rn(Cq[tt][q], h2[q], y2);
+              }
+              yq[tt] = y2.x + y2.y;
+            } else {
+              const float *Bt = reinterpret_cast<const float *>(Bq[tt]);
+              const float *Ct = reinterpret_cast<const float *>(Cq[tt]);
+              float *eat = reinterpret_cast<float *>(ea2[tq + tt]);
+              float *hst = reinterpret_cast<float *>(hs2[tq + tt]);
+              float y = 0.f;
+#pragma unroll
+              for (int j = 0; j < NS; j++) {
+                const float nw = Bt[j] * eq[tt].y * nIA[j];  // -B u / A
+                if (PRECISE) {
+                  const float em1 = expm1f(eq[tt].x * Acoef[j]);
+                  h[j] = fmaf(em1, h[j] - nw, h[j]);
+                  eat[j] = em1;
+                } else {
+                  const float a = ex2_approx(eq[tt].x * Acoef[j]);
+                  h[j] = fmaf(a, h[j] - nw, nw);
+                  eat[j] = a;
+                }
+                hst[j] = h[j];
+                y = fmaf(Ct[j], h[j], y);
+              }
+              yq[tt] = y;
+            }
+          }
+          *reinterpret_cast<float4 *>(my0 + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
         }
       }
-      // (f) per-element phase C for the steps this lane owns
+      __syncwarp();
+      float yfin[EPL];
+      {
+        float o[EPL];
 #pragma unroll
-      for (int j = 0; j < EPL; j++) {
-        const int tl = g * EPL + j, t = sb * kSub + tl;
-        const int64_t tg = t0 + t;
-        float du = 0.f, ddl = 0.f;
+        for (int j = 0; j < EPL; j++) o[j] = 0.f;
 #pragma unroll
         for (int gg = 0; gg < G; gg++) {
-          du += yb0[c * S::YC + gg * S::YG + tl];
-          ddl += yb1[c * S::YC + gg * S::YG + tl];
-        }
-        const float u = us[c * S::US + t], dy = dys[c * S::US + t];
-        du = fmaf(Dd, dy, du);
-        const bool in = live && tg < L;
-        if (in) accD = fmaf(dy, u, accD);
-        // gate
-        if (has_z && in) {
-          const float zz = to_f32(zrow[t]);
-          const float sg = sigmoid<PRECISE>(zz);
-          const float dz = to_f32(dorow[t]) * yfin[j] * sg * fmaf(zz, 1.f - sg, 1.f);
-          if (P.dz) P.dz[(b * p.Dn + d) * L + tg] = dz;
-        }
-        // Delta -> dt
-        const float v = to_f32(dtrow[t]) + dtb;
-        const float dv = p.delta_softplus ? ddl * sigmoid<PRECISE>(v) : ddl;
-        if (in) {
-          if (P.ddt) P.ddt[(b * p.Dn + d) * L + tg] = dv;
-          accDtb += dv;
-        }
-        // u -> conv pre-activation
-        if (has_conv) {
-          float acc = cbias;
+          float part[EPL];
+          load_floats<EPL>(part, y0 + c * S::YC + gg * S::YG + g * EPL);
 #pragma unroll
-          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], to_f32(xrow[t - k]), acc);
-          const float sg = sigmoid<PRECISE>(acc);
-          const float dc = in ? du * sg * fmaf(acc, 1.f - sg, 1.f) : 0.f;
-          dcs[c * S::DCS + t] = dc;
-          accCb += dc;
+          for (int j = 0; j < EPL; j++) o[j] += part[j];
+        }
 #pragma unroll
-          for (int k = 0; k < 4; k++) accW[k] = fmaf(dc, to_f32(xrow[t - k]), accW[k]);
-        } else if (in && P.dx) {
-          P.dx[(b * p.Dn + d) * L + tg] = du;
+        for (int j = 0; j < EPL; j++) yfin[j] = fmaf(Dd, e3[c * S::ES + g * EPL + j].y, o[j]);
+      }
+      __syncwarp();  // y0 is reused for the du partials
+
+      // (C) the adjoint backwards through the block, in two halves of RH steps; each half's
+      //     dB / dC partials are summed over the CTA's channels right after it
+#pragma unroll
+      for (int hf = kSub / RH - 1; hf >= 0; hf--) {
+        float *my0 = y0 + c * S::YC + g * S::YG;
+        float *my1 = y1 + c * S::YC + g * S::YG;
+#pragma unroll
+        for (int tq = hf * RH + RH - 4; tq >= hf * RH; tq -= 4) {
+          float duq[4], ddq[4];
+#pragma unroll
+          for (int tt = 3; tt >= 0; tt--) {
+            const int tl = tq + tt, t = sb * kSub + tl;
+            const float4 e = e3[c * S::ES + tl];  // (dl, u, dy, -)
+            float2 Bv[NH], Cv[NH];
+            load_states<NS>(reinterpret_cast<float *>(Bv), Bst + t * S::BS + g * NS);
+            load_states<NS>(reinterpret_cast<float *>(Cv), Cst + t * S::BS + g * NS);
+            float2 nB2[NH], dC2[NH];
+            float *nB = reinterpret_cast<float *>(nB2);
+            float *dCv = reinterpret_cast<float *>(dC2);
+            float ndu = 0.f, dd = 0.f;
+            if (PAIRS) {
+              float2 ndu2 = make_float2(0.f, 0.f), dd2 = make_float2(0.f, 0.f);
+              const float2 dl2 = make_float2(e.x, e.x), u2 = make_float2(e.y, e.y), dy2 = make_float2(e.z, e.z);
+#pragma unroll
+              for (int q = 0; q < NH; q++) {
+                const float2 an2 = (tl + 1 < kSub) ? ea2[tl + 1][q] : aN2[q];
+                lam2[q] = __ffma2_rn(an2, lam2[q], __fmul2_rn(Cv[q], dy2));           // lambda_t
+                const float2 em1n = __fmul2_rn(__fadd2_rn(ea2[tl][q], make_float2(-1.f, -1.f)),
+                                               nIA2[q]);                               // -(A_bar-1)/A
+                const float2 nlb = __fmul2_rn(lam2[q], __fmul2_rn(em1n, Bv[q]));      // -lambda B_bar
+                ndu2 = __fadd2_rn(ndu2, nlb);
+                nB2[q] = __fmul2_rn(__fmul2_rn(lam2[q], em1n), u2);                   // -dB partial
+                dC2[q] = __fmul2_rn(hs2[tl][q], dy2);
+                const float2 dterm = __fmul2_rn(lam2[q], __ffma2_rn(A2[q], hs2[tl][q], __fmul2_rn(Bv[q], u2)));
+                dd2 = __fadd2_rn(dd2, dterm);
+                dAl2[q] = __ffma2_rn(u2, nlb, __ffma2_rn(dl2, dterm, dAl2[q]));       // A dA
+              }
+              ndu = ndu2.x + ndu2.y;
+              dd = dd2.x + dd2.y;
+            } else {
+              const float *Bt = reinterpret_cast<const float *>(Bv);
+              const float *Ct = reinterpret_cast<const float *>(Cv);
+              const float *eat = reinterpret_cast<const float *>(ea2[tl]);
+              const float *ean = reinterpret_cast<const float *>(tl + 1 < kSub ? ea2[tl + 1] : aN2);
+              const float *hst = reinterpret_cast<const float *>(hs2[tl]);
+#pragma unroll
+              for (int j = 0; j < NS; j++) {
+                const float em1 = PRECISE ? eat[j] : eat[j] - 1.f;
+                const float an = (PRECISE && tl + 1 < kSub) ? 1.f + ean[j] : ean[j];
+                lam[j] = fmaf(an, lam[j], Ct[j] * e.z);
+                const float em1n = em1 * nIA[j];
+                const float nlb = lam[j] * (em1n * Bt[j]);
+                ndu += nlb;
+                nB[j] = lam[j] * em1n * e.y;
+                dCv[j] = hst[j] * e.z;
+                const float dterm = lam[j] * fmaf(A[j], hst[j], Bt[j] * e.y);
+                dd += dterm;
+                dAl[j] = fmaf(e.y, nlb, fmaf(e.x, dterm, dAl[j]));
+              }
+            }
+            store_states<NS>(rb + S::rb_index(0, tl - hf * RH, c, g * NS), nB);
+            store_states<NS>(rb + S::rb_index(1, tl - hf * RH, c, g * NS), dCv);
+            duq[tt] = -ndu;
+            ddq[tt] = dd;
+          }
+          *reinterpret_cast<float4 *>(my0 + tq) = make_float4(duq[0], duq[1], duq[2], duq[3]);
+          *reinterpret_cast<float4 *>(my1 + tq) = make_float4(ddq[0], ddq[1], ddq[2], ddq[3]);
+        }
+        __syncthreads();  // the half-block's dB / dC partials of every channel are in place
+        {
+          constexpr int NQ = NP / 4;
+          constexpr int NGRP = 2 * RH * NQ;
+          constexpr int SPLIT = NGRP >= kThreads ? 1 : (kThreads / NGRP > 2 ? 2 : kThreads / NGRP);
+          constexpr int CPS = CH / SPLIT;
+          const int part = tid % SPLIT;
+          for (int gi = tid / SPLIT; gi < NGRP; gi += kThreads / SPLIT) {
+            const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int ci = 0; ci < CPS; ci++) {
+              const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, part * CPS + ci, 4 * q));
+              acc.x += v.x;
+              acc.y += v.y;
+              acc.z += v.z;
+              acc.w += v.w;
+            }
+#pragma unroll
+            for (int off = 1; off < SPLIT; off <<= 1) {
+              acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+              acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+              acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+              acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+            }
+            const int64_t t = tblk + hf * RH + tt;
+            if (part == 0 && t < L) {
+              float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
+              const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
+              const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+              for (int k = 0; k < 4; k++)
+                if (4 * q + k < N) dst[(int64_t)(4 * q + k) * L] = sg * vals[k];
+            }
+          }
+        }
+        __syncthreads();  // rb is rewritten by the next half
+      }
+#pragma unroll
+      for (int q = 0; q < NH; q++) aN2[q] = PRECISE ? make_float2(1.f + ea2[0][q].x, 1.f + ea2[0][q].y) : ea2[0][q];
+
+      // (D) per-element gradients of the owned steps
+      {
+        float xw[EPL + 4], dtw[EPL], zw[EPL], dow[EPL], dup[EPL], ddp[EPL];
+        load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+        load_window<Tin, EPL>(dtw, dtrow + tb);
+        load_window<Tin, EPL>(dow, dorow + tb);
+        if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
+#pragma unroll
+        for (int j = 0; j < EPL; j++) {
+          dup[j] = 0.f;
+          ddp[j] = 0.f;
+        }
+#pragma unroll
+        for (int gg = 0; gg < G; gg++) {
+          float a0[EPL], a1[EPL];
+          load_floats<EPL>(a0, y0 + c * S::YC + gg * S::YG + g * EPL);
+          load_floats<EPL>(a1, y1 + c * S::YC + gg * S::YG + g * EPL);
+#pragma unroll
+          for (int j = 0; j < EPL; j++) {
+            dup[j] += a0[j];
+            ddp[j] += a1[j];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < EPL; j++) {
+          const int t = tb + j;
+          const int64_t tg = t0 + t;
+          const bool in = live && tg < L;
+          const float4 e = e3[c * S::ES + g * EPL + j];
+          const float du = fmaf(Dd, e.z, dup[j]);
+          if (in) accD = fmaf(e.z, e.y, accD);
+          if (has_z && in) {
+            const float sg = sigmoid<PRECISE>(zw[j]);
+            const float dz = dow[j] * yfin[j] * sg * fmaf(zw[j], 1.f - sg, 1.f);
+            if (P.dz) P.dz[(b * p.Dn + d) * L + tg] = dz;
+          }
+          const float v = dtw[j] + dtb;
+          const float dv = p.delta_softplus ? ddp[j] * sigmoid<PRECISE>(v) : ddp[j];
+          if (in) {
+            if (P.ddt) P.ddt[(b * p.Dn + d) * L + tg] = dv;
+            accDtb += dv;
+          }
+          if (has_conv) {
+            float acc = cbias;
+#pragma unroll
+            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
+            const float sg = sigmoid<PRECISE>(acc);
+            const float dc = in ? du * sg * fmaf(acc, 1.f - sg, 1.f) : 0.f;
+            dcs[c * S::DCS + t] = dc;
+            accCb += dc;
+#pragma unroll
+            for (int k = 0; k < 4; k++) accW[k] = fmaf(dc, xw[j + 4 - k], accW[k]);
+          } else if (in && P.dx) {
+            P.dx[(b * p.Dn + d) * L + tg] = du;
+          }
         }
       }
-      __syncthreads();
     }
 
-    // conv backward for the stage: dx_t = sum_k w[k] dc_{t+k} (dc beyond the stage = halo)
+    // conv backward for the stage: dx_t = sum_k w[k] dc_{t+k} (dc beyond the stage = halo).
+    // dcs rows are written and read by the G lanes of their own channel only.
     if (has_conv) {
+      __syncwarp();
 #pragma unroll
       for (int sb = 0; sb < kT / kSub; sb++) {
 #pragma unroll
@@ -396,12 +502,11 @@ ssm_bwd_kernel(const BwdParams P) {
           if (live && tg < L && P.dx) P.dx[(b * p.Dn + d) * L + tg] = acc;
         }
       }
-      __syncthreads();
+      __syncwarp();
       // this stage's first 3 dc values become the halo of the stage before it
-      if (g == 0) {
+      if (g == 0)
         for (int k = 0; k < 3; k++) dcs[c * S::DCS + kT + k] = dcs[c * S::DCS + k];
-      }
-      // (visible to the next stage after its top-of-loop barrier)
+      __syncwarp();
     }
   }
 
