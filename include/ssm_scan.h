@@ -150,6 +150,26 @@ size_t ssm_bwd_workspace_size(const ssm_bwd_args *args);
  */
 ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream);
 
+/* Size of the scratch array built into the library for ssm_scan_bwd_noalloc (64 MiB). */
+#define SSM_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * ssm_scan_bwd_noalloc -- the same backward as ssm_scan_bwd for callers that cannot allocate device
+ * memory (a host program or plugin that only receives device pointers and has no allocator, or
+ * code running where allocating is not permitted). The pages describe no such entry point: it has
+ * no counterpart there and exists only for these callers.
+ *
+ * Arguments are those of ssm_scan_bwd; args->workspace and args->workspace_bytes are ignored.
+ * Scratch comes from one library-owned device array of SSM_NOALLOC_SCRATCH_BYTES per GPU, held
+ * until the process exits. Problems whose ssm_bwd_workspace_size() exceeds that size are rejected
+ * with SSM_ERR_WORKSPACE before anything runs (pass chunk_states from the forward to keep the
+ * requirement small). The first call on a device looks up the array's device address (a runtime
+ * API call): make it before any stream capture on that device. All calls on a device share the
+ * array, so calls that overlap on the GPU race; order them (one stream, or events). The call
+ * allocates nothing (no cudaMalloc / cudaFree). Errors: as ssm_scan_bwd.
+ */
+ssm_status ssm_scan_bwd_noalloc(const ssm_bwd_args *args, void *stream);
+
 /*
  * Standalone causal depthwise conv1d + SiLU: u = SiLU(b + sum_k w[k] * x_{t-k}).
  * x: device (Bt, Dn, L) in_dtype; u: device (Bt, Dn, L) out_dtype; w: device [Dn, K] fp32,

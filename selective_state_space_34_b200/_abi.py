@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 
 SSM_F32, SSM_BF16 = 0, 1
 SSM_STATE_CHUNK = 16
+SSM_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 STATUS = {
     0: "SSM_OK", 1: "SSM_ERR_NULL", 2: "SSM_ERR_SHAPE", 3: "SSM_ERR_ALIGN", 4: "SSM_ERR_DTYPE",
@@ -47,6 +48,7 @@ SIGNATURES = [
     ("ssm_scan_fwd", ctypes.c_int, [ctypes.POINTER(FwdArgs), ctypes.c_void_p]),
     ("ssm_bwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(BwdArgs)]),
     ("ssm_scan_bwd", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
+    ("ssm_scan_bwd_noalloc", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_conv1d_silu", ctypes.c_int,
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
       ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
