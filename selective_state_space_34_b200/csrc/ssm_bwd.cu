@@ -50,7 +50,8 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr size_t bs_off = do_off + sizeof(Tin) * 2 * CH * kT;
   static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * kT * BS;
   static constexpr size_t e3_off = cs_off + sizeof(float) * 2 * kT * BS;
-  static constexpr size_t y0_off = e3_off + sizeof(float4) * CH * ES;
+  static constexpr size_t pe_off = e3_off + sizeof(float4) * CH * ES;   // (gc, sv, gz, -)
+  static constexpr size_t y0_off = pe_off + sizeof(float4) * CH * ES;
   static constexpr size_t y1_off = y0_off + sizeof(float) * CH * YC;
   static constexpr size_t dcs_off = y1_off + sizeof(float) * CH * YC;
   static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
@@ -90,6 +91,7 @@ ssm_bwd_kernel(const BwdParams P) {
   float *Bs = reinterpret_cast<float *>(smem + S::bs_off);
   float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
   float4 *e3 = reinterpret_cast<float4 *>(smem + S::e3_off);
+  float4 *pe = reinterpret_cast<float4 *>(smem + S::pe_off);
   float *y0 = reinterpret_cast<float *>(smem + S::y0_off);
   float *y1 = reinterpret_cast<float *>(smem + S::y1_off);
   float *dcs = reinterpret_cast<float *>(smem + S::dcs_off);
@@ -207,25 +209,41 @@ ssm_bwd_kernel(const BwdParams P) {
         if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
-          float u;
+          // u = SiLU(c) with dSiLU/dc = s (1 + c (1 - s)); Delta = softplus(v) with dDelta/dv =
+          // sigmoid(v); out = y SiLU(z) with dout/dz = y s_z (1 + z (1 - s_z))
+          float u, gc = 1.f;
           if (has_conv) {
             float acc = cbias;
 #pragma unroll
             for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
-            u = acc * sigmoid<PRECISE>(acc);
+            const float sc = sigmoid<PRECISE>(acc);
+            u = acc * sc;
+            gc = sc * fmaf(acc, 1.f - sc, 1.f);
           } else {
             u = xw[j + 4];
           }
           const float v = dtw[j] + dtb;
-          float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
-          float dy = dow[j];
-          if (has_z) dy *= zw[j] * sigmoid<PRECISE>(zw[j]);
+          float dl = v, sv = 1.f;
+          if (p.delta_softplus) {
+            dl = softplus<PRECISE>(v);
+            sv = sigmoid<PRECISE>(v);
+          }
+          float dy = dow[j], gz = 0.f;
+          if (has_z) {
+            const float sz = sigmoid<PRECISE>(zw[j]);
+            dy *= zw[j] * sz;
+            gz = dow[j] * sz * fmaf(zw[j], 1.f - sz, 1.f);
+          }
           if (t0 + tb + j >= L) {
             u = 0.f;
             dl = 0.f;
             dy = 0.f;
+            gc = 0.f;
+            sv = 0.f;
+            gz = 0.f;
           }
           e3[c * S::ES + g * EPL + j] = make_float4(dl, u, dy, 0.f);
+          pe[c * S::ES + g * EPL + j] = make_float4(gc, sv, gz, 0.f);
         }
       }
       __syncwarp();
@@ -395,15 +413,25 @@ ssm_bwd_kernel(const BwdParams P) {
           const int part = tid % SPLIT;
           for (int gi = tid / SPLIT; gi < NGRP; gi += kThreads / SPLIT) {
             const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+            if (CPS == S::CHH || CPS * 2 == S::CHH || CPS * 4 == S::CHH) {
+              // this thread's channels lie in one half: walk them with a fixed stride
+              const float *src = rb + S::rb_index(which, tt, part * CPS, 4 * q);
+#pragma unroll 8
+              for (int ci = 0; ci < CPS; ci++) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + ci * NP);
+                a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
+                a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
+              }
+            } else {
 #pragma unroll 4
-            for (int ci = 0; ci < CPS; ci++) {
-              const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, part * CPS + ci, 4 * q));
-              acc.x += v.x;
-              acc.y += v.y;
-              acc.z += v.z;
-              acc.w += v.w;
+              for (int ci = 0; ci < CPS; ci++) {
+                const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, part * CPS + ci, 4 * q));
+                a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
+                a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
+              }
             }
+            float4 acc = make_float4(a01.x, a01.y, a23.x, a23.y);
 #pragma unroll
             for (int off = 1; off < SPLIT; off <<= 1) {
               acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
@@ -429,11 +457,7 @@ ssm_bwd_kernel(const BwdParams P) {
 
       // (D) per-element gradients of the owned steps
       {
-        float xw[EPL + 4], dtw[EPL], zw[EPL], dow[EPL], dup[EPL], ddp[EPL];
-        load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
-        load_window<Tin, EPL>(dtw, dtrow + tb);
-        load_window<Tin, EPL>(dow, dorow + tb);
-        if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
+        float dup[EPL], ddp[EPL];
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
           dup[j] = 0.f;
@@ -450,38 +474,31 @@ ssm_bwd_kernel(const BwdParams P) {
             ddp[j] += a1[j];
           }
         }
+        float xw[EPL + 4];
+        if (has_conv) load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+        float dzv[EPL], dtv[EPL], dcv[EPL];
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
-          const int t = tb + j;
-          const int64_t tg = t0 + t;
-          const bool in = live && tg < L;
-          const float4 e = e3[c * S::ES + g * EPL + j];
+          const float4 e = e3[c * S::ES + g * EPL + j];  // (dl, u, dy, -); zero past L
+          const float4 f = pe[c * S::ES + g * EPL + j];  // (gc, sv, gz, -); zero past L
           const float du = fmaf(Dd, e.z, dup[j]);
-          if (in) accD = fmaf(e.z, e.y, accD);
-          if (has_z && in) {
-            const float sg = sigmoid<PRECISE>(zw[j]);
-            const float dz = dow[j] * yfin[j] * sg * fmaf(zw[j], 1.f - sg, 1.f);
-            if (P.dz) P.dz[(b * p.Dn + d) * L + tg] = dz;
-          }
-          const float v = dtw[j] + dtb;
-          const float dv = p.delta_softplus ? ddp[j] * sigmoid<PRECISE>(v) : ddp[j];
-          if (in) {
-            if (P.ddt) P.ddt[(b * p.Dn + d) * L + tg] = dv;
-            accDtb += dv;
-          }
+          accD = fmaf(e.z, e.y, accD);
+          dzv[j] = yfin[j] * f.z;
+          dtv[j] = ddp[j] * f.y;
+          accDtb += dtv[j];
+          dcv[j] = du * f.x;
           if (has_conv) {
-            float acc = cbias;
+            dcs[c * S::DCS + tb + j] = dcv[j];
+            accCb += dcv[j];
 #pragma unroll
-            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
-            const float sg = sigmoid<PRECISE>(acc);
-            const float dc = in ? du * sg * fmaf(acc, 1.f - sg, 1.f) : 0.f;
-            dcs[c * S::DCS + t] = dc;
-            accCb += dc;
-#pragma unroll
-            for (int k = 0; k < 4; k++) accW[k] = fmaf(dc, xw[j + 4 - k], accW[k]);
-          } else if (in && P.dx) {
-            P.dx[(b * p.Dn + d) * L + tg] = du;
+            for (int k = 0; k < 4; k++) accW[k] = fmaf(dcv[j], xw[j + 4 - k], accW[k]);
           }
+        }
+        if (live) {
+          const int64_t roff = (b * p.Dn + d) * L;
+          if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, L, dzv, vec);
+          if (P.ddt) store_run<float, EPL>(P.ddt + roff, t0 + tb, L, dtv, vec);
+          if (!has_conv && P.dx) store_run<float, EPL>(P.dx + roff, t0 + tb, L, dcv, vec);
         }
       }
     }
@@ -492,15 +509,17 @@ ssm_bwd_kernel(const BwdParams P) {
       __syncwarp();
 #pragma unroll
       for (int sb = 0; sb < kT / kSub; sb++) {
+        float dxv[EPL];
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
           const int t = sb * kSub + g * EPL + j;
-          const int64_t tg = t0 + t;
           float acc = 0.f;
 #pragma unroll
           for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
-          if (live && tg < L && P.dx) P.dx[(b * p.Dn + d) * L + tg] = acc;
+          dxv[j] = acc;
         }
+        if (live && P.dx)
+          store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + sb * kSub + g * EPL, L, dxv, vec);
       }
       __syncwarp();
       // this stage's first 3 dc values become the halo of the stage before it
