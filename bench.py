@@ -37,6 +37,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 FMA_LANES, MUFU_LANES, N_SM = 128, 16, 148
 
 
+def ncu_traffic(kernel, source):
+    """DRAM bytes per launch of `kernel` from profiles/ncu_traffic.md, or None when the recorded
+    capture was taken on a different version of the kernel's source file."""
+    import hashlib
+    try:
+        sha = hashlib.sha256(open(os.path.join(ROOT, "selective_state_space_34_b200", "csrc", source),
+                                  "rb").read()).hexdigest()[:16]
+        for ln in open(os.path.join(ROOT, "profiles", "ncu_traffic.md")):
+            f = [x.strip() for x in ln.strip().strip("|").split("|")]
+            if len(f) == 3 and f[0] == kernel and f[1] == sha:
+                return int(f[2])
+    except Exception:
+        return None
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -361,22 +377,32 @@ def main():
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fb = fwd_bytes(Bt, Dn, N, L, s_in, s_out, states=False)
     fwd_roof = {"bound": "hbm", "achieved": fb / (fo_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                "frac": fb / (fo_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+                "frac": fb / (fo_ms * 1e-3) / 1e9 / hbm,
+                "traffic": ncu_traffic("ssm_fwd_kernel", "ssm_fwd.cu") if (s_out == 2 and s_in == 2) else None,
                 "algorithmic_bytes": fb, "kernel": "ssm_fwd_kernel", "ms": fo_ms,
                 "peak_source": peaks.get("source")}
     sm_hz = (clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6
-    mufu_peak = MUFU_LANES * N_SM * sm_hz  # ex2 per second at the sampled clock
+    mufu_peak = MUFU_LANES * N_SM * sm_hz / 1e9  # Gexp2/s at the sampled SM clock
+
+    def alu_roof(kernel, ms):
+        # the irreducible exp of the method: one A_bar = exp(Delta A) per element-state, against
+        # the exp unit's rate (16 results/clk/SM x 148 SMs x sampled clock)
+        ach = es / (ms * 1e-3) / 1e9
+        return {"bound": "alu", "achieved": ach, "peak": mufu_peak, "unit": "Gexp/s",
+                "frac": ach / mufu_peak, "kernel": kernel,
+                "peak_source": "16 MUFU ex2 lanes/clk/SM x 148 SMs x sampled SM clock"}
     forward = {"ms": fo_ms, "value": es * world / (fo_ms * 1e-3), "unit": UNIT,
                "out_dtype": args.out_dtype, "roofline": fwd_roof,
-               "alu": {"exp2_per_s": es / (fo_ms * 1e-3), "mufu_peak_per_s": mufu_peak,
-                       "frac_of_one_mufu_exp_per_elem_state": es / (fo_ms * 1e-3) / mufu_peak}}
+               "alu_roofline": alu_roof("ssm_fwd_kernel", fo_ms)}
 
     if backward:
         bms = kern["ssm_bwd_kernel"]
         bb = bwd_bytes(Bt, Dn, N, L, s_in, states=True)
         roof = {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                "frac": bb / (bms * 1e-3) / 1e9 / hbm, "traffic": None, "algorithmic_bytes": bb,
-                "kernel": "ssm_bwd_kernel", "ms": bms, "peak_source": peaks.get("source")}
+                "frac": bb / (bms * 1e-3) / 1e9 / hbm,
+                "traffic": ncu_traffic("ssm_bwd_kernel", "ssm_bwd.cu") if s_in == 2 else None,
+                "algorithmic_bytes": bb, "kernel": "ssm_bwd_kernel", "ms": bms,
+                "peak_source": peaks.get("source")}
     else:
         roof = dict(fwd_roof)
     launches_per_step = 1 + (3 if backward else 0)
@@ -440,6 +466,8 @@ def main():
                                  + (bwd_bytes(Bt, Dn, N, L, s_in) if backward else 0)) / 1e9),
                        "parallelism": "replica per GPU" if world > 1 else "single GPU"},
             "roofline": roof,
+            "alu_roofline": alu_roof("ssm_bwd_kernel" if backward else "ssm_fwd_kernel",
+                                     kern["ssm_bwd_kernel"] if backward else fo_ms),
             "kernels_ms": kern,
             "forward": forward,
             "cpu_baseline": cpu,
