@@ -49,11 +49,11 @@ def bind(lib):
     lib.ssm_oracle_zoh.argtypes = [ctypes.c_double] * 3 + [_dp, _dp]
     lib.ssm_oracle_conv1d_silu.restype = None
     lib.ssm_oracle_conv1d_silu.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, _dp]
-    common = [_dp] * 10 + [_i64] * 5 + [ctypes.c_int]
+    common = [_dp] * 10 + [_i64] * 5 + [ctypes.c_int, ctypes.c_int, _dp, _dp]
     lib.ssm_oracle_fwd.restype = ctypes.c_int
-    lib.ssm_oracle_fwd.argtypes = common + [_dp, _dp, _dp, ctypes.c_int]
+    lib.ssm_oracle_fwd.argtypes = common + [_dp] * 5 + [ctypes.c_int]
     lib.ssm_oracle_bwd.restype = ctypes.c_int
-    lib.ssm_oracle_bwd.argtypes = common + [_dp] * 11 + [ctypes.c_int]
+    lib.ssm_oracle_bwd.argtypes = common + [_dp] * 2 + [_dp] * 12 + [ctypes.c_int]
     return lib
 
 
@@ -113,38 +113,50 @@ def _shapes(x, A_log, conv_w):
 
 
 def fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, conv_b=None,
-        delta_softplus=True, want_u=False, want_y=False, n_threads=0):
+        delta_softplus=True, want_u=False, want_y=False, n_threads=0, euler=False, h0=None,
+        conv_hist=None, want_state=False):
     """Selective-scan forward. x, dt, z: (Bt, Dn, L); B, C: (Bt, N, L); A_log: (Dn, N);
-    D, dt_bias, conv_b: (Dn,); conv_w: (Dn, K). Returns out, or (out, extras) when extras are
-    requested: extras has 'u' (scan input) and/or 'y' (pre-gate output incl. D*u)."""
+    D, dt_bias, conv_b: (Dn,); conv_w: (Dn, K); h0: (Bt, Dn, N) carried state; conv_hist:
+    (Bt, Dn, K-1) carried pre-conv inputs, newest-first. Returns out, or (out, extras) when extras
+    are requested: 'u' (scan input), 'y' (pre-gate output incl. D*u), 'h_last' and
+    'conv_hist' (the carried state after this chunk)."""
     x, dt, A_log, B, C = _in(x), _in(dt), _in(A_log), _in(B), _in(C)
     D, z, dt_bias, conv_w, conv_b = _in(D), _in(z), _in(dt_bias), _in(conv_w), _in(conv_b)
+    h0, conv_hist = _in(h0), _in(conv_hist)
     Bt, Dn, N, L, K = _shapes(x, A_log, conv_w)
     out = np.empty_like(x)
     u = np.empty_like(x) if want_u else None
     y = np.empty_like(x) if want_y else None
+    hl = np.empty((Bt, Dn, N)) if want_state else None
+    ch = np.empty((Bt, Dn, max(K - 1, 0))) if (want_state and conv_w is not None) else None
     rc = _load().ssm_oracle_fwd(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log), _ptr(B), _ptr(C),
                                 _ptr(D), _ptr(z), _ptr(conv_w), _ptr(conv_b), Bt, Dn, N, L, K,
-                                int(bool(delta_softplus)), _ptr(out), _ptr(u), _ptr(y),
+                                int(bool(delta_softplus)), int(bool(euler)), _ptr(h0),
+                                _ptr(conv_hist), _ptr(out), _ptr(u), _ptr(y), _ptr(hl), _ptr(ch),
                                 int(n_threads))
     if rc != 0:
         raise MemoryError("ssm_oracle_fwd: allocation failed")
-    if want_u or want_y:
+    if want_u or want_y or want_state:
         ex = {}
         if want_u:
             ex["u"] = u
         if want_y:
             ex["y"] = y
+        if want_state:
+            ex["h_last"] = hl
+            ex["conv_hist"] = ch
         return out, ex
     return out
 
 
 def bwd(x, dt, A_log, B, C, dout, D=None, z=None, dt_bias=None, conv_w=None, conv_b=None,
-        delta_softplus=True, n_threads=0):
-    """Selective-scan backward (VJP of :func:`fwd` against ``dout``). Returns a dict with
-    dx, ddt, dA_log, dB, dC, dD, ddt_bias, and dz / dconv_w / dconv_b where those inputs exist."""
+        delta_softplus=True, n_threads=0, euler=False, h0=None, conv_hist=None, dh_last=None):
+    """Selective-scan backward (VJP of :func:`fwd` against ``dout`` and, optionally, ``dh_last``
+    for the carried state). Returns a dict with dx, ddt, dA_log, dB, dC, dD, ddt_bias, dh0, and
+    dz / dconv_w / dconv_b / dconv_hist where those inputs exist."""
     x, dt, A_log, B, C = _in(x), _in(dt), _in(A_log), _in(B), _in(C)
     D, z, dt_bias, conv_w, conv_b = _in(D), _in(z), _in(dt_bias), _in(conv_w), _in(conv_b)
+    h0, conv_hist, dh_last = _in(h0), _in(conv_hist), _in(dh_last)
     dout = _in(dout)
     Bt, Dn, N, L, K = _shapes(x, A_log, conv_w)
     g = {
@@ -154,15 +166,18 @@ def bwd(x, dt, A_log, B, C, dout, D=None, z=None, dt_bias=None, conv_w=None, con
     }
     if z is not None:
         g["dz"] = np.empty_like(x)
+    g["dh0"] = np.empty((Bt, Dn, N))
     if conv_w is not None:
         g["dconv_w"] = np.empty((Dn, K))
         g["dconv_b"] = np.empty(Dn)
+        g["dconv_hist"] = np.empty((Bt, Dn, max(K - 1, 0)))
     rc = _load().ssm_oracle_bwd(
         _ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-        _ptr(conv_w), _ptr(conv_b), Bt, Dn, N, L, K, int(bool(delta_softplus)), _ptr(dout),
+        _ptr(conv_w), _ptr(conv_b), Bt, Dn, N, L, K, int(bool(delta_softplus)), int(bool(euler)),
+        _ptr(h0), _ptr(conv_hist), _ptr(dout), _ptr(dh_last),
         _ptr(g["dx"]), _ptr(g["ddt"]), _ptr(g["dA_log"]), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dD"]), _ptr(g["ddt_bias"]), _ptr(g.get("dz")), _ptr(g.get("dconv_w")),
-        _ptr(g.get("dconv_b")), int(n_threads))
+        _ptr(g.get("dconv_b")), _ptr(g["dh0"]), _ptr(g.get("dconv_hist")), int(n_threads))
     if rc != 0:
         raise MemoryError("ssm_oracle_bwd: allocation failed")
     return g

@@ -37,6 +37,14 @@
  *  - softplus has no large-argument cut-off; the pages give none.
  *  - Delta = dt + dt_bias, then softplus when delta_softplus != 0 (dt_bias may be absent = 0).
  *  - Without a conv (conv_w == NULL) the input x is u itself.
+ *  - State carry ([TL] State, step, runArray): h0 is the state after the previous chunk (NULL =
+ *    zeroState), conv_hist holds the previous chunk's last K-1 pre-conv inputs newest-first
+ *    (history[0] is the most recent token; NULL = zero padding). The page keeps up to K entries
+ *    after a step, but a step only ever reads the K-1 newest of them together with the new token,
+ *    so K-1 entries carry everything the next chunk needs. h_last / conv_hist_out are the same
+ *    objects after this chunk; an empty chunk (L = 0) returns them unchanged.
+ *  - euler = 1 selects Mamba's first-order input discretisation B-bar = Delta * B
+ *    ([SSMK] mamba_selective_scan_step; [TL] step); A-bar stays exp(Delta * A).
  */
 #include <math.h>
 #include <stdint.h>
@@ -77,13 +85,25 @@ void ssm_oracle_zoh(double A, double B, double delta, double *Abar, double *Bbar
  * token; history newest-first and zero-padded), u_t = SiLU(c_t). [TL] convKernel / convBias /
  * State.history; [RT] "causal depthwise conv1d -> SiLU". Writes c (may be NULL) and u. */
 static void conv_silu_channel(const double *x, const double *w, double b, int64_t L, int64_t K,
-                              double *c, double *u) {
+                              const double *hist, double *c, double *u) {
   for (int64_t t = 0; t < L; t++) {
     double acc = b;
-    for (int64_t k = 0; k < K; k++)
-      if (t - k >= 0) acc += w[k] * x[t - k];
+    for (int64_t k = 0; k < K; k++) {
+      if (t - k >= 0)
+        acc += w[k] * x[t - k];
+      else if (hist)
+        acc += w[k] * hist[k - t - 1]; /* x_{t-k} with t-k < 0 is history[k-t-1] */
+    }
     if (c) c[t] = acc;
     u[t] = ssm_oracle_silu(acc);
+  }
+}
+
+/* The K-1 newest pre-conv inputs after this chunk, newest-first, continuing the input history. */
+static void conv_hist_after(const double *x, const double *hist, int64_t L, int64_t K, double *out) {
+  for (int64_t j = 0; j < K - 1; j++) {
+    const int64_t t = L - 1 - j;
+    out[j] = (t >= 0) ? x[t] : (hist ? hist[j - L] : 0.0);
   }
 }
 
@@ -93,7 +113,7 @@ void ssm_oracle_conv1d_silu(const double *x, const double *w, const double *b, i
   for (int64_t bi = 0; bi < Bt; bi++)
     for (int64_t d = 0; d < Dn; d++) {
       const int64_t off = (bi * Dn + d) * L;
-      conv_silu_channel(x + off, w + d * K, b ? b[d] : 0.0, L, K, NULL, u + off);
+      conv_silu_channel(x + off, w + d * K, b ? b[d] : 0.0, L, K, NULL, NULL, u + off);
     }
 }
 
@@ -104,18 +124,23 @@ void ssm_oracle_conv1d_silu(const double *x, const double *w, const double *b, i
 static void fwd_channel(const double *x, const double *dt, const double *dt_bias,
                         const double *A_log, const double *B, const double *C, const double *D,
                         const double *z, const double *conv_w, const double *conv_b, int64_t Dn,
-                        int64_t N, int64_t L, int64_t K, int delta_softplus, int64_t bi, int64_t d,
-                        double *out, double *u_out, double *y_out, double *h, double *u) {
+                        int64_t N, int64_t L, int64_t K, int delta_softplus, int euler,
+                        const double *h0, const double *conv_hist, int64_t bi, int64_t d,
+                        double *out, double *u_out, double *y_out, double *h_last,
+                        double *conv_hist_out, double *h, double *u) {
   const int64_t off = (bi * Dn + d) * L;
   const double *Bb = B + bi * N * L, *Cb = C + bi * N * L;
+  const int64_t ch = bi * Dn + d;
+  const double *hist = (conv_hist && K > 1) ? conv_hist + ch * (K - 1) : NULL;
 
   /* u: conv + SiLU, or x itself when there is no conv. */
   if (conv_w)
-    conv_silu_channel(x + off, conv_w + d * K, conv_b ? conv_b[d] : 0.0, L, K, NULL, u);
+    conv_silu_channel(x + off, conv_w + d * K, conv_b ? conv_b[d] : 0.0, L, K, hist, NULL, u);
   else
     for (int64_t t = 0; t < L; t++) u[t] = x[off + t];
 
-  for (int64_t n = 0; n < N; n++) h[n] = 0.0; /* h_{-1} = 0 ([SSM]; [TL] zeroState) */
+  /* h_{-1} = 0 ([SSM]; [TL] zeroState), or the carried state */
+  for (int64_t n = 0; n < N; n++) h[n] = h0 ? h0[ch * N + n] : 0.0;
   for (int64_t t = 0; t < L; t++) {
     const double v = dt[off + t] + (dt_bias ? dt_bias[d] : 0.0);
     const double delta = delta_softplus ? ssm_oracle_softplus(v) : v;
@@ -124,6 +149,7 @@ static void fwd_channel(const double *x, const double *dt, const double *dt_bias
       const double A = -exp(A_log[d * N + n]); /* [TL] logA; [RT] A = -exp(A_log) */
       double Abar, Bbar;
       ssm_oracle_zoh(A, Bb[n * L + t], delta, &Abar, &Bbar);
+      if (euler) Bbar = delta * Bb[n * L + t]; /* [SSMK] mamba_selective_scan_step */
       h[n] = Abar * h[n] + Bbar * u[t]; /* [SSMK] ssm_recurrence_step */
       y += Cb[n * L + t] * h[n];        /* [SSMK] ssm_output_step */
     }
@@ -132,15 +158,21 @@ static void fwd_channel(const double *x, const double *dt, const double *dt_bias
     if (u_out) u_out[off + t] = u[t];
     out[off + t] = z ? y * ssm_oracle_silu(z[off + t]) : y; /* [TL] zProj gate; [RT] SiLU(z) */
   }
+  if (h_last)
+    for (int64_t n = 0; n < N; n++) h_last[ch * N + n] = h[n];
+  if (conv_hist_out && K > 1) conv_hist_after(x + off, hist, L, K, conv_hist_out + ch * (K - 1));
 }
 
-/* Whole forward. Nullable: dt_bias, D, z, conv_w (then x is u), conv_b, u_out, y_out (pre-gate
- * output including D*u). n_threads <= 0 means "all". Returns 0, or -1 on allocation failure. */
+/* Whole forward. Nullable: dt_bias, D, z, conv_w (then x is u), conv_b, h0 ((Bt, Dn, N) carried
+ * state), conv_hist ((Bt, Dn, K-1) carried inputs, newest-first), u_out, y_out (pre-gate output
+ * including D*u), h_last ((Bt, Dn, N) state after the chunk), conv_hist_out ((Bt, Dn, K-1)).
+ * n_threads <= 0 means "all". Returns 0, or -1 on allocation failure. */
 int ssm_oracle_fwd(const double *x, const double *dt, const double *dt_bias, const double *A_log,
                    const double *B, const double *C, const double *D, const double *z,
                    const double *conv_w, const double *conv_b, int64_t Bt, int64_t Dn, int64_t N,
-                   int64_t L, int64_t K, int delta_softplus, double *out, double *u_out,
-                   double *y_out, int n_threads) {
+                   int64_t L, int64_t K, int delta_softplus, int euler, const double *h0,
+                   const double *conv_hist, double *out, double *u_out, double *y_out,
+                   double *h_last, double *conv_hist_out, int n_threads) {
   int failed = 0;
   const int64_t channels = Bt * Dn;
 #ifdef _OPENMP
@@ -157,7 +189,8 @@ int ssm_oracle_fwd(const double *x, const double *dt, const double *dt_bias, con
     for (int64_t ch = 0; ch < channels; ch++)
       if (h && u)
         fwd_channel(x, dt, dt_bias, A_log, B, C, D, z, conv_w, conv_b, Dn, N, L, K,
-                    delta_softplus, ch / Dn, ch % Dn, out, u_out, y_out, h, u);
+                    delta_softplus, euler, h0, conv_hist, ch / Dn, ch % Dn, out, u_out, y_out,
+                    h_last, conv_hist_out, h, u);
     free(h);
     free(u);
   }
@@ -183,6 +216,14 @@ int ssm_oracle_fwd(const double *x, const double *dt, const double *dt_bias, con
  *   dv_t       = dDelta_t * s(v_t) (softplus) or dDelta_t;  ddt_t = dv_t;  ddt_bias += dv_t
  *   dc_t       = du_t * s(c_t)(1 + c_t(1 - s(c_t)))      (conv pre-activation)
  *   dx_j       = sum_k w[k] * dc_{j+k};  dw[k] = sum_t dc_t x_{t-k};  dconv_b = sum_t dc_t
+ *   dh0        = a_0 * lambda_0                          (gradient of the carried state)
+ *   dh_last (input) is the gradient arriving at the state after the chunk (from the next chunk's
+ *   dh0): it enters as lambda_{L-1} = dy C + dh_last. The carried inputs' output history needs no
+ *   such term here: its gradient is the next chunk's dhist added to dx of the last K-1 steps.
+ *   dhist_j    = sum_{k > j} w[k] * dc_{k-j-1}           (gradient of the carried inputs x_{-1-j})
+ *
+ * With euler = 1 (B-bar = Delta * B): bb = Delta B, dB_t[n] += lambda u Delta,
+ * dDelta_t = sum_n lambda (A a h_{t-1} + B u), dA_n += lambda Delta a h_{t-1}.
  *
  * Without a conv, dx = du. Every output is overwritten (not accumulated into). Nullable outputs
  * are skipped. Parallel over batch elements only; each batch element runs its channels in order
@@ -191,9 +232,11 @@ int ssm_oracle_fwd(const double *x, const double *dt, const double *dt_bias, con
 int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, const double *A_log,
                    const double *B, const double *C, const double *D, const double *z,
                    const double *conv_w, const double *conv_b, int64_t Bt, int64_t Dn, int64_t N,
-                   int64_t L, int64_t K, int delta_softplus, const double *dout, double *dx,
-                   double *ddt, double *dA_log, double *dB, double *dC, double *dD,
-                   double *ddt_bias, double *dz, double *dconv_w, double *dconv_b, int n_threads) {
+                   int64_t L, int64_t K, int delta_softplus, int euler, const double *h0,
+                   const double *conv_hist, const double *dout, const double *dh_last, double *dx, double *ddt,
+                   double *dA_log, double *dB, double *dC, double *dD, double *ddt_bias,
+                   double *dz, double *dconv_w, double *dconv_b, double *dh0, double *dconv_hist,
+                   int n_threads) {
   /* per-batch-element partials of the per-channel parameter gradients */
   const size_t nb = (size_t)(Bt > 0 ? Bt : 1);
   double *pA = (double *)calloc(nb * (size_t)(Dn * N), sizeof(double));
@@ -233,10 +276,12 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
       if (dCb) memset(dCb, 0, sizeof(double) * LN);
       for (int64_t d = 0; d < Dn; d++) {
         const int64_t off = (bi * Dn + d) * L;
+        const int64_t chn = bi * Dn + d;
         const double Dd = D ? D[d] : 0.0;
+        const double *hist = (conv_hist && K > 1) ? conv_hist + chn * (K - 1) : NULL;
         /* forward recompute with the whole trajectory kept */
         if (conv_w)
-          conv_silu_channel(x + off, conv_w + d * K, conv_b ? conv_b[d] : 0.0, L, K, c, u);
+          conv_silu_channel(x + off, conv_w + d * K, conv_b ? conv_b[d] : 0.0, L, K, hist, c, u);
         else
           for (int64_t t = 0; t < L; t++) u[t] = x[off + t];
         for (int64_t n = 0; n < N; n++) A[n] = -exp(A_log[d * N + n]);
@@ -248,8 +293,8 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
             const size_t i = (size_t)(t * N + n);
             a[i] = exp(dl[t] * A[n]);
             em1[i] = expm1(dl[t] * A[n]);
-            bb[i] = em1[i] / A[n] * Bb[n * L + t];
-            h[i] = a[i] * (t > 0 ? h[i - (size_t)N] : 0.0) + bb[i] * u[t];
+            bb[i] = euler ? dl[t] * Bb[n * L + t] : em1[i] / A[n] * Bb[n * L + t];
+            h[i] = a[i] * (t > 0 ? h[i - (size_t)N] : (h0 ? h0[chn * N + n] : 0.0)) + bb[i] * u[t];
             yt += Cb[n * L + t] * h[i];
           }
           y[t] = yt + Dd * u[t];
@@ -265,7 +310,10 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
           }
         }
         /* reverse-time adjoint recurrence */
-        for (int64_t n = 0; n < N; n++) { lam[n] = 0.0; dA[n] = 0.0; }
+        for (int64_t n = 0; n < N; n++) {
+          lam[n] = dh_last ? dh_last[chn * N + n] : 0.0;
+          dA[n] = 0.0;
+        }
         double accD = 0.0, accdtb = 0.0;
         for (int64_t t = L - 1; t >= 0; t--) {
           double du = Dd * dy[t];
@@ -273,16 +321,22 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
           accD += dy[t] * u[t];
           for (int64_t n = 0; n < N; n++) {
             const size_t i = (size_t)(t * N + n);
-            const double anext = (t + 1 < L) ? a[i + (size_t)N] : 0.0;
+            const double anext = (t + 1 < L) ? a[i + (size_t)N] : 1.0; /* lambda_L := dh_last */
             lam[n] = dy[t] * Cb[n * L + t] + anext * lam[n];
-            const double hprev = t > 0 ? h[i - (size_t)N] : 0.0;
+            const double hprev = t > 0 ? h[i - (size_t)N] : (h0 ? h0[chn * N + n] : 0.0);
             const double Bt_n = Bb[n * L + t];
             const double xx = dl[t] * A[n];
             if (dCb) dCb[n * L + t] += dy[t] * h[i];
-            if (dBb) dBb[n * L + t] += lam[n] * u[t] * em1[i] / A[n];
-            ddelta += lam[n] * a[i] * (A[n] * hprev + Bt_n * u[t]);
-            dA[n] += lam[n] * (hprev * dl[t] * a[i] +
-                               u[t] * Bt_n * (xx * a[i] - em1[i]) / (A[n] * A[n]));
+            if (euler) {
+              if (dBb) dBb[n * L + t] += lam[n] * u[t] * dl[t];
+              ddelta += lam[n] * (A[n] * a[i] * hprev + Bt_n * u[t]);
+              dA[n] += lam[n] * dl[t] * a[i] * hprev;
+            } else {
+              if (dBb) dBb[n * L + t] += lam[n] * u[t] * em1[i] / A[n];
+              ddelta += lam[n] * a[i] * (A[n] * hprev + Bt_n * u[t]);
+              dA[n] += lam[n] * (hprev * dl[t] * a[i] +
+                                 u[t] * Bt_n * (xx * a[i] - em1[i]) / (A[n] * A[n]));
+            }
             du += lam[n] * bb[i];
           }
           const double dv = delta_softplus ? ddelta * ssm_oracle_sigmoid(v[t]) : ddelta;
@@ -295,9 +349,19 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
             dc[t] = du;
           }
         }
+        /* gradient of the carried state: h0 enters only through h_0 = a_0 h0 + ... */
+        if (dh0)
+          for (int64_t n = 0; n < N; n++) dh0[chn * N + n] = (L > 0) ? a[(size_t)n] * lam[n] : lam[n];
         /* conv backward (or identity) */
         if (conv_w) {
           const double *w = conv_w + d * K;
+          if (dconv_hist && K > 1)
+            for (int64_t j = 0; j < K - 1; j++) {
+              double acc = 0.0; /* x_{-1-j} feeds c_t through tap k = t + 1 + j */
+              for (int64_t t = 0; t < L; t++)
+                if (t + 1 + j < K) acc += w[t + 1 + j] * dc[t];
+              dconv_hist[chn * (K - 1) + j] = acc;
+            }
           if (dx)
             for (int64_t j = 0; j < L; j++) {
               double acc = 0.0;
@@ -308,8 +372,12 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
           double accb = 0.0;
           for (int64_t k = 0; k < K; k++) {
             double acc = 0.0;
-            for (int64_t t = 0; t < L; t++)
-              if (t - k >= 0) acc += dc[t] * x[off + t - k];
+            for (int64_t t = 0; t < L; t++) {
+              if (t - k >= 0)
+                acc += dc[t] * x[off + t - k];
+              else if (hist)
+                acc += dc[t] * hist[k - t - 1];
+            }
             pcw[(size_t)bi * (size_t)(Dn * K) + (size_t)(d * K + k)] = acc;
           }
           for (int64_t t = 0; t < L; t++) accb += dc[t];

@@ -22,8 +22,8 @@
 namespace ssm {
 
 // Shared-memory plan of one CTA (all offsets in bytes, 16-byte aligned).
-template <int G, int NS, typename Tin> struct FwdSmem {
-  static constexpr int CH = kThreads / G;    // channels per CTA
+template <int G, int NS, typename Tin, int NT> struct FwdSmem {
+  static constexpr int CH = NT / G;          // channels per CTA
   static constexpr int NP = G * NS;          // padded state count
   static constexpr int XS = kPre + kT;       // x row length (elements)
   static constexpr int BS = NP + 4;          // Bs/Cs row stride (floats)
@@ -40,10 +40,10 @@ template <int G, int NS, typename Tin> struct FwdSmem {
   static constexpr size_t bytes = yp_off + sizeof(float) * CH * YC;
 };
 
-template <int G, int NS, typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads, 4)
+template <int G, int NS, typename Tin, typename Tout, int NT>
+__global__ void __launch_bounds__(NT, 512 / NT)
 ssm_fwd_kernel(const FwdParams p) {
-  using S = FwdSmem<G, NS, Tin>;
+  using S = FwdSmem<G, NS, Tin, NT>;
   constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G;
   constexpr bool PRECISE = sizeof(Tin) == 4;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -104,7 +104,7 @@ ssm_fwd_kernel(const FwdParams p) {
   const int n_rows = (int)imin64(NP, N);
 
   // zero the conv-halo prefixes of both x buffers (the sequence starts from zero history)
-  for (int i = tid; i < 2 * CH * kPre; i += kThreads) {
+  for (int i = tid; i < 2 * CH * kPre; i += NT) {
     const int r = i / kPre, k = i % kPre;
     xs[r * S::XS + k] = zero_val<Tin>();
   }
@@ -112,13 +112,13 @@ ssm_fwd_kernel(const FwdParams p) {
   const int64_t n_stages = (L + kT - 1) / kT;
   auto issue = [&](int64_t stage, int buf) {
     const int64_t t0 = stage * kT;
-    stage_rows<Tin, CH>(xs + buf * CH * S::XS + kPre, S::XS, gx, L, rows_valid, t0, L, vec);
-    stage_rows<Tin, CH>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
-    if (has_z) stage_rows<Tin, CH>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
+    stage_rows<Tin, CH, kT, NT>(xs + buf * CH * S::XS + kPre, S::XS, gx, L, rows_valid, t0, L, vec);
+    stage_rows<Tin, CH, kT, NT>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
+    if (has_z) stage_rows<Tin, CH, kT, NT>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
     cp_async_commit();
   };
 
-  BCStager<Tin, NP> bc;
+  BCStager<Tin, NP, NT> bc;
   if (n_stages > 0) {
     issue(0, 0);
     bc.load(gB, gC, n_rows, 0, L, vec);
@@ -322,16 +322,21 @@ LaneLayout choose_layout(int64_t N, int64_t channels) {
 
 int channels_per_cta(const LaneLayout &lay) { return kThreads / lay.G; }
 
+// Threads per forward CTA (a template parameter of the kernel; 128 measured best on the
+// 4x4096x16x4096 shape, 64 was no faster).
+constexpr int kFwdThreads = 128;
+
 template <int G, int NS, typename Tin, typename Tout>
 static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
-  using S = FwdSmem<G, NS, Tin>;
-  auto kern = ssm_fwd_kernel<G, NS, Tin, Tout>;
+  constexpr int NT = kFwdThreads;
+  using S = FwdSmem<G, NS, Tin, NT>;
+  auto kern = ssm_fwd_kernel<G, NS, Tin, Tout, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
   if (e != cudaSuccess) return e;
   const int64_t n_dtiles = (p.Dn + S::CH - 1) / S::CH;
   const int64_t grid = n_dtiles * p.Bt;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)grid, kThreads, S::bytes, stream>>>(p);
+  kern<<<(unsigned)grid, NT, S::bytes, stream>>>(p);
   return cudaGetLastError();
 }
 

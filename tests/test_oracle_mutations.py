@@ -33,6 +33,11 @@ MUTATIONS = [
     ("bwd_gate_derivative", "s * (1.0 + zz * (1.0 - s))", "s"),
     ("bwd_conv_dx_taps", "acc += w[k] * dc[j + k];", "acc += w[K - 1 - k] * dc[j + k];"),
     ("bwd_dAlog_chain", "= dA[n] * A[n];", "= dA[n];"),
+    ("history_off_by_one", "acc += w[k] * hist[k - t - 1];", "acc += w[k] * hist[k - t];"),
+    ("euler_missing_delta", "if (euler) Bbar = delta * Bb[n * L + t];", "if (euler) Bbar = Bb[n * L + t];"),
+    ("dh0_missing_decay", "? a[(size_t)n] * lam[n] : lam[n];", "? lam[n] : lam[n];"),
+    ("dh_last_decayed", "a[i + (size_t)N] : 1.0;", "a[i + (size_t)N] : 0.0;"),
+    ("bwd_euler_dB", "dBb[n * L + t] += lam[n] * u[t] * dl[t];", "dBb[n * L + t] += lam[n] * u[t];"),
 ]
 
 
@@ -40,18 +45,31 @@ def _pin_functions():
     return [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
 
 
+def _param_sets(fn):
+    """Expand a pin's @pytest.mark.parametrize marks into keyword-argument dicts."""
+    import itertools
+    sets = [{}]
+    for m in getattr(fn, "pytestmark", []):
+        if m.name != "parametrize":
+            continue
+        names = [n.strip() for n in m.args[0].split(",")] if isinstance(m.args[0], str) else list(m.args[0])
+        values = [v if len(names) > 1 else (v,) for v in m.args[1]]
+        sets = [dict(s, **dict(zip(names, v))) for s, v in itertools.product(sets, values)]
+    return sets
+
+
 def _run_pins(gold):
     failed = []
     for fn in _pin_functions():
-        try:
+        for kw in _param_sets(fn):
             if "gold" in fn.__code__.co_varnames[:fn.__code__.co_argcount]:
-                fn(gold)
-            else:
-                fn()
-        except AssertionError:
-            failed.append(fn.__name__)
-        except Exception:
-            failed.append(fn.__name__ + "(error)")
+                kw = dict(kw, gold=gold)
+            try:
+                fn(**kw)
+            except AssertionError:
+                failed.append(fn.__name__)
+            except Exception:
+                failed.append(fn.__name__ + "(error)")
     return failed
 
 

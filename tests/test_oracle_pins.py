@@ -356,3 +356,116 @@ def test_backward_without_conv_and_gate_and_multibatch():
         xm.reshape(-1)[i] -= 1e-6
         fd.reshape(-1)[i] = (loss(xp) - loss(xm)) / 2e-6
     np.testing.assert_allclose(g["dx"], fd, rtol=1e-6, atol=1e-8)
+
+
+# ---- state carry across chunks ("Selective Mamba": State, step, runArray) and the Euler step ----
+
+def _carry_case(L=37, Dn=3, N=4, K=4, seed=31, euler=False):
+    w = wl.shaped("fd_slice", Dn=Dn, N=N, L=L, K=K, seed=seed)
+    a = wl.generate(w)
+    kw = dict(D=a["D"], z=a["z"], dt_bias=a["dt_bias"], conv_w=a["conv_w"], conv_b=a["conv_b"],
+              euler=euler)
+    return a, kw
+
+
+@pytest.mark.parametrize("split", [0, 1, 2, 3, 16, 36, 37])
+@pytest.mark.parametrize("euler", [False, True])
+def test_chunked_continuation_equals_one_pass(split, euler):
+    # runArray: a chunk returns the hidden state and the conv history the next chunk needs; chunk
+    # boundaries change nothing, so two chunks reproduce one pass exactly.
+    a, kw = _carry_case(euler=euler)
+    whole, ex = oracle.fwd(a["x"], a["dt"], a["A_log"], a["B"], a["C"], want_state=True, **kw)
+    s1 = slice(0, split)
+    s2 = slice(split, None)
+    o1, e1 = oracle.fwd(a["x"][..., s1], a["dt"][..., s1], a["A_log"], a["B"][..., s1],
+                        a["C"][..., s1], want_state=True, **dict(kw, z=a["z"][..., s1]))
+    o2, e2 = oracle.fwd(a["x"][..., s2], a["dt"][..., s2], a["A_log"], a["B"][..., s2],
+                        a["C"][..., s2], want_state=True, h0=e1["h_last"], conv_hist=e1["conv_hist"],
+                        **dict(kw, z=a["z"][..., s2]))
+    assert np.array_equal(np.concatenate([o1, o2], axis=-1), whole)
+    assert np.array_equal(e2["h_last"], ex["h_last"])
+    assert np.array_equal(e2["conv_hist"], ex["conv_hist"])
+
+
+def test_empty_chunk_preserves_state():
+    a, kw = _carry_case()
+    rng = np.random.default_rng(4)
+    h0 = rng.standard_normal((1, 3, 4))
+    hist = rng.standard_normal((1, 3, 3))
+    e = a["x"][..., :0]
+    _, ex = oracle.fwd(e, e, a["A_log"], a["B"][..., :0], a["C"][..., :0], want_state=True,
+                       h0=h0, conv_hist=hist, **dict(kw, z=e))
+    assert np.array_equal(ex["h_last"], h0)
+    assert np.array_equal(ex["conv_hist"], hist)
+
+
+def test_single_token_steps_equal_one_pass():
+    # step: one token at a time with the carried state reproduces the sequence.
+    a, kw = _carry_case(L=12)
+    whole = oracle.fwd(a["x"], a["dt"], a["A_log"], a["B"], a["C"], **kw)
+    h, hist, outs = None, None, []
+    for t in range(12):
+        s = slice(t, t + 1)
+        o, ex = oracle.fwd(a["x"][..., s], a["dt"][..., s], a["A_log"], a["B"][..., s],
+                           a["C"][..., s], want_state=True, h0=h, conv_hist=hist,
+                           **dict(kw, z=a["z"][..., s]))
+        h, hist = ex["h_last"], ex["conv_hist"]
+        outs.append(o)
+    assert np.array_equal(np.concatenate(outs, axis=-1), whole)
+
+
+def test_euler_first_step_worked_value(gold):
+    # "Sequence and state-space models": mamba_selective_scan_step gives h_1 = 1.0 exactly.
+    g = gold["euler_h1"]
+    y = oracle.fwd(np.array([[[g["x"]]]]), np.array([[[g["delta"]]]]), np.zeros((1, 1)),
+                   np.array([[[g["B"]]]]), np.ones((1, 1, 1)), D=np.zeros(1), delta_softplus=False,
+                   euler=True)
+    assert y[0, 0, 0] == g["value"]
+
+
+def test_euler_approaches_exact_zoh_for_small_steps():
+    # (A-bar - 1)/A = Delta (1 + Delta A / 2 + ...): the two discretisations agree to O(Delta A).
+    for delta in [1e-1, 1e-2, 1e-3]:
+        ye = oracle.fwd(np.ones((1, 1, 1)), np.full((1, 1, 1), delta), np.zeros((1, 1)),
+                        np.ones((1, 1, 1)), np.ones((1, 1, 1)), delta_softplus=False, euler=True)
+        yz = oracle.fwd(np.ones((1, 1, 1)), np.full((1, 1, 1), delta), np.zeros((1, 1)),
+                        np.ones((1, 1, 1)), np.ones((1, 1, 1)), delta_softplus=False)
+        rel = (ye - yz)[0, 0, 0] / yz[0, 0, 0]
+        assert abs(rel - delta / 2) < delta * delta
+
+
+@pytest.mark.parametrize("euler", [False, True])
+def test_carried_state_gradients_match_finite_differences(euler):
+    # gradients of every input including h0, the conv history, and an incoming dh_last
+    a, kw = _carry_case(L=9, Dn=2, N=3, euler=euler)
+    rng = np.random.default_rng(9)
+    h0 = rng.standard_normal((1, 2, 3))
+    hist = rng.standard_normal((1, 2, 3))
+    dout = rng.standard_normal(a["x"].shape)
+    dhl = rng.standard_normal((1, 2, 3))
+    p = {"x": np.array(a["x"], float), "dt": np.array(a["dt"], float), "B": np.array(a["B"], float),
+         "C": np.array(a["C"], float), "A_log": np.array(a["A_log"], float),
+         "conv_w": np.array(a["conv_w"], float), "h0": h0.copy(), "conv_hist": hist.copy()}
+
+    def loss():
+        o, ex = oracle.fwd(p["x"], p["dt"], p["A_log"], p["B"], p["C"], want_state=True,
+                           h0=p["h0"], conv_hist=p["conv_hist"],
+                           **dict(kw, conv_w=p["conv_w"]))
+        return float(np.sum(o * dout) + np.sum(ex["h_last"] * dhl))
+    g = oracle.bwd(p["x"], p["dt"], p["A_log"], p["B"], p["C"], dout, h0=h0, conv_hist=hist,
+                   dh_last=dhl, **dict(kw, conv_w=p["conv_w"]))
+    names = {"x": "dx", "dt": "ddt", "B": "dB", "C": "dC", "A_log": "dA_log", "conv_w": "dconv_w",
+             "h0": "dh0", "conv_hist": "dconv_hist"}
+    for k, gk in names.items():
+        flat = p[k].reshape(-1)
+        fd = np.zeros(flat.size)
+        for i in range(flat.size):
+            old = flat[i]
+            flat[i] = old + 1e-6
+            lp = loss()
+            flat[i] = old - 1e-6
+            lm = loss()
+            flat[i] = old
+            fd[i] = (lp - lm) / 2e-6
+        np.testing.assert_allclose(g[gk].reshape(-1), fd, rtol=1e-6, atol=1e-7 * max(1, np.abs(fd).max()),
+                                   err_msg=gk)
