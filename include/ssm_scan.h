@@ -68,6 +68,12 @@ typedef enum ssm_status {
 
 typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
 
+/* Input discretisation. SSM_ZOH: B_bar = (A_bar - 1)/A * B, the exact zero-order hold
+ * ("Sequence and state-space models", ssm_discretize_b). SSM_EULER: B_bar = Delta * B, Mamba's
+ * first-order simplification ("Sequence and state-space models", mamba_selective_scan_step;
+ * "Selective Mamba", step). A_bar = exp(Delta * A) in both. */
+typedef enum ssm_discretization { SSM_ZOH = 0, SSM_EULER = 1 } ssm_discretization;
+
 /* Time steps between saved states (chunk_states) and of the backward's recompute blocks. */
 #define SSM_STATE_CHUNK 16
 
@@ -100,6 +106,16 @@ typedef struct ssm_fwd_args {
   int32_t in_dtype;      /* ssm_dtype of x, dt, z, B, C */
   int32_t out_dtype;     /* ssm_dtype of out and u_out */
   int32_t delta_softplus;/* 1: Delta = softplus(dt + dt_bias); 0: Delta = dt + dt_bias */
+  /* State carried between calls ("Selective Mamba", State / runArray): a sequence processed as
+   * consecutive chunks, each call given the previous call's h_last and conv_hist_out, produces
+   * exactly the outputs of one call over the whole sequence. */
+  const float *h0;       /* device (Bt, Dn, N) fp32 or NULL (= 0): the state before step 0 */
+  const void *conv_hist; /* device (Bt, Dn, K-1) in_dtype or NULL (= 0): the K-1 pre-conv inputs
+                            before step 0, newest-first (ignored without conv_w) */
+  float *h_last;         /* device (Bt, Dn, N) fp32 or NULL: the state after step L-1 */
+  void *conv_hist_out;   /* device (Bt, Dn, K-1) in_dtype or NULL: the K-1 newest pre-conv inputs
+                            after this call, newest-first (may alias conv_hist) */
+  int32_t discretization;/* ssm_discretization */
 } ssm_fwd_args;
 
 /*
@@ -137,6 +153,12 @@ typedef struct ssm_bwd_args {
                                  `stream` just before the main backward kernel, [1] just after it
                                  (before the cross-tile reductions); lets a caller time the
                                  kernel alone. Recording does not synchronise. */
+  const float *dh_last;  /* (Bt, Dn, N) or NULL: gradient arriving at fwd.h_last (the next
+                            chunk's dh0 when chunks are chained) */
+  float *dh0;            /* (Bt, Dn, N) or NULL: gradient w.r.t. fwd.h0 */
+  float *dconv_hist;     /* (Bt, Dn, K-1) or NULL: gradient w.r.t. fwd.conv_hist. When chunks are
+                            chained, add it to the previous chunk's dx over its last K-1 steps
+                            (entry j belongs to step L-1-j). */
 } ssm_bwd_args;
 
 /* Bytes of device scratch ssm_scan_bwd needs for these arguments (0 for an empty problem). */
@@ -149,6 +171,34 @@ size_t ssm_bwd_workspace_size(const ssm_bwd_args *args);
  * are reduced in a fixed order. Errors as ssm_scan_fwd, plus SSM_ERR_WORKSPACE.
  */
 ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream);
+
+/*
+ * Single-token decode step ("Selective Mamba", step): advance every channel by one token, reading
+ * and updating the carried state in place. Same arithmetic as ssm_scan_fwd with L = 1, h0 =
+ * h_last = h and conv_hist = conv_hist_out = conv_hist, without the scan machinery.
+ */
+typedef struct ssm_step_args {
+  const void *x;        /* device (Bt, Dn) in_dtype: this token's pre-conv input (u without conv) */
+  const void *dt;       /* device (Bt, Dn) in_dtype */
+  const float *dt_bias; /* device [Dn] or NULL */
+  const float *A_log;   /* device [Dn, N] */
+  const void *B;        /* device (Bt, N) in_dtype */
+  const void *C;        /* device (Bt, N) in_dtype */
+  const float *D;       /* device [Dn] or NULL */
+  const void *z;        /* device (Bt, Dn) in_dtype or NULL */
+  const float *conv_w;  /* device [Dn, K] or NULL */
+  const float *conv_b;  /* device [Dn] or NULL */
+  float *h;             /* device (Bt, Dn, N) fp32: state, read then overwritten */
+  void *conv_hist;      /* device (Bt, Dn, K-1) in_dtype: history, read then overwritten (with a
+                           conv; may be NULL without one) */
+  void *out;            /* device (Bt, Dn) out_dtype */
+  int64_t Bt, Dn, N;
+  int32_t K, in_dtype, out_dtype, delta_softplus, discretization;
+} ssm_step_args;
+
+/* One decode step. Errors: SSM_ERR_NULL, SSM_ERR_SHAPE, SSM_ERR_ALIGN, SSM_ERR_DTYPE,
+ * SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA. Bt = 0 is a no-op. */
+ssm_status ssm_scan_step(const ssm_step_args *args, void *stream);
 
 /* Size of the scratch array built into the library for ssm_scan_bwd_noalloc (64 MiB). */
 #define SSM_NOALLOC_SCRATCH_BYTES (64u << 20)

@@ -9,6 +9,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 
 SSM_F32, SSM_BF16 = 0, 1
+SSM_ZOH, SSM_EULER = 0, 1
 SSM_STATE_CHUNK = 16
 SSM_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -28,6 +29,8 @@ class FwdArgs(ctypes.Structure):
         ("Bt", ctypes.c_int64), ("Dn", ctypes.c_int64), ("N", ctypes.c_int64), ("L", ctypes.c_int64),
         ("K", ctypes.c_int32), ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
         ("delta_softplus", ctypes.c_int32),
+        ("h0", ctypes.c_void_p), ("conv_hist", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
+        ("conv_hist_out", ctypes.c_void_p), ("discretization", ctypes.c_int32),
     ]
 
 
@@ -39,6 +42,20 @@ class BwdArgs(ctypes.Structure):
         ("dD", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p), ("dconv_w", ctypes.c_void_p),
         ("dconv_b", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("timing_events", ctypes.c_void_p),
+        ("dh_last", ctypes.c_void_p), ("dh0", ctypes.c_void_p), ("dconv_hist", ctypes.c_void_p),
+    ]
+
+
+class StepArgs(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+        ("A_log", ctypes.c_void_p), ("B", ctypes.c_void_p), ("C", ctypes.c_void_p),
+        ("D", ctypes.c_void_p), ("z", ctypes.c_void_p), ("conv_w", ctypes.c_void_p),
+        ("conv_b", ctypes.c_void_p), ("h", ctypes.c_void_p), ("conv_hist", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("Bt", ctypes.c_int64), ("Dn", ctypes.c_int64),
+        ("N", ctypes.c_int64), ("K", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
+        ("out_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+        ("discretization", ctypes.c_int32),
     ]
 
 
@@ -49,6 +66,7 @@ SIGNATURES = [
     ("ssm_bwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(BwdArgs)]),
     ("ssm_scan_bwd", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_bwd_noalloc", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
+    ("ssm_scan_step", ctypes.c_int, [ctypes.POINTER(StepArgs), ctypes.c_void_p]),
     ("ssm_conv1d_silu", ctypes.c_int,
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
       ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,

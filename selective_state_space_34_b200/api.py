@@ -46,7 +46,11 @@ def ssm_num_state_chunks(L: int) -> int:
     return int(_abi.load().ssm_num_state_chunks(int(L)))
 
 
-def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype):
+_DISC = {"zoh": _abi.SSM_ZOH, "euler": _abi.SSM_EULER}
+
+
+def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
+              discretization="zoh", h0=None, conv_hist=None):
     for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
         _need_cuda(n, t)
     if x.dtype not in _DT:
@@ -85,15 +89,32 @@ def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
     a.Bt, a.Dn, a.N, a.L, a.K = Bt, Dn, N, L, K
     a.in_dtype, a.out_dtype = _DT[act], _DT[od]
     a.delta_softplus = 1 if delta_softplus else 0
+    if discretization not in _DISC:
+        raise ValueError("discretization must be 'zoh' or 'euler'")
+    a.discretization = _DISC[discretization]
+    if h0 is not None:
+        _opt("h0", h0, torch.float32)
+        if tuple(h0.shape) != (Bt, Dn, N):
+            raise ValueError("h0 must be (Bt, Dn, N)")
+        a.h0 = _ptr(h0)
+    if conv_hist is not None:
+        _opt("conv_hist", conv_hist, act)
+        if conv_w is None or tuple(conv_hist.shape) != (Bt, Dn, K - 1):
+            raise ValueError("conv_hist must be (Bt, Dn, K-1) and needs conv_w")
+        a.conv_hist = _ptr(conv_hist)
     return a, od
 
 
 def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, conv_b=None,
                  delta_softplus: bool = True, out_dtype=None, save_states: bool = False,
-                 return_u: bool = False, out: Optional[torch.Tensor] = None):
+                 return_u: bool = False, out: Optional[torch.Tensor] = None,
+                 discretization: str = "zoh", h0=None, conv_hist=None, return_state: bool = False):
     """Fused forward. Returns ``out`` or a dict with ``out`` and, when asked, ``chunk_states``
-    ((Bt, Dn, ceil(L/16), N) fp32, for ssm_scan_bwd) and ``u`` (the scan input)."""
-    a, od = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype)
+    ((Bt, Dn, ceil(L/16), N) fp32, for ssm_scan_bwd), ``u`` (the scan input), and ``h_last`` /
+    ``conv_hist`` (the state to carry into the next chunk). ``h0`` / ``conv_hist`` carry the state
+    in from a previous chunk; ``discretization`` is "zoh" (exact) or "euler" (Delta * B)."""
+    a, od = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
+                      discretization, h0, conv_hist)
     Bt, Dn, L = x.shape
     N = A_log.shape[1]
     if out is None:
@@ -110,14 +131,23 @@ def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, 
         u = torch.empty((Bt, Dn, L), dtype=od, device=x.device)
         a.u_out = _ptr(u)
         res["u"] = u
+    if return_state:
+        hl = torch.empty((Bt, Dn, N), dtype=torch.float32, device=x.device)
+        a.h_last = _ptr(hl)
+        res["h_last"] = hl
+        if conv_w is not None and conv_w.shape[1] > 1:
+            ch = torch.empty((Bt, Dn, conv_w.shape[1] - 1), dtype=x.dtype, device=x.device)
+            a.conv_hist_out = _ptr(ch)
+            res["conv_hist"] = ch
     lib = _abi.load()
     _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(a), _stream_handle(x.device)))
-    return res if (save_states or return_u) else out
+    return res if (save_states or return_u or return_state) else out
 
 
 def _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
-                chunk_states):
-    a, _ = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, None)
+                chunk_states, discretization="zoh", h0=None, conv_hist=None, dh_last=None):
+    a, _ = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, None,
+                     discretization, h0, conv_hist)
     _need_cuda("dout", dout)
     if dout.dtype != x.dtype or dout.shape != x.shape:
         raise ValueError("dout must match x in shape and dtype")
@@ -126,6 +156,9 @@ def _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_s
     bw.fwd = a
     bw.dout = _ptr(dout)
     bw.chunk_states = _ptr(chunk_states)
+    if dh_last is not None:
+        _opt("dh_last", dh_last, torch.float32)
+        bw.dh_last = _ptr(dh_last)
     return bw
 
 
@@ -139,14 +172,15 @@ def ssm_bwd_workspace_size(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=Non
 def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None,
                  conv_b=None, delta_softplus: bool = True, chunk_states=None,
                  workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None,
-                 timing_events=None):
+                 timing_events=None, discretization: str = "zoh", h0=None, conv_hist=None,
+                 dh_last=None, state_grads: bool = False):
     """Backward. Returns a dict of fp32 gradients: dx, ddt, dA_log, dB, dC, and dD / ddt_bias /
     dz / dconv_w / dconv_b where the corresponding input exists. ``workspace`` (uint8, at least
     ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call.
     ``timing_events``: optional pair of recorded-once torch.cuda.Event(enable_timing=True); the
     library records them just before and just after its main backward kernel."""
     bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
-                     chunk_states)
+                     chunk_states, discretization, h0, conv_hist, dh_last)
     Bt, Dn, L = x.shape
     N = A_log.shape[1]
     dev = x.device
@@ -164,6 +198,10 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
         if conv_w is not None:
             grads["dconv_w"] = torch.empty(tuple(conv_w.shape), **f32)
             grads["dconv_b"] = torch.empty((Dn,), **f32)
+        if state_grads or h0 is not None or dh_last is not None:
+            grads["dh0"] = torch.empty((Bt, Dn, N), **f32)
+        if conv_w is not None and conv_w.shape[1] > 1 and (state_grads or conv_hist is not None):
+            grads["dconv_hist"] = torch.empty((Bt, Dn, conv_w.shape[1] - 1), **f32)
     for k, v in grads.items():
         _opt(k, v, torch.float32)
         setattr(bw, k, _ptr(v))
@@ -186,6 +224,45 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
         bw.timing_events = ctypes.cast(ev_arr, ctypes.c_void_p)
     _abi.check("ssm_scan_bwd", lib.ssm_scan_bwd(ctypes.byref(bw), _stream_handle(dev)))
     return grads
+
+
+def ssm_scan_step(x, dt, A_log, B, C, h, conv_hist=None, D=None, z=None, dt_bias=None,
+                  conv_w=None, conv_b=None, delta_softplus: bool = True, out_dtype=None,
+                  discretization: str = "zoh", out: Optional[torch.Tensor] = None):
+    """One decode step. x, dt, z: (Bt, Dn); B, C: (Bt, N); h: (Bt, Dn, N) fp32 and conv_hist:
+    (Bt, Dn, K-1) are read and updated in place. Returns the output (Bt, Dn)."""
+    for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C), ("h", h)):
+        _need_cuda(n, t)
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    act = x.dtype
+    for n, t in (("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != act:
+            raise TypeError("%s must have the activation dtype %s" % (n, act))
+    _opt("z", z, act)
+    _opt("conv_hist", conv_hist, act)
+    for n, t in (("A_log", A_log), ("D", D), ("dt_bias", dt_bias), ("conv_w", conv_w),
+                 ("conv_b", conv_b), ("h", h)):
+        _opt(n, t, torch.float32)
+    Bt, Dn = x.shape
+    N = A_log.shape[1]
+    if tuple(h.shape) != (Bt, Dn, N) or tuple(B.shape) != (Bt, N) or tuple(C.shape) != (Bt, N):
+        raise ValueError("h must be (Bt, Dn, N); B, C (Bt, N)")
+    od = act if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((Bt, Dn), dtype=od, device=x.device)
+    a = _abi.StepArgs()
+    a.x, a.dt, a.dt_bias, a.A_log, a.B, a.C = _ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log), _ptr(B), _ptr(C)
+    a.D, a.z, a.conv_w, a.conv_b = _ptr(D), _ptr(z), _ptr(conv_w), _ptr(conv_b)
+    a.h, a.conv_hist, a.out = _ptr(h), _ptr(conv_hist), _ptr(out)
+    a.Bt, a.Dn, a.N = Bt, Dn, N
+    a.K = int(conv_w.shape[1]) if conv_w is not None else 0
+    a.in_dtype, a.out_dtype = _DT[act], _DT[od]
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.discretization = _DISC[discretization]
+    lib = _abi.load()
+    _abi.check("ssm_scan_step", lib.ssm_scan_step(ctypes.byref(a), _stream_handle(x.device)))
+    return out
 
 
 def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = None):

@@ -32,6 +32,7 @@ bool mul_ok(int64_t a, int64_t b, int64_t *out) {
 ssm_status check_fwd(const ssm_fwd_args *a, bool need_out, bool *empty) {
   if (!a) return SSM_ERR_NULL;
   if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
+  if (a->discretization != SSM_ZOH && a->discretization != SSM_EULER) return SSM_ERR_UNSUPPORTED;
   if (a->Bt < 0 || a->Dn < 0 || a->N < 0 || a->L < 0) return SSM_ERR_SHAPE;
   if (a->Dn == 0 || a->N == 0) return SSM_ERR_SHAPE;  // empty internal axes are rejected
   if (a->conv_w && a->K <= 0) return SSM_ERR_SHAPE;
@@ -49,10 +50,32 @@ ssm_status check_fwd(const ssm_fwd_args *a, bool need_out, bool *empty) {
   for (const void *p : in_ptrs)
     if (p && !aligned(p, ei)) return SSM_ERR_ALIGN;
   if ((a->out && !aligned(a->out, eo)) || (a->u_out && !aligned(a->u_out, eo))) return SSM_ERR_ALIGN;
-  const void *f32_ptrs[6] = {a->dt_bias, a->A_log, a->D, a->conv_w, a->conv_b, a->chunk_states};
+  const void *f32_ptrs[8] = {a->dt_bias, a->A_log, a->D, a->conv_w, a->conv_b, a->chunk_states,
+                             a->h0, a->h_last};
   for (const void *p : f32_ptrs)
     if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  if ((a->conv_hist && !aligned(a->conv_hist, ei)) || (a->conv_hist_out && !aligned(a->conv_hist_out, ei)))
+    return SSM_ERR_ALIGN;
   return SSM_OK;
+}
+
+// An empty chunk keeps the carried state ("Selective Mamba", runArray): copy it through.
+cudaError_t carry_through_empty(const ssm_fwd_args *a, cudaStream_t s) {
+  if (a->Bt <= 0) return cudaSuccess;
+  const size_t nh = sizeof(float) * (size_t)(a->Bt * a->Dn * a->N);
+  cudaError_t e = cudaSuccess;
+  if (a->h_last) {
+    e = a->h0 ? (a->h0 == a->h_last ? cudaSuccess : cudaMemcpyAsync(a->h_last, a->h0, nh, cudaMemcpyDeviceToDevice, s))
+              : cudaMemsetAsync(a->h_last, 0, nh, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (a->conv_w && a->K > 1 && a->conv_hist_out) {
+    const size_t nc = dtype_size(a->in_dtype) * (size_t)(a->Bt * a->Dn * (a->K - 1));
+    e = a->conv_hist ? (a->conv_hist == a->conv_hist_out ? cudaSuccess
+                                                         : cudaMemcpyAsync(a->conv_hist_out, a->conv_hist, nc, cudaMemcpyDeviceToDevice, s))
+                     : cudaMemsetAsync(a->conv_hist_out, 0, nc, s);
+  }
+  return e;
 }
 
 // 16-byte staging / vector stores are allowed when every row starts on a 16-byte boundary.
@@ -90,6 +113,11 @@ ssm::FwdParams make_fwd_params(const ssm_fwd_args *a, int vec) {
   p.K = a->conv_w ? a->K : 0;
   p.delta_softplus = a->delta_softplus ? 1 : 0;
   p.vec = vec;
+  p.euler = a->discretization == SSM_EULER ? 1 : 0;
+  p.h0 = a->h0;
+  p.conv_hist = a->conv_w ? a->conv_hist : nullptr;
+  p.h_last = a->h_last;
+  p.conv_hist_out = a->conv_w ? a->conv_hist_out : nullptr;
   return p;
 }
 
@@ -121,7 +149,8 @@ int ssm_last_cuda_error(void) { return g_last_cuda_error; }
 ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream) {
   bool empty = false;
   ssm_status st = check_fwd(args, true, &empty);
-  if (st != SSM_OK || empty) return st;
+  if (st != SSM_OK) return st;
+  if (empty) return cuda_status(carry_through_empty(args, static_cast<cudaStream_t>(stream)));
   const ssm::FwdParams p = make_fwd_params(args, vec_ok(args, nullptr, 0));
   return cuda_status(ssm::launch_fwd(p, args->in_dtype == SSM_BF16, args->out_dtype == SSM_BF16,
                                      static_cast<cudaStream_t>(stream)));
@@ -147,6 +176,51 @@ ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *
                                              static_cast<cudaStream_t>(stream)));
 }
 
+ssm_status ssm_scan_step(const ssm_step_args *a, void *stream) {
+  if (!a) return SSM_ERR_NULL;
+  if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
+  if (a->discretization != SSM_ZOH && a->discretization != SSM_EULER) return SSM_ERR_UNSUPPORTED;
+  if (a->Bt < 0 || a->Dn <= 0 || a->N <= 0) return SSM_ERR_SHAPE;
+  if (a->conv_w && a->K <= 0) return SSM_ERR_SHAPE;
+  if (a->N > 64 || (a->conv_w && a->K > 4)) return SSM_ERR_UNSUPPORTED;
+  int64_t rows;
+  if (!mul_ok(a->Bt, a->Dn, &rows) || rows > (INT64_C(1) << 40)) return SSM_ERR_SHAPE;
+  if (a->Bt == 0) return SSM_OK;
+  if (!a->x || !a->dt || !a->A_log || !a->B || !a->C || !a->h || !a->out) return SSM_ERR_NULL;
+  if (a->conv_w && a->K > 1 && !a->conv_hist) return SSM_ERR_NULL;
+  const size_t ei = dtype_size(a->in_dtype), eo = dtype_size(a->out_dtype);
+  const void *in_ptrs[6] = {a->x, a->dt, a->z, a->B, a->C, a->conv_hist};
+  for (const void *p : in_ptrs)
+    if (p && !aligned(p, ei)) return SSM_ERR_ALIGN;
+  if (!aligned(a->out, eo)) return SSM_ERR_ALIGN;
+  const void *f32_ptrs[7] = {a->dt_bias, a->A_log, a->D, a->conv_w, a->conv_b, a->h, nullptr};
+  for (const void *p : f32_ptrs)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  ssm::StepParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = a->x;
+  p.dt = a->dt;
+  p.B = a->B;
+  p.C = a->C;
+  p.z = a->z;
+  p.dt_bias = a->dt_bias;
+  p.A_log = a->A_log;
+  p.D = a->D;
+  p.conv_w = a->conv_w;
+  p.conv_b = a->conv_w ? a->conv_b : nullptr;
+  p.h = a->h;
+  p.conv_hist = a->conv_w ? a->conv_hist : nullptr;
+  p.out = a->out;
+  p.Bt = a->Bt;
+  p.Dn = a->Dn;
+  p.N = a->N;
+  p.K = a->conv_w ? a->K : 0;
+  p.delta_softplus = a->delta_softplus ? 1 : 0;
+  p.euler = a->discretization == SSM_EULER ? 1 : 0;
+  return cuda_status(ssm::launch_step(p, a->in_dtype == SSM_BF16, a->out_dtype == SSM_BF16,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {
   if (!args) return 0;
   const ssm_fwd_args *a = &args->fwd;
@@ -160,12 +234,33 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   ssm_status st = check_fwd(&args->fwd, false, &empty);
   if (st != SSM_OK) return st;
   const ssm_fwd_args *a = &args->fwd;
-  if (empty) return SSM_OK;
+  if (empty) {
+    // nothing flows: parameter gradients are zero, the carried-state gradient passes through
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t fz = sizeof(float);
+    const int64_t BD = a->Bt * a->Dn;
+    cudaError_t e = cudaSuccess;
+    auto zero = [&](void *ptr, size_t bytes) {
+      if (ptr && bytes && e == cudaSuccess) e = cudaMemsetAsync(ptr, 0, bytes, s);
+    };
+    zero(args->dA_log, fz * (size_t)(a->Dn * a->N));
+    zero(args->dD, fz * (size_t)a->Dn);
+    zero(args->ddt_bias, fz * (size_t)a->Dn);
+    if (a->conv_w) {
+      zero(args->dconv_w, fz * (size_t)(a->Dn * a->K));
+      zero(args->dconv_b, fz * (size_t)a->Dn);
+      if (a->K > 1) zero(args->dconv_hist, fz * (size_t)(BD * (a->K - 1)));
+    }
+    if (args->dh0 && BD > 0 && e == cudaSuccess)
+      e = args->dh_last ? cudaMemcpyAsync(args->dh0, args->dh_last, fz * (size_t)(BD * a->N), cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(args->dh0, 0, fz * (size_t)(BD * a->N), s);
+    return cuda_status(e);
+  }
   if (!args->dout) return SSM_ERR_NULL;
   if (!aligned(args->dout, dtype_size(a->in_dtype))) return SSM_ERR_ALIGN;
-  const void *g32[12] = {args->chunk_states, args->dx, args->ddt, args->dz, args->dA_log, args->dB,
+  const void *g32[14] = {args->chunk_states, args->dx, args->ddt, args->dz, args->dA_log, args->dB,
                          args->dC, args->dD, args->ddt_bias, args->dconv_w, args->dconv_b,
-                         nullptr};
+                         args->dh_last, args->dh0, args->dconv_hist};
   for (const void *p : g32)
     if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
   const size_t need = ssm_bwd_workspace_size(args);
@@ -177,6 +272,8 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   fa.out = nullptr;
   fa.u_out = nullptr;
   fa.chunk_states = nullptr;
+  fa.h_last = nullptr;
+  fa.conv_hist_out = nullptr;
   ssm::BwdParams p;
   memset(&p, 0, sizeof(p));
   p.f = make_fwd_params(&fa, vec_ok(&fa, extra, 4));
@@ -193,6 +290,9 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   p.dconv_w = a->conv_w ? args->dconv_w : nullptr;
   p.dconv_b = a->conv_w ? args->dconv_b : nullptr;
   p.timing_events = args->timing_events;
+  p.dh_last = args->dh_last;
+  p.dh0 = args->dh0;
+  p.dconv_hist = (a->conv_w && a->K > 1) ? args->dconv_hist : nullptr;
   // carve the workspace (layout mirrored by ssm::bwd_workspace_bytes)
   char *ws = static_cast<char *>(args->workspace);
   auto take = [&](size_t bytes) {

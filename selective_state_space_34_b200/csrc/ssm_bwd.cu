@@ -75,7 +75,7 @@ template <int NS> __device__ __forceinline__ void store_states(float *dst, const
   }
 }
 
-template <int G, int NS, typename Tin>
+template <int G, int NS, typename Tin, bool EULER>
 __global__ void __launch_bounds__(kThreads, 2)
 ssm_bwd_kernel(const BwdParams P) {
   using S = BwdSmem<G, NS, Tin>;
@@ -121,8 +121,8 @@ ssm_bwd_kernel(const BwdParams P) {
 #pragma unroll
   for (int j = 0; j < 2 * NH; j++) {
     const int n = g * NS + j;
-    lam[j] = 0.f;
-    aN[j] = 0.f;
+    lam[j] = (P.dh_last && j < NS && live && n < N) ? P.dh_last[(b * p.Dn + d) * N + n] : 0.f;
+    aN[j] = 1.f;
     dAl[j] = 0.f;
     if (j < NS && live && n < N) {
       A[j] = -expf(p.A_log[d * N + n]);
@@ -195,6 +195,14 @@ ssm_bwd_kernel(const BwdParams P) {
     const Tin *dtrow = dts + (buf * CH + c) * kT;
     const Tin *zrow = zs + (buf * CH + c) * kT;
     const Tin *dorow = dos + (buf * CH + c) * kT;
+    if (st == 0 && has_conv && p.conv_hist && p.K > 1) {
+      // the carried inputs before step 0 (newest-first) replace the zero fill of the prefix
+      if (live && g == 0) {
+        const Tin *hr = static_cast<const Tin *>(p.conv_hist) + (b * p.Dn + d) * (p.K - 1);
+        for (int j = 0; j < p.K - 1; j++) xs[(buf * CH + c) * S::XS + kPre - 1 - j] = hr[j];
+      }
+      __syncwarp();
+    }
 
 #pragma unroll
     for (int sb = kT / kSub - 1; sb >= 0; sb--) {
@@ -258,7 +266,13 @@ ssm_bwd_kernel(const BwdParams P) {
 #pragma unroll
         for (int j = 0; j < 2 * NH; j++) {
           const int n = g * NS + j;
-          h[j] = (j < NS && kk > 0 && live && n < N) ? states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n] : 0.f;
+          h[j] = 0.f;
+          if (j < NS && live && n < N) {
+            if (kk > 0)
+              h[j] = states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n];
+            else if (p.h0)
+              h[j] = p.h0[(b * p.Dn + d) * N + n];
+          }
         }
         float *my0 = y0 + c * S::YC + g * S::YG;
 #pragma unroll
@@ -284,8 +298,12 @@ ssm_bwd_kernel(const BwdParams P) {
                 float2 a;
                 a.x = ex2_approx(x.x);
                 a.y = ex2_approx(x.y);
-                const float2 nw = __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), nIA2[q]);  // -B u / A
-                h2[q] = __ffma2_rn(a, __ffma2_rn(nw, make_float2(-1.f, -1.f), h2[q]), nw);
+                if (EULER) {
+                  h2[q] = __ffma2_rn(a, h2[q], __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), dl2));  // a h + Delta B u
+                } else {
+                  const float2 nw = __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), nIA2[q]);  // -B u / A
+                  h2[q] = __ffma2_rn(a, __ffma2_rn(nw, make_float2(-1.f, -1.f), h2[q]), nw);
+                }
                 ea2[tq + tt][q] = a;
                 hs2[tq + tt][q] = h2[q];
                 y2 = __ffma2_rn(Cq[tt][q], h2[q], y2);
@@ -302,11 +320,12 @@ ssm_bwd_kernel(const BwdParams P) {
                 const float nw = Bt[j] * eq[tt].y * nIA[j];  // -B u / A
                 if (PRECISE) {
                   const float em1 = expm1f(eq[tt].x * Acoef[j]);
-                  h[j] = fmaf(em1, h[j] - nw, h[j]);
+                  h[j] = EULER ? fmaf(em1, h[j], fmaf(eq[tt].x * Bt[j], eq[tt].y, h[j]))
+                               : fmaf(em1, h[j] - nw, h[j]);
                   eat[j] = em1;
                 } else {
                   const float a = ex2_approx(eq[tt].x * Acoef[j]);
-                  h[j] = fmaf(a, h[j] - nw, nw);
+                  h[j] = EULER ? fmaf(a, h[j], eq[tt].x * Bt[j] * eq[tt].y) : fmaf(a, h[j] - nw, nw);
                   eat[j] = a;
                 }
                 hst[j] = h[j];
@@ -363,13 +382,17 @@ ssm_bwd_kernel(const BwdParams P) {
               for (int q = 0; q < NH; q++) {
                 const float2 an2 = (tl + 1 < kSub) ? ea2[tl + 1][q] : aN2[q];
                 lam2[q] = __ffma2_rn(an2, lam2[q], __fmul2_rn(Cv[q], dy2));           // lambda_t
-                const float2 em1n = __fmul2_rn(__fadd2_rn(ea2[tl][q], make_float2(-1.f, -1.f)),
-                                               nIA2[q]);                               // -(A_bar-1)/A
+                // kb = -dB_bar/dB: (A_bar - 1)(-1/A) for the exact ZOH, -Delta for Euler
+                const float2 em1n = EULER ? make_float2(-e.x, -e.x)
+                                          : __fmul2_rn(__fadd2_rn(ea2[tl][q], make_float2(-1.f, -1.f)), nIA2[q]);
                 const float2 nlb = __fmul2_rn(lam2[q], __fmul2_rn(em1n, Bv[q]));      // -lambda B_bar
                 ndu2 = __fadd2_rn(ndu2, nlb);
                 nB2[q] = __fmul2_rn(__fmul2_rn(lam2[q], em1n), u2);                   // -dB partial
                 dC2[q] = __fmul2_rn(hs2[tl][q], dy2);
-                const float2 dterm = __fmul2_rn(lam2[q], __ffma2_rn(A2[q], hs2[tl][q], __fmul2_rn(Bv[q], u2)));
+                // dh_t/dDelta = A h_t + B u (ZOH) or A h_t + B u (1 - A Delta) (Euler)
+                float2 bu = __fmul2_rn(Bv[q], u2);
+                if (EULER) bu = __fmul2_rn(bu, __ffma2_rn(A2[q], make_float2(-e.x, -e.x), make_float2(1.f, 1.f)));
+                const float2 dterm = __fmul2_rn(lam2[q], __ffma2_rn(A2[q], hs2[tl][q], bu));
                 dd2 = __fadd2_rn(dd2, dterm);
                 dAl2[q] = __ffma2_rn(u2, nlb, __ffma2_rn(dl2, dterm, dAl2[q]));       // A dA
               }
@@ -386,12 +409,13 @@ ssm_bwd_kernel(const BwdParams P) {
                 const float em1 = PRECISE ? eat[j] : eat[j] - 1.f;
                 const float an = (PRECISE && tl + 1 < kSub) ? 1.f + ean[j] : ean[j];
                 lam[j] = fmaf(an, lam[j], Ct[j] * e.z);
-                const float em1n = em1 * nIA[j];
+                const float em1n = EULER ? -e.x : em1 * nIA[j];
                 const float nlb = lam[j] * (em1n * Bt[j]);
                 ndu += nlb;
                 nB[j] = lam[j] * em1n * e.y;
                 dCv[j] = hst[j] * e.z;
-                const float dterm = lam[j] * fmaf(A[j], hst[j], Bt[j] * e.y);
+                const float bu = EULER ? Bt[j] * e.y * fmaf(-A[j], e.x, 1.f) : Bt[j] * e.y;
+                const float dterm = lam[j] * fmaf(A[j], hst[j], bu);
                 dd += dterm;
                 dAl[j] = fmaf(e.y, nlb, fmaf(e.x, dterm, dAl[j]));
               }
@@ -522,6 +546,14 @@ ssm_bwd_kernel(const BwdParams P) {
           store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + sb * kSub + g * EPL, L, dxv, vec);
       }
       __syncwarp();
+      if (st == 0 && live && g == 0 && P.dconv_hist && p.K > 1) {
+        // x_{-1-j} reaches c_t through tap k = t + 1 + j
+        for (int j = 0; j < p.K - 1; j++) {
+          float acc = 0.f;
+          for (int k = j + 1; k < p.K; k++) acc = fmaf(w4[k], dcs[c * S::DCS + k - j - 1], acc);
+          P.dconv_hist[(b * p.Dn + d) * (p.K - 1) + j] = acc;
+        }
+      }
       // this stage's first 3 dc values become the halo of the stage before it
       if (g == 0)
         for (int k = 0; k < 3; k++) dcs[c * S::DCS + kT + k] = dcs[c * S::DCS + k];
@@ -529,12 +561,16 @@ ssm_bwd_kernel(const BwdParams P) {
     }
   }
 
-  // per-channel parameter partials for this batch element
+  // per-channel parameter partials for this batch element; gradient of the carried state
+  // (h_0 = A_bar_0 h0 + ..., so dh0 = A_bar_0 lambda_0)
   if (live) {
 #pragma unroll
     for (int j = 0; j < NS; j++) {
       const int n = g * NS + j;
-      if (n < N) P.p_dA_log[(b * p.Dn + d) * N + n] = dAl[j];
+      if (n < N) {
+        P.p_dA_log[(b * p.Dn + d) * N + n] = dAl[j];
+        if (P.dh0) P.dh0[(b * p.Dn + d) * N + n] = aN[j] * lam[j];
+      }
     }
   }
 #pragma unroll
@@ -614,7 +650,7 @@ size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int nee
 template <int G, int NS, typename Tin>
 static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   using S = BwdSmem<G, NS, Tin>;
-  auto kern = ssm_bwd_kernel<G, NS, Tin>;
+  auto kern = P.f.euler ? ssm_bwd_kernel<G, NS, Tin, true> : ssm_bwd_kernel<G, NS, Tin, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
   if (e != cudaSuccess) return e;
   const int64_t grid = P.n_dtiles * P.f.Bt;

@@ -40,7 +40,7 @@ template <int G, int NS, typename Tin, int NT> struct FwdSmem {
   static constexpr size_t bytes = yp_off + sizeof(float) * CH * YC;
 };
 
-template <int G, int NS, typename Tin, typename Tout, int NT>
+template <int G, int NS, typename Tin, typename Tout, int NT, bool EULER>
 __global__ void __launch_bounds__(NT, 512 / NT)
 ssm_fwd_kernel(const FwdParams p) {
   using S = FwdSmem<G, NS, Tin, NT>;
@@ -72,7 +72,7 @@ ssm_fwd_kernel(const FwdParams p) {
 #pragma unroll
   for (int j = 0; j < NS; j++) {
     const int n = g * NS + j;
-    h[j] = 0.0f;
+    h[j] = (p.h0 && live && n < N) ? p.h0[(b * p.Dn + d) * N + n] : 0.0f;  // carried state or 0
     if (live && n < N) {
       const float A = -expf(p.A_log[d * N + n]);
       Acoef[j] = PRECISE ? A : A * kLog2e;
@@ -103,10 +103,14 @@ ssm_fwd_kernel(const FwdParams p) {
   const Tin *gC = static_cast<const Tin *>(p.C) + b * N * L;
   const int n_rows = (int)imin64(NP, N);
 
-  // zero the conv-halo prefixes of both x buffers (the sequence starts from zero history)
+  // conv-halo prefixes of both x buffers: the carried history (newest-first) in front of the
+  // first stage, zero where there is none
+  const Tin *hist = (has_conv && p.conv_hist && p.K > 1) ? static_cast<const Tin *>(p.conv_hist) : nullptr;
   for (int i = tid; i < 2 * CH * kPre; i += NT) {
-    const int r = i / kPre, k = i % kPre;
-    xs[r * S::XS + k] = zero_val<Tin>();
+    const int r = i / kPre, k = i % kPre, j = kPre - 1 - k;  // x_{-1-j}
+    Tin v = zero_val<Tin>();
+    if (hist && r < rows_valid && j < p.K - 1) v = hist[(b * p.Dn + d0 + r) * (p.K - 1) + j];
+    xs[r * S::XS + k] = v;
   }
 
   const int64_t n_stages = (L + kT - 1) / kT;
@@ -204,9 +208,13 @@ ssm_fwd_kernel(const FwdParams p) {
             float y = 0.0f;
 #pragma unroll
             for (int j = 0; j < NS; j++) {
-              const float nw = Bq[tt][j] * uq[tt] * nIA[j];   // -B u / A
               const float em1 = expm1f(dlq[tt] * Acoef[j]);    // A_bar - 1
-              h[j] = fmaf(em1, h[j] - nw, h[j]);               // A_bar h + (A_bar - 1) B u / A
+              if (EULER) {
+                h[j] = fmaf(em1, h[j], fmaf(dlq[tt] * Bq[tt][j], uq[tt], h[j]));  // A_bar h + Delta B u
+              } else {
+                const float nw = Bq[tt][j] * uq[tt] * nIA[j];   // -B u / A
+                h[j] = fmaf(em1, h[j] - nw, h[j]);               // A_bar h + (A_bar - 1) B u / A
+              }
               y = fmaf(Cq[tt][j], h[j], y);
             }
             yq[tt] = y;
@@ -234,11 +242,17 @@ ssm_fwd_kernel(const FwdParams p) {
               const float2 u2 = make_float2(uq[tt], uq[tt]);
 #pragma unroll
               for (int j = 0; j < NS; j += 2) {
-                const float2 nw = __fmul2_rn(__fmul2_rn(make_float2(Bq[tt][j], Bq[tt][j + 1]), u2),
-                                             make_float2(nIA[j], nIA[j + 1]));  // -B u / A
                 float2 hh = make_float2(h[j], h[j + 1]);
-                const float2 sum = __ffma2_rn(nw, make_float2(-1.0f, -1.0f), hh);  // h + w
-                hh = __ffma2_rn(make_float2(a[tt][j], a[tt][j + 1]), sum, nw);     // a (h+w) - w
+                if (EULER) {
+                  const float2 bdu = __fmul2_rn(__fmul2_rn(make_float2(Bq[tt][j], Bq[tt][j + 1]), u2),
+                                                make_float2(dlq[tt], dlq[tt]));  // Delta B u
+                  hh = __ffma2_rn(make_float2(a[tt][j], a[tt][j + 1]), hh, bdu);
+                } else {
+                  const float2 nw = __fmul2_rn(__fmul2_rn(make_float2(Bq[tt][j], Bq[tt][j + 1]), u2),
+                                               make_float2(nIA[j], nIA[j + 1]));  // -B u / A
+                  const float2 sum = __ffma2_rn(nw, make_float2(-1.0f, -1.0f), hh);  // h + w
+                  hh = __ffma2_rn(make_float2(a[tt][j], a[tt][j + 1]), sum, nw);     // a (h+w) - w
+                }
                 h[j] = hh.x;
                 h[j + 1] = hh.y;
                 y2 = __ffma2_rn(make_float2(Cq[tt][j], Cq[tt][j + 1]), hh, y2);
@@ -248,8 +262,12 @@ ssm_fwd_kernel(const FwdParams p) {
               float y = 0.0f;
 #pragma unroll
               for (int j = 0; j < NS; j++) {
-                const float nw = Bq[tt][j] * uq[tt] * nIA[j];
-                h[j] = fmaf(a[tt][j], h[j] - nw, nw);
+                if (EULER) {
+                  h[j] = fmaf(a[tt][j], h[j], dlq[tt] * Bq[tt][j] * uq[tt]);
+                } else {
+                  const float nw = Bq[tt][j] * uq[tt] * nIA[j];
+                  h[j] = fmaf(a[tt][j], h[j] - nw, nw);
+                }
                 y = fmaf(Cq[tt][j], h[j], y);
               }
               yq[tt] = y;
@@ -284,6 +302,29 @@ ssm_fwd_kernel(const FwdParams p) {
       }
       __syncwarp();  // ud / yp are rewritten by the next block
     }
+  }
+  // carried state after step L-1 (padded tail steps are identity steps)
+  if (live && p.h_last) {
+#pragma unroll
+    for (int j = 0; j < NS; j++)
+      if (g * NS + j < N) p.h_last[(b * p.Dn + d) * N + g * NS + j] = h[j];
+  }
+  // the K-1 newest pre-conv inputs, newest-first; read everything before writing (the output
+  // may alias the input history)
+  if (live && has_conv && p.conv_hist_out && p.K > 1 && g == 0) {
+    const Tin *xr = static_cast<const Tin *>(p.x) + (b * p.Dn + d) * L;
+    const Tin *hr = hist ? hist + (b * p.Dn + d) * (p.K - 1) : nullptr;
+    Tin v[3];
+#pragma unroll
+    for (int j = 0; j < 3; j++) {
+      const int64_t t = L - 1 - j;
+      v[j] = zero_val<Tin>();
+      if (j < p.K - 1) v[j] = (t >= 0) ? xr[t] : (hr ? hr[j - L] : zero_val<Tin>());
+    }
+    Tin *o = static_cast<Tin *>(p.conv_hist_out) + (b * p.Dn + d) * (p.K - 1);
+#pragma unroll
+    for (int j = 0; j < 3; j++)
+      if (j < p.K - 1) o[j] = v[j];
   }
 }
 
@@ -330,7 +371,7 @@ template <int G, int NS, typename Tin, typename Tout>
 static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
   constexpr int NT = kFwdThreads;
   using S = FwdSmem<G, NS, Tin, NT>;
-  auto kern = ssm_fwd_kernel<G, NS, Tin, Tout, NT>;
+  auto kern = p.euler ? ssm_fwd_kernel<G, NS, Tin, Tout, NT, true> : ssm_fwd_kernel<G, NS, Tin, Tout, NT, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
   if (e != cudaSuccess) return e;
   const int64_t n_dtiles = (p.Dn + S::CH - 1) / S::CH;

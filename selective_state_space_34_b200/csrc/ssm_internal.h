@@ -29,6 +29,20 @@ struct FwdParams {
   int K;
   int delta_softplus;
   int vec;  // 1: rows are 16-byte aligned, stage with cp.async and store with vector stores
+  int euler;  // input discretisation: 0 exact ZOH, 1 Delta * B
+  const float *h0;        // (Bt, Dn, N) or null
+  const void *conv_hist;  // (Bt, Dn, K-1) in-dtype or null
+  float *h_last;          // (Bt, Dn, N) or null
+  void *conv_hist_out;    // (Bt, Dn, K-1) in-dtype or null
+};
+
+struct StepParams {
+  const void *x, *dt, *B, *C, *z;
+  const float *dt_bias, *A_log, *D, *conv_w, *conv_b;
+  float *h;
+  void *conv_hist, *out;
+  int64_t Bt, Dn, N;
+  int K, delta_softplus, euler;
 };
 
 struct BwdParams {
@@ -47,6 +61,9 @@ struct BwdParams {
   int64_t n_dtiles;
   float *dA_log, *dD, *ddt_bias, *dconv_w, *dconv_b;
   void *const *timing_events;  // optional: 2 cudaEvent_t around the main backward kernel
+  const float *dh_last;        // (Bt, Dn, N) or null
+  float *dh0;                  // (Bt, Dn, N) or null
+  float *dconv_hist;           // (Bt, Dn, K-1) or null
 };
 
 LaneLayout choose_layout(int64_t N, int64_t channels);
@@ -55,6 +72,7 @@ int channels_per_cta(const LaneLayout &lay);
 cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
 size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states);
+cudaError_t launch_step(const StepParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
                                int64_t Dn, int64_t L, int K, int in_bf16, int out_bf16, int vec,
                                cudaStream_t stream);

@@ -11,13 +11,13 @@ namespace ssm {
 template <typename T> __device__ __forceinline__ T zero_val() { return from_f32<T>(0.0f); }
 
 // dst[r][i] = src[r][t0 + i] for r < rows_valid and 0 <= t0 + i < L, else 0, for i in [0, LEN).
-template <typename T, int ROWS, int LEN = kT>
+template <typename T, int ROWS, int LEN = kT, int NT = kThreads>
 __device__ __forceinline__ void stage_rows(T *dst, int dst_stride, const T *src, int64_t src_stride,
                                            int rows_valid, int64_t t0, int64_t L, bool vec) {
   constexpr int EPV = 16 / sizeof(T);
   constexpr int VPR = LEN / EPV;
   if (vec) {
-    for (int idx = threadIdx.x; idx < ROWS * VPR; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < ROWS * VPR; idx += NT) {
       const int r = idx / VPR, v = idx % VPR;
       const int64_t t = t0 + (int64_t)v * EPV;
       T *d = dst + r * dst_stride + v * EPV;
@@ -27,7 +27,7 @@ __device__ __forceinline__ void stage_rows(T *dst, int dst_stride, const T *src,
         *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
     }
   } else {
-    for (int idx = threadIdx.x; idx < ROWS * LEN; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < ROWS * LEN; idx += NT) {
       const int r = idx / LEN, i = idx % LEN;
       const int64_t t = t0 + i;
       dst[r * dst_stride + i] =
@@ -136,18 +136,18 @@ template <int NS> __device__ __forceinline__ void load_states(float *dst, const 
 // registers -> transposed fp32 rows [t][n] in shared memory, so that the scan reads all of a
 // lane's states at one step with one 16-byte broadcast load. Loads for stage s+1 are issued one
 // stage early into registers; the transposed stores happen after the next barrier-free point.
-template <typename Tin, int NP> struct BCStager {
+template <typename Tin, int NP, int NT = kThreads> struct BCStager {
   static constexpr int EPV = 16 / sizeof(Tin);               // elements per 16-byte vector
   static constexpr int VPR = kT / EPV;                       // vectors per row
   static constexpr int NV = 2 * NP * VPR;                    // B and C vectors per stage
-  static constexpr int PER = (NV + kThreads - 1) / kThreads; // per thread
+  static constexpr int PER = (NV + NT - 1) / NT;             // per thread
   uint4 v[PER];
 
   __device__ __forceinline__ void load(const Tin *gB, const Tin *gC, int n_rows, int64_t t0,
                                        int64_t L, bool vec) {
 #pragma unroll
     for (int k = 0; k < PER; k++) {
-      const int i = threadIdx.x + k * kThreads;
+      const int i = threadIdx.x + k * NT;
       v[k] = make_uint4(0u, 0u, 0u, 0u);
       if (i >= NV) continue;
       const int which = i / (NP * VPR), r = (i / VPR) % NP, q = i % VPR;
@@ -167,7 +167,7 @@ template <typename Tin, int NP> struct BCStager {
   __device__ __forceinline__ void store(float *Bs, float *Cs, int BS) const {
 #pragma unroll
     for (int k = 0; k < PER; k++) {
-      const int i = threadIdx.x + k * kThreads;
+      const int i = threadIdx.x + k * NT;
       if (i >= NV) continue;
       const int which = i / (NP * VPR), r = (i / VPR) % NP, q = i % VPR;
       float *dst = (which ? Cs : Bs) + (q * EPV) * BS + r;

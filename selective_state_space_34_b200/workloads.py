@@ -122,6 +122,19 @@ def generate(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     return out
 
 
+def carried_state(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[np.ndarray]]:
+    """State carried in from a previous chunk and the gradient arriving at the final state:
+    h0 ~ N(0, 0.5) and dh_last ~ N(0, 0.1), both (Bt, Dn, N) float32; conv_hist ~ N(0, 1),
+    (Bt, Dn, K-1) in the input dtype (None without a conv)."""
+    s = (w.seed if seed is None else int(seed)) + 7919
+    rnd = round_to_bf16 if w.in_dtype == "bf16" else (lambda a: a)
+    return {
+        "h0": _normal(s, 11, (w.Bt, w.Dn, w.N), 0.5),
+        "conv_hist": rnd(_normal(s, 12, (w.Bt, w.Dn, w.K - 1), 1.0)) if w.conv else None,
+        "dh_last": _normal(s, 13, (w.Bt, w.Dn, w.N), 0.1),
+    }
+
+
 def shaped(base: str, **overrides) -> Workload:
     """A named workload with some fields replaced (e.g. smaller Bt/Dn/L for a parity case)."""
     return replace(WORKLOADS[base], **overrides)

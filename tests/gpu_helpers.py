@@ -31,7 +31,7 @@ def dev_arrays(a, in_dtype, device="cuda"):
     for k, v in a.items():
         if v is None:
             out[k] = None
-        elif k in ("x", "dt", "z", "B", "C", "dout"):
+        elif k in ("x", "dt", "z", "B", "C", "dout", "conv_hist"):
             out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=act)
         else:
             out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=torch.float32)

@@ -34,18 +34,29 @@ def test_every_declared_function_is_exported(lib):
     assert sorted(n for n, _, _ in _abi.SIGNATURES) == names
 
 
-def test_struct_layout_matches_header_field_order():
-    src = open(HEADER).read()
-    body = src[src.index("typedef struct ssm_fwd_args"):src.index("} ssm_fwd_args;")]
-    fields = re.findall(r"\b(\w+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
-    flat = []
-    for line in re.sub(r"/\*.*?\*/", "", body, flags=re.S).split(";"):
-        names = re.findall(r"[\*\s](\w+)\s*(?:,|$)", line.strip() + " ")
-        if names:
-            flat.extend(re.findall(r"(\w+)\s*(?=,|$)", line.split("{")[-1].strip()))
-    ct = [f[0] for f in _abi.FwdArgs._fields_]
-    assert [f for f in flat if f in ct] == ct
-    assert ctypes.sizeof(_abi.FwdArgs) == 13 * 8 + 4 * 8 + 4 * 4
+def _header_fields(struct):
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = src[src.index("typedef struct %s {" % struct) + len("typedef struct %s {" % struct):
+               src.index("} %s;" % struct)]
+    names = []
+    for decl in body.split(";"):
+        if decl.strip():
+            names.extend(re.findall(r"(\w+)\s*$", part)[0] for part in decl.split(","))
+    return names
+
+
+@pytest.mark.parametrize("struct,cls,size", [
+    # 17 pointers, 4 int64, 5 int32 (+4 bytes of tail padding)
+    ("ssm_fwd_args", "FwdArgs", 17 * 8 + 4 * 8 + 5 * 4 + 4),
+    # the forward block, 17 pointers and one size
+    ("ssm_bwd_args", "BwdArgs", 192 + 17 * 8 + 8),
+    # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
+    ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
+])
+def test_struct_layout_matches_header_field_order(struct, cls, size):
+    ct = [f[0] for f in getattr(_abi, cls)._fields_]
+    assert _header_fields(struct) == ct
+    assert ctypes.sizeof(getattr(_abi, cls)) == size
 
 
 def test_status_strings(lib):
@@ -130,6 +141,43 @@ def test_bwd_validation_codes(lib):
     full = lib.ssm_bwd_workspace_size(ctypes.byref(bw))
     bw.chunk_states = 0xA000
     assert lib.ssm_bwd_workspace_size(ctypes.byref(bw)) < full
+
+
+def test_state_carry_validation_codes(lib):
+    assert _fwd(lib, _args(discretization=2)) == 5
+    assert _fwd(lib, _args(discretization=1, x=0x1001)) == 3   # Euler passes the flag check
+    assert _fwd(lib, _args(h0=0x7002)) == 3
+    assert _fwd(lib, _args(h_last=0x7001)) == 3
+    assert _fwd(lib, _args(conv_w=0x7000, conv_hist=0x7001)) == 3
+    assert _fwd(lib, _args(in_dtype=1, conv_w=0x7000, conv_hist_out=0x7001)) == 3
+    # an empty chunk carries the state through without touching NULL pointers
+    assert _fwd(lib, _args(L=0, x=None, out=None)) == 0
+
+
+def _step(**kw):
+    a = _abi.StepArgs()
+    a.x, a.dt, a.A_log, a.B, a.C, a.h, a.out = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0x7000
+    a.Bt, a.Dn, a.N, a.K = 2, 8, 4, 4
+    a.in_dtype, a.out_dtype, a.delta_softplus = 0, 0, 1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_step_validation_codes(lib):
+    f = lambda a: lib.ssm_scan_step(ctypes.byref(a), None)
+    assert lib.ssm_scan_step(None, None) == 1
+    assert f(_step(h=None)) == 1
+    assert f(_step(in_dtype=3)) == 4
+    assert f(_step(discretization=5)) == 5
+    assert f(_step(Dn=0)) == 2
+    assert f(_step(N=0)) == 2
+    assert f(_step(N=65)) == 5
+    assert f(_step(conv_w=0x8000, K=5, conv_hist=0x9000)) == 5
+    assert f(_step(conv_w=0x8000, K=4)) == 1          # a conv needs its history
+    assert f(_step(conv_w=0x8000, K=4, conv_hist=0x9001)) == 3
+    assert f(_step(h=0x6002)) == 3
+    assert f(_step(Bt=0, x=None, h=None)) == 0        # no rows: nothing to do
 
 
 def test_conv_validation_codes(lib):
