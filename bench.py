@@ -37,6 +37,34 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 FMA_LANES, MUFU_LANES, N_SM = 128, 16, 148
 
 
+# ---- rank plumbing (host only; covered by world-size-2 gloo tests on CPU) -----------------------
+
+def rank_env():
+    """(world, rank, local_rank) from the launcher's environment; a plain run is rank 0 of 1."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(w, rank):
+    """Every rank draws its own batch of the same workload (weak scaling): seed + rank."""
+    return w.seed + rank
+
+
+def max_over_ranks(x, world, device):
+    """The slowest rank's value of x (a device time in ms); a no-op on one rank."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, steps, max_ms):
+    """Whole-job rate: the units every rank processed in `steps` steps over the slowest time."""
+    return units_per_rank * world * steps / (max_ms * 1e-3)
+
+
 def ncu_traffic(kernel, source):
     """DRAM bytes per launch of `kernel` from profiles/ncu_traffic.md, or None when the recorded
     capture was taken on a different version of the kernel's source file."""
@@ -148,13 +176,18 @@ def oracle_sample(w, a, n_channels, threads):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     per = max(1, min(16, n_channels // max(1, threads)))
-    picks = [(i // w.Dn % w.Bt, i % w.Dn) for i in range(n_channels)]
-    groups = [picks[i:i + per] for i in range(0, len(picks), per)]
+    # contiguous channel runs of one batch element each, wrapping over (batch, channel) when the
+    # sample is larger than the workload
+    total, groups, i = w.Bt * w.Dn, [], 0
+    while i < n_channels:
+        b, d = divmod(i % total, w.Dn)
+        n = min(per, w.Dn - d, n_channels - i)
+        groups.append((b, d, d + n))
+        i += n
 
     def run(group):
-        b = group[0][0]
-        ds = [d for bb, d in group if bb == b]
-        sl = slice(ds[0], ds[-1] + 1)
+        b, lo, hi = group
+        sl = slice(lo, hi)
         kw = dict(D=a["D"][sl], z=None if a["z"] is None else a["z"][b:b + 1, sl],
                   dt_bias=a["dt_bias"][sl], conv_w=None if a["conv_w"] is None else a["conv_w"][sl],
                   conv_b=None if a["conv_b"] is None else a["conv_b"][sl])
@@ -163,7 +196,7 @@ def oracle_sample(w, a, n_channels, threads):
         oracle.fwd(x, dt, Al, B, C, n_threads=1, **kw)
         if w.backward:
             oracle.bwd(x, dt, Al, B, C, a["dout"][b:b + 1, sl], n_threads=1, **kw)
-        return len(ds) * w.L * w.N
+        return (hi - lo) * w.L * w.N
 
     oracle.build()
     t0 = time.perf_counter()
@@ -173,8 +206,9 @@ def oracle_sample(w, a, n_channels, threads):
 
 
 def reference_arm(args, w):
-    """--impl reference: the float64 oracle timed on the host cores, on bounded samples."""
-    rank = int(os.environ.get("RANK", "0"))
+    """--impl reference: the float64 oracle timed on the host cores, on bounded samples. Under a
+    multi-rank launch rank 0 alone runs it; the other ranks return without work."""
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     from selective_state_space_34_b200 import workloads as wl
@@ -230,9 +264,7 @@ def main():
     import torch.distributed as dist
     import selective_state_space_34_b200 as ssm
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -240,7 +272,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     # each rank draws its own batch (weak scaling)
-    a = wl.generate(w, seed=w.seed + rank)
+    a = wl.generate(w, seed=rank_seed(w, rank))
     act = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
     odt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
 
@@ -341,13 +373,9 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(el, op=dist.ReduceOp.MAX)
-    max_ms = float(el.item())
+    max_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     ms_step = max_ms / args.steps
-    value = es * world * args.steps / (max_ms * 1e-3)
+    value = job_throughput(es, world, args.steps, max_ms)
 
     fwd_ms = float(np.mean([ev_f0[i].elapsed_time(ev_f1[i]) for i in range(args.steps)]))
     kern = {"ssm_fwd_kernel": fwd_ms}
@@ -367,11 +395,7 @@ def main():
         fwd_only()
     f1.record(s)
     torch.cuda.synchronize()
-    fo_ms = f0.elapsed_time(f1) / nf
-    fo = torch.tensor([fo_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(fo, op=dist.ReduceOp.MAX)
-    fo_ms = float(fo.item())
+    fo_ms = max_over_ranks(f0.elapsed_time(f1) / nf, world, dev)
 
     peaks = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -391,7 +415,7 @@ def main():
         return {"bound": "alu", "achieved": ach, "peak": mufu_peak, "unit": "Gexp/s",
                 "frac": ach / mufu_peak, "kernel": kernel,
                 "peak_source": "16 MUFU ex2 lanes/clk/SM x 148 SMs x sampled SM clock"}
-    forward = {"ms": fo_ms, "value": es * world / (fo_ms * 1e-3), "unit": UNIT,
+    forward = {"ms": fo_ms, "value": job_throughput(es, world, 1, fo_ms), "unit": UNIT,
                "out_dtype": args.out_dtype, "roofline": fwd_roof,
                "alu_roofline": alu_roof("ssm_fwd_kernel", fo_ms)}
 
@@ -436,13 +460,10 @@ def main():
         e2e_step()
     e1.record(s)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
-    e2e = {"value": es * world * args.e2e_steps / (float(et.item()) * 1e-3), "unit": UNIT,
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": job_throughput(es, world, args.e2e_steps, e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": float(et.item()) / args.e2e_steps}
+           "ms_per_step": e_ms / args.e2e_steps}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
