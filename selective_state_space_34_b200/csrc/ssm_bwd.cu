@@ -17,45 +17,53 @@
 // difference x a - (a - 1) for small x.
 //
 // Decomposition mirrors the forward: a CTA owns CH = 128/G channels of one batch element, lanes
-// hold NS states each, and the sequence is walked backwards in stages of kT steps, each split in
-// blocks of kSub = 16 steps: recompute the block forward from its saved start state (a_t and h_t
-// kept in registers), then run the adjoint backwards through it. dB and dC are summed over the
-// CTA's channels in shared memory and written as per-tile partials; a second kernel adds the
-// tiles (and the per-batch partials of the per-channel parameter gradients) in a fixed order, so
-// the result is deterministic.
+// hold NS states each, and the sequence is walked backwards in stages of 16 steps (one saved-state
+// chunk each): recompute the stage forward from its saved start state, keeping h_t and a_t of every
+// step in the thread's lane of tensor memory (TMEM, otherwise idle here) instead of registers, then
+// run the adjoint backwards through it one 4-step group at a time. Moving that trajectory out of
+// the register file is what lets four CTAs share an SM. dB and dC are summed over the CTA's
+// channels in shared memory after every 4 steps and written as per-tile partials; a second kernel
+// adds the tiles (and the per-batch partials of the per-channel parameter gradients) in a fixed
+// order, so the result is deterministic.
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
+#include "ssm_tmem.cuh"
 
 namespace ssm {
 
 template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr int CH = kThreads / G;
   static constexpr int NP = G * NS;
-  static constexpr int XS = kPre + kT;
+  static constexpr int TS = kSub;                 // steps per stage = one saved-state chunk
+  static constexpr int XS = kPre + TS;
   static constexpr int BS = NP + 4;
-  static constexpr int ES = kSub + 1;             // e3 row stride (float4: dl, u, dy, -)
-  static constexpr int YG = kSub + 4;
+  static constexpr int ES = TS + 1;               // e3 / pe row stride
+  static constexpr int YG = TS;
   static constexpr int YC = G * YG + 4;
-  static constexpr int DCS = kT + 8;              // dc row: this stage, then the next stage's 3
-  static constexpr int RH = kSub / 2;             // steps per cross-channel reduction
+  // with 4 lanes per channel the du / dDelta lane sums go through shuffles (no shared rows)
+  static constexpr bool SHFL = (G == 4);
+  static constexpr int DCS = TS + 8;              // dc row: this stage, then the next stage's 3
+  static constexpr int RH = 4;                    // steps per cross-channel reduction
   static constexpr int CHH = CH / 2;
   static constexpr int RBC = CHH * NP + 16;       // half-tile of channels (+16 words: banks)
   static constexpr int RBT = 2 * RBC + 4;         // one step
   static constexpr int RBW = RH * RBT;            // one quantity (dB or dC)
+  static constexpr uint32_t NCOLS = 32 * NS;      // TMEM: h and A_bar of TS steps x NS states
   static constexpr size_t x_off = 0;
   static constexpr size_t dt_off = x_off + sizeof(Tin) * 2 * CH * XS;
-  static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t do_off = z_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t bs_off = do_off + sizeof(Tin) * 2 * CH * kT;
-  static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * kT * BS;
-  static constexpr size_t e3_off = cs_off + sizeof(float) * 2 * kT * BS;
-  static constexpr size_t pe_off = e3_off + sizeof(float4) * CH * ES;   // (gc, sv, gz, -)
-  static constexpr size_t y0_off = pe_off + sizeof(float4) * CH * ES;
+  static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * TS;
+  static constexpr size_t do_off = z_off + sizeof(Tin) * 2 * CH * TS;
+  static constexpr size_t bs_off = do_off + sizeof(Tin) * 2 * CH * TS;
+  static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * TS * BS;
+  static constexpr size_t e3_off = cs_off + sizeof(float) * 2 * TS * BS;   // (dl, u, dy, gc)
+  static constexpr size_t pe_off = e3_off + sizeof(float4) * CH * ES;      // (sv, gz)
+  static constexpr size_t y0_off = pe_off + sizeof(float2) * CH * ES;
   static constexpr size_t y1_off = y0_off + sizeof(float) * CH * YC;
-  static constexpr size_t dcs_off = y1_off + sizeof(float) * CH * YC;
+  static constexpr size_t dcs_off = y1_off + (SHFL ? 0 : sizeof(float) * CH * YC);
   static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
-  static constexpr size_t bytes = rb_off + sizeof(float) * 2 * RBW;
+  static constexpr size_t slot_off = rb_off + sizeof(float) * 2 * RBW;
+  static constexpr size_t bytes = slot_off + 16;
   __host__ __device__ static constexpr int rb_index(int which, int tt, int c, int n) {
     return which * RBW + tt * RBT + (c / CHH) * RBC + (c % CHH) * NP + n;
   }
@@ -76,12 +84,14 @@ template <int NS> __device__ __forceinline__ void store_states(float *dst, const
 }
 
 template <int G, int NS, typename Tin, bool EULER>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 4)
 ssm_bwd_kernel(const BwdParams P) {
   using S = BwdSmem<G, NS, Tin>;
-  constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G, RH = S::RH;
+  constexpr int CH = S::CH, NP = S::NP, TS = S::TS, EPL = TS / G, RH = S::RH;
+  constexpr int GV = 4 * NS;  // TMEM columns of one quantity over a 4-step group
   constexpr bool PRECISE = sizeof(Tin) == 4;
   constexpr bool PAIRS = !PRECISE && (NS % 2 == 0);
+  static_assert(RH == 4 && TS % 4 == 0, "a reduction quarter is one 4-step TMEM group");
   const FwdParams &p = P.f;
   extern __shared__ __align__(16) unsigned char smem[];
   Tin *xs = reinterpret_cast<Tin *>(smem + S::x_off);
@@ -91,11 +101,18 @@ ssm_bwd_kernel(const BwdParams P) {
   float *Bs = reinterpret_cast<float *>(smem + S::bs_off);
   float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
   float4 *e3 = reinterpret_cast<float4 *>(smem + S::e3_off);
-  float4 *pe = reinterpret_cast<float4 *>(smem + S::pe_off);
+  float2 *pe = reinterpret_cast<float2 *>(smem + S::pe_off);
   float *y0 = reinterpret_cast<float *>(smem + S::y0_off);
   float *y1 = reinterpret_cast<float *>(smem + S::y1_off);
   float *dcs = reinterpret_cast<float *>(smem + S::dcs_off);
   float *rb = reinterpret_cast<float *>(smem + S::rb_off);
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + S::slot_off);
+
+  // h and A_bar (A_bar - 1 on the precise path) of the stage's steps live in this thread's TMEM
+  // lane: column t*NS + j holds step t, state j
+  const uint32_t tbase = tmem_alloc_cta(slot, S::NCOLS);
+  const uint32_t th = tmem_lane_addr(tbase);
+  const uint32_t ta = th + TS * NS;
 
   const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
   const int64_t tile = blockIdx.x % n_dtiles;
@@ -161,40 +178,40 @@ ssm_bwd_kernel(const BwdParams P) {
   // dc of the (non-existent) steps after the sequence end are zero
   for (int i = tid; i < CH * S::DCS; i += kThreads) dcs[i] = 0.f;
 
-  const int64_t n_stages = (L + kT - 1) / kT;
+  const int64_t n_stages = (L + TS - 1) / TS;
   auto issue = [&](int64_t stage, int buf) {
-    const int64_t t0 = stage * kT;
-    stage_rows<Tin, CH, kPre + kT>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
-    stage_rows<Tin, CH>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
-    if (has_z) stage_rows<Tin, CH>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
-    stage_rows<Tin, CH>(dos + buf * CH * kT, kT, gdo, L, rows_valid, t0, L, vec);
+    const int64_t t0 = stage * TS;
+    stage_rows<Tin, CH, kPre + TS>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
+    stage_rows<Tin, CH, TS>(dts + buf * CH * TS, TS, gdt, L, rows_valid, t0, L, vec);
+    if (has_z) stage_rows<Tin, CH, TS>(zs + buf * CH * TS, TS, gz, L, rows_valid, t0, L, vec);
+    stage_rows<Tin, CH, TS>(dos + buf * CH * TS, TS, gdo, L, rows_valid, t0, L, vec);
     cp_async_commit();
   };
 
-  BCStager<Tin, NP> bc;
+  BCStager<Tin, NP, kThreads, TS> bc;
   if (n_stages > 0) {
     const int lbuf = (int)((n_stages - 1) & 1);
     issue(n_stages - 1, lbuf);
-    bc.load(gB, gC, n_rows, (n_stages - 1) * kT, L, vec);
-    bc.store(Bs + lbuf * kT * S::BS, Cs + lbuf * kT * S::BS, S::BS);
-    if (n_stages > 1) bc.load(gB, gC, n_rows, (n_stages - 2) * kT, L, vec);
+    bc.load(gB, gC, n_rows, (n_stages - 1) * TS, L, vec);
+    bc.store(Bs + lbuf * TS * S::BS, Cs + lbuf * TS * S::BS, S::BS);
+    if (n_stages > 1) bc.load(gB, gC, n_rows, (n_stages - 2) * TS, L, vec);
   }
   for (int64_t st = n_stages - 1; st >= 0; st--) {
     const int buf = (int)(st & 1), pbuf = buf ^ 1;
-    const int64_t t0 = st * kT;
+    const int64_t t0 = st * TS;
     cp_async_wait<0>();
     __syncthreads();  // stage st landed; B/C rows of stage st written; stage st+1's buffers free
     if (st > 0) {
       issue(st - 1, pbuf);
-      bc.store(Bs + pbuf * kT * S::BS, Cs + pbuf * kT * S::BS, S::BS);
-      if (st > 1) bc.load(gB, gC, n_rows, (st - 2) * kT, L, vec);
+      bc.store(Bs + pbuf * TS * S::BS, Cs + pbuf * TS * S::BS, S::BS);
+      if (st > 1) bc.load(gB, gC, n_rows, (st - 2) * TS, L, vec);
     }
-    const float *Bst = Bs + buf * kT * S::BS;
-    const float *Cst = Cs + buf * kT * S::BS;
+    const float *Bst = Bs + buf * TS * S::BS;
+    const float *Cst = Cs + buf * TS * S::BS;
     const Tin *xrow = xs + (buf * CH + c) * S::XS + kPre;
-    const Tin *dtrow = dts + (buf * CH + c) * kT;
-    const Tin *zrow = zs + (buf * CH + c) * kT;
-    const Tin *dorow = dos + (buf * CH + c) * kT;
+    const Tin *dtrow = dts + (buf * CH + c) * TS;
+    const Tin *zrow = zs + (buf * CH + c) * TS;
+    const Tin *dorow = dos + (buf * CH + c) * TS;
     if (st == 0 && has_conv && p.conv_hist && p.K > 1) {
       // the carried inputs before step 0 (newest-first) replace the zero fill of the prefix
       if (live && g == 0) {
@@ -203,242 +220,272 @@ ssm_bwd_kernel(const BwdParams P) {
       }
       __syncwarp();
     }
+    const int tb = g * EPL;  // first owned step (stage-local)
 
+    // (A) per-element values of the owned steps: (Delta, u, dy, dSiLU/dc) -> e3, (dDelta/dv,
+    //     dout/dz) -> pe
+    {
+      float xw[EPL + 4], dtw[EPL], zw[EPL], dow[EPL];
+      load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+      load_window<Tin, EPL>(dtw, dtrow + tb);
+      load_window<Tin, EPL>(dow, dorow + tb);
+      if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
 #pragma unroll
-    for (int sb = kT / kSub - 1; sb >= 0; sb--) {
-      const int tb = sb * kSub + g * EPL;  // first owned step (stage-local)
-      const int64_t tblk = t0 + sb * kSub;  // first step of the block (global)
-      // (A) per-element values of the owned steps: u, Delta, dy -> e3
-      {
-        float xw[EPL + 4], dtw[EPL], zw[EPL], dow[EPL];
-        load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
-        load_window<Tin, EPL>(dtw, dtrow + tb);
-        load_window<Tin, EPL>(dow, dorow + tb);
-        if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
+      for (int j = 0; j < EPL; j++) {
+        // u = SiLU(c) with dSiLU/dc = s (1 + c (1 - s)); Delta = softplus(v) with dDelta/dv =
+        // sigmoid(v); out = y SiLU(z) with dout/dz = y s_z (1 + z (1 - s_z))
+        float u, gc = 1.f;
+        if (has_conv) {
+          float acc = cbias;
 #pragma unroll
-        for (int j = 0; j < EPL; j++) {
-          // u = SiLU(c) with dSiLU/dc = s (1 + c (1 - s)); Delta = softplus(v) with dDelta/dv =
-          // sigmoid(v); out = y SiLU(z) with dout/dz = y s_z (1 + z (1 - s_z))
-          float u, gc = 1.f;
-          if (has_conv) {
-            float acc = cbias;
+          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
+          const float sc = sigmoid<PRECISE>(acc);
+          u = acc * sc;
+          gc = sc * fmaf(acc, 1.f - sc, 1.f);
+        } else {
+          u = xw[j + 4];
+        }
+        const float v = dtw[j] + dtb;
+        float dl = v, sv = 1.f;
+        if (p.delta_softplus) {
+          dl = softplus<PRECISE>(v);
+          sv = sigmoid<PRECISE>(v);
+        }
+        float dy = dow[j], gz = 0.f;
+        if (has_z) {
+          const float sz = sigmoid<PRECISE>(zw[j]);
+          dy *= zw[j] * sz;
+          gz = dow[j] * sz * fmaf(zw[j], 1.f - sz, 1.f);
+        }
+        if (t0 + tb + j >= L) {  // padded steps are identity steps with no inputs
+          u = 0.f;
+          dl = 0.f;
+          dy = 0.f;
+          gc = 0.f;
+          sv = 0.f;
+          gz = 0.f;
+        }
+        e3[c * S::ES + tb + j] = make_float4(dl, u, dy, gc);
+        pe[c * S::ES + tb + j] = make_float2(sv, gz);
+      }
+    }
+    __syncwarp();
+
+    // (B) recompute the stage forward from its saved start state; h and A_bar of every step go
+    //     to TMEM, the readout partials to y0
+    {
+      float2 h2[NH];
+      float *h = reinterpret_cast<float *>(h2);
 #pragma unroll
-            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], xw[j + 4 - k], acc);
-            const float sc = sigmoid<PRECISE>(acc);
-            u = acc * sc;
-            gc = sc * fmaf(acc, 1.f - sc, 1.f);
+      for (int j = 0; j < 2 * NH; j++) {
+        const int n = g * NS + j;
+        h[j] = 0.f;
+        if (j < NS && live && n < N) {
+          if (st > 0)
+            h[j] = states[((b * p.Dn + d) * p.n_ck + (st - 1)) * N + n];
+          else if (p.h0)
+            h[j] = p.h0[(b * p.Dn + d) * N + n];
+        }
+      }
+      float *my0 = y0 + c * S::YC + g * S::YG;
+#pragma unroll
+      for (int tq = 0; tq < TS; tq += 4) {
+        float4 eq[4];
+        float2 Bq[4][NH], Cq[4][NH];
+#pragma unroll
+        for (int tt = 0; tt < 4; tt++) {
+          const int t = tq + tt;
+          eq[tt] = e3[c * S::ES + t];
+          load_states<NS>(reinterpret_cast<float *>(Bq[tt]), Bst + t * S::BS + g * NS);
+          load_states<NS>(reinterpret_cast<float *>(Cq[tt]), Cst + t * S::BS + g * NS);
+        }
+        float hv[GV], av[GV], yq[4];
+#pragma unroll
+        for (int tt = 0; tt < 4; tt++) {
+          if (PAIRS) {
+            const float2 dl2 = make_float2(eq[tt].x, eq[tt].x), u2 = make_float2(eq[tt].y, eq[tt].y);
+            float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < NH; q++) {
+              const float2 x = __fmul2_rn(dl2, Ac2[q]);
+              float2 a;
+              a.x = ex2_approx(x.x);
+              a.y = ex2_approx(x.y);
+              if (EULER) {
+                h2[q] = __ffma2_rn(a, h2[q], __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), dl2));  // a h + Delta B u
+              } else {
+                const float2 nw = __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), nIA2[q]);  // -B u / A
+                h2[q] = __ffma2_rn(a, __ffma2_rn(nw, make_float2(-1.f, -1.f), h2[q]), nw);
+              }
+              av[tt * NS + 2 * q] = a.x;
+              av[tt * NS + 2 * q + 1] = a.y;
+              hv[tt * NS + 2 * q] = h2[q].x;
+              hv[tt * NS + 2 * q + 1] = h2[q].y;
+              y2 = __ffma2_rn(Cq[tt][q], h2[q], y2);
+            }
+            yq[tt] = y2.x + y2.y;
           } else {
-            u = xw[j + 4];
-          }
-          const float v = dtw[j] + dtb;
-          float dl = v, sv = 1.f;
-          if (p.delta_softplus) {
-            dl = softplus<PRECISE>(v);
-            sv = sigmoid<PRECISE>(v);
-          }
-          float dy = dow[j], gz = 0.f;
-          if (has_z) {
-            const float sz = sigmoid<PRECISE>(zw[j]);
-            dy *= zw[j] * sz;
-            gz = dow[j] * sz * fmaf(zw[j], 1.f - sz, 1.f);
-          }
-          if (t0 + tb + j >= L) {
-            u = 0.f;
-            dl = 0.f;
-            dy = 0.f;
-            gc = 0.f;
-            sv = 0.f;
-            gz = 0.f;
-          }
-          e3[c * S::ES + g * EPL + j] = make_float4(dl, u, dy, 0.f);
-          pe[c * S::ES + g * EPL + j] = make_float4(gc, sv, gz, 0.f);
-        }
-      }
-      __syncwarp();
-
-      // (B) recompute the block forward from its saved start state; keep A_bar (or A_bar - 1
-      //     on the precise path) and h of every step in registers
-      float2 ea2[kSub][NH], hs2[kSub][NH];
-      {
-        float2 h2[NH];
-        float *h = reinterpret_cast<float *>(h2);
-        const int64_t kk = tblk / kSub;
+            const float *Bt = reinterpret_cast<const float *>(Bq[tt]);
+            const float *Ct = reinterpret_cast<const float *>(Cq[tt]);
+            float y = 0.f;
 #pragma unroll
-        for (int j = 0; j < 2 * NH; j++) {
-          const int n = g * NS + j;
-          h[j] = 0.f;
-          if (j < NS && live && n < N) {
-            if (kk > 0)
-              h[j] = states[((b * p.Dn + d) * p.n_ck + (kk - 1)) * N + n];
-            else if (p.h0)
-              h[j] = p.h0[(b * p.Dn + d) * N + n];
-          }
-        }
-        float *my0 = y0 + c * S::YC + g * S::YG;
-#pragma unroll
-        for (int tq = 0; tq < kSub; tq += 4) {
-          float4 eq[4];
-          float2 Bq[4][NH], Cq[4][NH];
-#pragma unroll
-          for (int tt = 0; tt < 4; tt++) {
-            const int t = sb * kSub + tq + tt;
-            eq[tt] = e3[c * S::ES + tq + tt];
-            load_states<NS>(reinterpret_cast<float *>(Bq[tt]), Bst + t * S::BS + g * NS);
-            load_states<NS>(reinterpret_cast<float *>(Cq[tt]), Cst + t * S::BS + g * NS);
-          }
-          float yq[4];
-#pragma unroll
-          for (int tt = 0; tt < 4; tt++) {
-            if (PAIRS) {
-              const float2 dl2 = make_float2(eq[tt].x, eq[tt].x), u2 = make_float2(eq[tt].y, eq[tt].y);
-              float2 y2 = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int q = 0; q < NH; q++) {
-                const float2 x = __fmul2_rn(dl2, Ac2[q]);
-                float2 a;
-                a.x = ex2_approx(x.x);
-                a.y = ex2_approx(x.y);
-                if (EULER) {
-                  h2[q] = __ffma2_rn(a, h2[q], __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), dl2));  // a h + Delta B u
-                } else {
-                  const float2 nw = __fmul2_rn(__fmul2_rn(Bq[tt][q], u2), nIA2[q]);  // -B u / A
-                  h2[q] = __ffma2_rn(a, __ffma2_rn(nw, make_float2(-1.f, -1.f), h2[q]), nw);
-                }
-                ea2[tq + tt][q] = a;
-                hs2[tq + tt][q] = h2[q];
-                y2 = __ffma2_rn(Cq[tt][q], h2[q], y2);
+            for (int j = 0; j < NS; j++) {
+              const float nw = Bt[j] * eq[tt].y * nIA[j];  // -B u / A
+              if (PRECISE) {
+                const float em1 = expm1f(eq[tt].x * Acoef[j]);
+                h[j] = EULER ? fmaf(em1, h[j], fmaf(eq[tt].x * Bt[j], eq[tt].y, h[j]))
+                             : fmaf(em1, h[j] - nw, h[j]);
+                av[tt * NS + j] = em1;
+              } else {
+                const float a = ex2_approx(eq[tt].x * Acoef[j]);
+                h[j] = EULER ? fmaf(a, h[j], eq[tt].x * Bt[j] * eq[tt].y) : fmaf(a, h[j] - nw, nw);
+                av[tt * NS + j] = a;
               }
-              yq[tt] = y2.x + y2.y;
-            } else {
-              const float *Bt = reinterpret_cast<const float *>(Bq[tt]);
-              const float *Ct = reinterpret_cast<const float *>(Cq[tt]);
-              float *eat = reinterpret_cast<float *>(ea2[tq + tt]);
-              float *hst = reinterpret_cast<float *>(hs2[tq + tt]);
-              float y = 0.f;
-#pragma unroll
-              for (int j = 0; j < NS; j++) {
-                const float nw = Bt[j] * eq[tt].y * nIA[j];  // -B u / A
-                if (PRECISE) {
-                  const float em1 = expm1f(eq[tt].x * Acoef[j]);
-                  h[j] = EULER ? fmaf(em1, h[j], fmaf(eq[tt].x * Bt[j], eq[tt].y, h[j]))
-                               : fmaf(em1, h[j] - nw, h[j]);
-                  eat[j] = em1;
-                } else {
-                  const float a = ex2_approx(eq[tt].x * Acoef[j]);
-                  h[j] = EULER ? fmaf(a, h[j], eq[tt].x * Bt[j] * eq[tt].y) : fmaf(a, h[j] - nw, nw);
-                  eat[j] = a;
-                }
-                hst[j] = h[j];
-                y = fmaf(Ct[j], h[j], y);
-              }
-              yq[tt] = y;
+              hv[tt * NS + j] = h[j];
+              y = fmaf(Ct[j], h[j], y);
             }
+            yq[tt] = y;
           }
-          *reinterpret_cast<float4 *>(my0 + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
         }
+        *reinterpret_cast<float4 *>(my0 + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
+        __syncwarp();  // the TMEM stores are warp-collective
+        tmem_st<GV>(th + tq * NS, hv);
+        tmem_st<GV>(ta + tq * NS, av);
       }
-      __syncwarp();
-      float yfin[EPL];
-      {
-        float o[EPL];
+    }
+    tmem_wait_st();
+    __syncwarp();
+    float yfin[EPL];
+    {
+      float o[EPL];
 #pragma unroll
-        for (int j = 0; j < EPL; j++) o[j] = 0.f;
+      for (int j = 0; j < EPL; j++) o[j] = 0.f;
 #pragma unroll
-        for (int gg = 0; gg < G; gg++) {
-          float part[EPL];
-          load_floats<EPL>(part, y0 + c * S::YC + gg * S::YG + g * EPL);
+      for (int gg = 0; gg < G; gg++) {
+        float part[EPL];
+        load_floats<EPL>(part, y0 + c * S::YC + gg * S::YG + tb);
 #pragma unroll
-          for (int j = 0; j < EPL; j++) o[j] += part[j];
-        }
-#pragma unroll
-        for (int j = 0; j < EPL; j++) yfin[j] = fmaf(Dd, e3[c * S::ES + g * EPL + j].y, o[j]);
+        for (int j = 0; j < EPL; j++) o[j] += part[j];
       }
-      __syncwarp();  // y0 is reused for the du partials
+#pragma unroll
+      for (int j = 0; j < EPL; j++) yfin[j] = fmaf(Dd, e3[c * S::ES + tb + j].y, o[j]);
+    }
+    __syncwarp();  // y0 is reused for the du partials
 
-      // (C) the adjoint backwards through the block, in two halves of RH steps; each half's
-      //     dB / dC partials are summed over the CTA's channels right after it
+    // (C) the adjoint backwards through the stage, one 4-step TMEM group per quarter; each
+    //     quarter's dB / dC partials are summed over the CTA's channels right after it
+    float duo[EPL], ddo[EPL];  // lane sums of du / dDelta of the owned steps (shuffle path)
 #pragma unroll
-      for (int hf = kSub / RH - 1; hf >= 0; hf--) {
-        float *my0 = y0 + c * S::YC + g * S::YG;
-        float *my1 = y1 + c * S::YC + g * S::YG;
+    for (int j = 0; j < EPL; j++) {
+      duo[j] = 0.f;
+      ddo[j] = 0.f;
+    }
 #pragma unroll
-        for (int tq = hf * RH + RH - 4; tq >= hf * RH; tq -= 4) {
-          float duq[4], ddq[4];
+    for (int hf = TS / RH - 1; hf >= 0; hf--) {
+      const int tq = hf * RH;
+      float hv[GV], av[GV];
+      tmem_ld2<GV>(th + tq * NS, hv, ta + tq * NS, av);
+      float duq[4], ddq[4];
 #pragma unroll
-          for (int tt = 3; tt >= 0; tt--) {
-            const int tl = tq + tt, t = sb * kSub + tl;
-            const float4 e = e3[c * S::ES + tl];  // (dl, u, dy, -)
-            float2 Bv[NH], Cv[NH];
-            load_states<NS>(reinterpret_cast<float *>(Bv), Bst + t * S::BS + g * NS);
-            load_states<NS>(reinterpret_cast<float *>(Cv), Cst + t * S::BS + g * NS);
-            float2 nB2[NH], dC2[NH];
-            float *nB = reinterpret_cast<float *>(nB2);
-            float *dCv = reinterpret_cast<float *>(dC2);
-            float ndu = 0.f, dd = 0.f;
-            if (PAIRS) {
-              float2 ndu2 = make_float2(0.f, 0.f), dd2 = make_float2(0.f, 0.f);
-              const float2 dl2 = make_float2(e.x, e.x), u2 = make_float2(e.y, e.y), dy2 = make_float2(e.z, e.z);
+      for (int tt = 3; tt >= 0; tt--) {
+        const int tl = tq + tt;
+        const float4 e = e3[c * S::ES + tl];  // (dl, u, dy, gc)
+        float2 Bv[NH], Cv[NH];
+        load_states<NS>(reinterpret_cast<float *>(Bv), Bst + tl * S::BS + g * NS);
+        load_states<NS>(reinterpret_cast<float *>(Cv), Cst + tl * S::BS + g * NS);
+        float2 nB2[NH], dC2[NH];
+        float *nB = reinterpret_cast<float *>(nB2);
+        float *dCv = reinterpret_cast<float *>(dC2);
+        float ndu = 0.f, dd = 0.f;
+        if (PAIRS) {
+          float2 ndu2 = make_float2(0.f, 0.f), dd2 = make_float2(0.f, 0.f);
+          const float2 dl2 = make_float2(e.x, e.x), u2 = make_float2(e.y, e.y), dy2 = make_float2(e.z, e.z);
 #pragma unroll
-              for (int q = 0; q < NH; q++) {
-                const float2 an2 = (tl + 1 < kSub) ? ea2[tl + 1][q] : aN2[q];
-                lam2[q] = __ffma2_rn(an2, lam2[q], __fmul2_rn(Cv[q], dy2));           // lambda_t
-                // kb = -dB_bar/dB: (A_bar - 1)(-1/A) for the exact ZOH, -Delta for Euler
-                const float2 em1n = EULER ? make_float2(-e.x, -e.x)
-                                          : __fmul2_rn(__fadd2_rn(ea2[tl][q], make_float2(-1.f, -1.f)), nIA2[q]);
-                const float2 nlb = __fmul2_rn(lam2[q], __fmul2_rn(em1n, Bv[q]));      // -lambda B_bar
-                ndu2 = __fadd2_rn(ndu2, nlb);
-                nB2[q] = __fmul2_rn(__fmul2_rn(lam2[q], em1n), u2);                   // -dB partial
-                dC2[q] = __fmul2_rn(hs2[tl][q], dy2);
-                // dh_t/dDelta = A h_t + B u (ZOH) or A h_t + B u (1 - A Delta) (Euler)
-                float2 bu = __fmul2_rn(Bv[q], u2);
-                if (EULER) bu = __fmul2_rn(bu, __ffma2_rn(A2[q], make_float2(-e.x, -e.x), make_float2(1.f, 1.f)));
-                const float2 dterm = __fmul2_rn(lam2[q], __ffma2_rn(A2[q], hs2[tl][q], bu));
-                dd2 = __fadd2_rn(dd2, dterm);
-                dAl2[q] = __ffma2_rn(u2, nlb, __ffma2_rn(dl2, dterm, dAl2[q]));       // A dA
-              }
-              ndu = ndu2.x + ndu2.y;
-              dd = dd2.x + dd2.y;
-            } else {
-              const float *Bt = reinterpret_cast<const float *>(Bv);
-              const float *Ct = reinterpret_cast<const float *>(Cv);
-              const float *eat = reinterpret_cast<const float *>(ea2[tl]);
-              const float *ean = reinterpret_cast<const float *>(tl + 1 < kSub ? ea2[tl + 1] : aN2);
-              const float *hst = reinterpret_cast<const float *>(hs2[tl]);
-#pragma unroll
-              for (int j = 0; j < NS; j++) {
-                const float em1 = PRECISE ? eat[j] : eat[j] - 1.f;
-                const float an = (PRECISE && tl + 1 < kSub) ? 1.f + ean[j] : ean[j];
-                lam[j] = fmaf(an, lam[j], Ct[j] * e.z);
-                const float em1n = EULER ? -e.x : em1 * nIA[j];
-                const float nlb = lam[j] * (em1n * Bt[j]);
-                ndu += nlb;
-                nB[j] = lam[j] * em1n * e.y;
-                dCv[j] = hst[j] * e.z;
-                const float bu = EULER ? Bt[j] * e.y * fmaf(-A[j], e.x, 1.f) : Bt[j] * e.y;
-                const float dterm = lam[j] * fmaf(A[j], hst[j], bu);
-                dd += dterm;
-                dAl[j] = fmaf(e.y, nlb, fmaf(e.x, dterm, dAl[j]));
-              }
-            }
-            store_states<NS>(rb + S::rb_index(0, tl - hf * RH, c, g * NS), nB);
-            store_states<NS>(rb + S::rb_index(1, tl - hf * RH, c, g * NS), dCv);
-            duq[tt] = -ndu;
-            ddq[tt] = dd;
+          for (int q = 0; q < NH; q++) {
+            const float2 a2 = make_float2(av[tt * NS + 2 * q], av[tt * NS + 2 * q + 1]);
+            const float2 hs = make_float2(hv[tt * NS + 2 * q], hv[tt * NS + 2 * q + 1]);
+            lam2[q] = __ffma2_rn(aN2[q], lam2[q], __fmul2_rn(Cv[q], dy2));         // lambda_t
+            aN2[q] = a2;
+            // kb = -dB_bar/dB: (A_bar - 1)(-1/A) for the exact ZOH, -Delta for Euler
+            const float2 em1n = EULER ? make_float2(-e.x, -e.x)
+                                      : __fmul2_rn(__fadd2_rn(a2, make_float2(-1.f, -1.f)), nIA2[q]);
+            const float2 k = __fmul2_rn(lam2[q], em1n);
+            const float2 nlb = __fmul2_rn(k, Bv[q]);                                // -lambda B_bar
+            ndu2 = __fadd2_rn(ndu2, nlb);
+            nB2[q] = __fmul2_rn(k, u2);                                             // -dB partial
+            dC2[q] = __fmul2_rn(hs, dy2);
+            // dh_t/dDelta = A h_t + B u (ZOH) or A h_t + B u (1 - A Delta) (Euler)
+            float2 bu = __fmul2_rn(Bv[q], u2);
+            if (EULER) bu = __fmul2_rn(bu, __ffma2_rn(A2[q], make_float2(-e.x, -e.x), make_float2(1.f, 1.f)));
+            const float2 dterm = __fmul2_rn(lam2[q], __ffma2_rn(A2[q], hs, bu));
+            dd2 = __fadd2_rn(dd2, dterm);
+            dAl2[q] = __ffma2_rn(u2, nlb, __ffma2_rn(dl2, dterm, dAl2[q]));       // A dA
           }
-          *reinterpret_cast<float4 *>(my0 + tq) = make_float4(duq[0], duq[1], duq[2], duq[3]);
-          *reinterpret_cast<float4 *>(my1 + tq) = make_float4(ddq[0], ddq[1], ddq[2], ddq[3]);
+          ndu = ndu2.x + ndu2.y;
+          dd = dd2.x + dd2.y;
+        } else {
+          const float *Bt = reinterpret_cast<const float *>(Bv);
+          const float *Ct = reinterpret_cast<const float *>(Cv);
+#pragma unroll
+          for (int j = 0; j < NS; j++) {
+            const float em1 = PRECISE ? av[tt * NS + j] : av[tt * NS + j] - 1.f;
+            const float hs = hv[tt * NS + j];
+            lam[j] = fmaf(aN[j], lam[j], Ct[j] * e.z);
+            aN[j] = PRECISE ? 1.f + av[tt * NS + j] : av[tt * NS + j];
+            const float em1n = EULER ? -e.x : em1 * nIA[j];
+            const float nlb = lam[j] * (em1n * Bt[j]);
+            ndu += nlb;
+            nB[j] = lam[j] * em1n * e.y;
+            dCv[j] = hs * e.z;
+            const float bu = EULER ? Bt[j] * e.y * fmaf(-A[j], e.x, 1.f) : Bt[j] * e.y;
+            const float dterm = lam[j] * fmaf(A[j], hs, bu);
+            dd += dterm;
+            dAl[j] = fmaf(e.y, nlb, fmaf(e.x, dterm, dAl[j]));
+          }
         }
-        __syncthreads();  // the half-block's dB / dC partials of every channel are in place
-        {
-          constexpr int NQ = NP / 4;
-          constexpr int NGRP = 2 * RH * NQ;
-          constexpr int SPLIT = NGRP >= kThreads ? 1 : (kThreads / NGRP > 2 ? 2 : kThreads / NGRP);
-          constexpr int CPS = CH / SPLIT;
-          const int part = tid % SPLIT;
-          for (int gi = tid / SPLIT; gi < NGRP; gi += kThreads / SPLIT) {
-            const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
-            float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
-            if (CPS == S::CHH || CPS * 2 == S::CHH || CPS * 4 == S::CHH) {
+        store_states<NS>(rb + S::rb_index(0, tt, c, g * NS), nB);
+        store_states<NS>(rb + S::rb_index(1, tt, c, g * NS), dCv);
+        if (S::SHFL) {
+          // sum over the channel's G lanes; the step's owner keeps it
+          float su = -ndu, sd = dd;
+#pragma unroll
+          for (int off = 1; off < G; off <<= 1) {
+            su += __shfl_xor_sync(0xffffffffu, su, off);
+            sd += __shfl_xor_sync(0xffffffffu, sd, off);
+          }
+          if (g == tl / EPL) {
+            duo[tl % EPL] = su;
+            ddo[tl % EPL] = sd;
+          }
+        } else {
+          duq[tt] = -ndu;
+          ddq[tt] = dd;
+        }
+      }
+      if (!S::SHFL) {
+        *reinterpret_cast<float4 *>(y0 + c * S::YC + g * S::YG + tq) = make_float4(duq[0], duq[1], duq[2], duq[3]);
+        *reinterpret_cast<float4 *>(y1 + c * S::YC + g * S::YG + tq) = make_float4(ddq[0], ddq[1], ddq[2], ddq[3]);
+      }
+      __syncthreads();  // the quarter's dB / dC partials of every channel are in place
+      {
+        // every thread runs the same number of rounds, so the shuffles below see whole warps
+        // (threads without a column still take part in them)
+        constexpr int NQ = NP / 4;
+        constexpr int NGRP = 2 * RH * NQ;
+        // two threads per column: fewer shuffles than a wider split, and half the CTA's warps
+        // stay free (measured fastest on B200)
+        constexpr int SPLIT = NGRP >= kThreads ? 1 : 2;
+        constexpr int CPS = CH / SPLIT;
+        constexpr int ROUNDS = (NGRP * SPLIT + kThreads - 1) / kThreads;
+        const int part = tid % SPLIT;
+#pragma unroll
+        for (int r = 0; r < ROUNDS; r++) {
+          const int gi = (r * kThreads + tid) / SPLIT;
+          const bool ok = gi < NGRP;
+          const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
+          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+          if (ok) {
+            if (SPLIT > 1) {
               // this thread's channels lie in one half: walk them with a fixed stride
               const float *src = rb + S::rb_index(which, tt, part * CPS, 4 * q);
 #pragma unroll 8
@@ -450,38 +497,45 @@ ssm_bwd_kernel(const BwdParams P) {
             } else {
 #pragma unroll 4
               for (int ci = 0; ci < CPS; ci++) {
-                const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, part * CPS + ci, 4 * q));
+                const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, ci, 4 * q));
                 a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
                 a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
               }
             }
-            float4 acc = make_float4(a01.x, a01.y, a23.x, a23.y);
+          }
+          float4 acc = make_float4(a01.x, a01.y, a23.x, a23.y);
 #pragma unroll
-            for (int off = 1; off < SPLIT; off <<= 1) {
-              acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
-              acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-              acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
-              acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-            }
-            const int64_t t = tblk + hf * RH + tt;
-            if (part == 0 && t < L) {
-              float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
-              const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
-              const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+          for (int off = 1; off < SPLIT; off <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+          }
+          const int64_t t = t0 + tq + tt;
+          if (ok && part == 0 && t < L) {
+            float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
+            const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
+            const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-              for (int k = 0; k < 4; k++)
-                if (4 * q + k < N) dst[(int64_t)(4 * q + k) * L] = sg * vals[k];
-            }
+            for (int k = 0; k < 4; k++)
+              if (4 * q + k < N) dst[(int64_t)(4 * q + k) * L] = sg * vals[k];
           }
         }
-        __syncthreads();  // rb is rewritten by the next half
       }
-#pragma unroll
-      for (int q = 0; q < NH; q++) aN2[q] = PRECISE ? make_float2(1.f + ea2[0][q].x, 1.f + ea2[0][q].y) : ea2[0][q];
+      __syncthreads();  // rb is rewritten by the next quarter
+    }
 
-      // (D) per-element gradients of the owned steps
-      {
-        float dup[EPL], ddp[EPL];
+    __syncwarp();  // the du / dDelta partial rows (shared-memory path) are complete
+    // (D) per-element gradients of the owned steps
+    {
+      float dup[EPL], ddp[EPL];
+      if (S::SHFL) {
+#pragma unroll
+        for (int j = 0; j < EPL; j++) {
+          dup[j] = duo[j];
+          ddp[j] = ddo[j];
+        }
+      } else {
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
           dup[j] = 0.f;
@@ -490,40 +544,40 @@ ssm_bwd_kernel(const BwdParams P) {
 #pragma unroll
         for (int gg = 0; gg < G; gg++) {
           float a0[EPL], a1[EPL];
-          load_floats<EPL>(a0, y0 + c * S::YC + gg * S::YG + g * EPL);
-          load_floats<EPL>(a1, y1 + c * S::YC + gg * S::YG + g * EPL);
+          load_floats<EPL>(a0, y0 + c * S::YC + gg * S::YG + tb);
+          load_floats<EPL>(a1, y1 + c * S::YC + gg * S::YG + tb);
 #pragma unroll
           for (int j = 0; j < EPL; j++) {
             dup[j] += a0[j];
             ddp[j] += a1[j];
           }
         }
-        float xw[EPL + 4];
-        if (has_conv) load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
-        float dzv[EPL], dtv[EPL], dcv[EPL];
+      }
+      float xw[EPL + 4];
+      if (has_conv) load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
+      float dzv[EPL], dtv[EPL], dcv[EPL];
 #pragma unroll
-        for (int j = 0; j < EPL; j++) {
-          const float4 e = e3[c * S::ES + g * EPL + j];  // (dl, u, dy, -); zero past L
-          const float4 f = pe[c * S::ES + g * EPL + j];  // (gc, sv, gz, -); zero past L
-          const float du = fmaf(Dd, e.z, dup[j]);
-          accD = fmaf(e.z, e.y, accD);
-          dzv[j] = yfin[j] * f.z;
-          dtv[j] = ddp[j] * f.y;
-          accDtb += dtv[j];
-          dcv[j] = du * f.x;
-          if (has_conv) {
-            dcs[c * S::DCS + tb + j] = dcv[j];
-            accCb += dcv[j];
+      for (int j = 0; j < EPL; j++) {
+        const float4 e = e3[c * S::ES + tb + j];  // (dl, u, dy, gc); zero past L
+        const float2 f = pe[c * S::ES + tb + j];  // (sv, gz); zero past L
+        const float du = fmaf(Dd, e.z, dup[j]);
+        accD = fmaf(e.z, e.y, accD);
+        dzv[j] = yfin[j] * f.y;
+        dtv[j] = ddp[j] * f.x;
+        accDtb += dtv[j];
+        dcv[j] = du * e.w;
+        if (has_conv) {
+          dcs[c * S::DCS + tb + j] = dcv[j];
+          accCb += dcv[j];
 #pragma unroll
-            for (int k = 0; k < 4; k++) accW[k] = fmaf(dcv[j], xw[j + 4 - k], accW[k]);
-          }
+          for (int k = 0; k < 4; k++) accW[k] = fmaf(dcv[j], xw[j + 4 - k], accW[k]);
         }
-        if (live) {
-          const int64_t roff = (b * p.Dn + d) * L;
-          if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, L, dzv, vec);
-          if (P.ddt) store_run<float, EPL>(P.ddt + roff, t0 + tb, L, dtv, vec);
-          if (!has_conv && P.dx) store_run<float, EPL>(P.dx + roff, t0 + tb, L, dcv, vec);
-        }
+      }
+      if (live) {
+        const int64_t roff = (b * p.Dn + d) * L;
+        if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, L, dzv, vec);
+        if (P.ddt) store_run<float, EPL>(P.ddt + roff, t0 + tb, L, dtv, vec);
+        if (!has_conv && P.dx) store_run<float, EPL>(P.dx + roff, t0 + tb, L, dcv, vec);
       }
     }
 
@@ -531,19 +585,17 @@ ssm_bwd_kernel(const BwdParams P) {
     // dcs rows are written and read by the G lanes of their own channel only.
     if (has_conv) {
       __syncwarp();
-#pragma unroll
-      for (int sb = 0; sb < kT / kSub; sb++) {
+      {
         float dxv[EPL];
 #pragma unroll
         for (int j = 0; j < EPL; j++) {
-          const int t = sb * kSub + g * EPL + j;
+          const int t = tb + j;
           float acc = 0.f;
 #pragma unroll
           for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
           dxv[j] = acc;
         }
-        if (live && P.dx)
-          store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + sb * kSub + g * EPL, L, dxv, vec);
+        if (live && P.dx) store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + tb, L, dxv, vec);
       }
       __syncwarp();
       if (st == 0 && live && g == 0 && P.dconv_hist && p.K > 1) {
@@ -556,7 +608,7 @@ ssm_bwd_kernel(const BwdParams P) {
       }
       // this stage's first 3 dc values become the halo of the stage before it
       if (g == 0)
-        for (int k = 0; k < 3; k++) dcs[c * S::DCS + kT + k] = dcs[c * S::DCS + k];
+        for (int k = 0; k < 3; k++) dcs[c * S::DCS + TS + k] = dcs[c * S::DCS + k];
       __syncwarp();
     }
   }
@@ -588,6 +640,7 @@ ssm_bwd_kernel(const BwdParams P) {
     P.p_dconv_b[bd] = accCb;
     for (int k = 0; k < 4; k++) P.p_dconv_w[bd * 4 + k] = accW[k];
   }
+  tmem_free_cta(tbase, S::NCOLS);
 }
 
 // dB/dC: add the channel-tile partials in tile order.
@@ -651,11 +704,24 @@ template <int G, int NS, typename Tin>
 static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   using S = BwdSmem<G, NS, Tin>;
   auto kern = P.f.euler ? ssm_bwd_kernel<G, NS, Tin, true> : ssm_bwd_kernel<G, NS, Tin, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
+  // Each resident CTA holds S::NCOLS of the SM's 512 TMEM columns. Ask for enough shared memory
+  // that no more CTAs fit on an SM than the columns allow, so no allocation ever has to wait.
+  int dev = 0, smem_sm = 0, reserved = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  size_t smem = S::bytes;
+  const int max_ctas = 512 / (int)S::NCOLS;
+  if (max_ctas < kMaxThreadsPerSM / kThreads) {
+    const size_t floor_bytes = (size_t)smem_sm / (max_ctas + 1) + 16 - (size_t)reserved;
+    if (smem < floor_bytes) smem = (floor_bytes + 15) & ~size_t(15);
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = P.n_dtiles * P.f.Bt;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)grid, kThreads, S::bytes, stream>>>(P);
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(P);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@ constexpr int kThreads = 128;  // threads per CTA for the scan kernels
 constexpr int kT = 32;         // time steps staged per CTA pipeline stage
 constexpr int kSub = 16;       // recompute / state-save block (SSM_STATE_CHUNK)
 constexpr int kPre = 8;        // conv halo prefix kept in front of each staged x row
+constexpr int kMaxThreadsPerSM = 2048;  // resident threads per SM on sm_100
 
 // Lane layout of the scan kernels: a channel's N states are spread over G adjacent lanes of one
 // warp, NS states per lane (G * NS >= N, padded states are inert).

@@ -132,13 +132,13 @@ template <int NS> __device__ __forceinline__ void load_states(float *dst, const 
   load_floats<NS>(dst, src);
 }
 
-// B and C of one stage (NP rows x kT steps, row stride L in global memory) go global ->
+// B and C of one stage (NP rows x LEN steps, row stride L in global memory) go global ->
 // registers -> transposed fp32 rows [t][n] in shared memory, so that the scan reads all of a
 // lane's states at one step with one 16-byte broadcast load. Loads for stage s+1 are issued one
 // stage early into registers; the transposed stores happen after the next barrier-free point.
-template <typename Tin, int NP, int NT = kThreads> struct BCStager {
+template <typename Tin, int NP, int NT = kThreads, int LEN = kT> struct BCStager {
   static constexpr int EPV = 16 / sizeof(Tin);               // elements per 16-byte vector
-  static constexpr int VPR = kT / EPV;                       // vectors per row
+  static constexpr int VPR = LEN / EPV;                      // vectors per row
   static constexpr int NV = 2 * NP * VPR;                    // B and C vectors per stage
   static constexpr int PER = (NV + NT - 1) / NT;             // per thread
   uint4 v[PER];
