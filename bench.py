@@ -468,11 +468,14 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        n_ch = min(w.Bt * w.Dn, 256 * threads)
+        # a short calibration sample sizes the measured one to about 12 s of host work
+        c_secs, c_done = oracle_sample(w, a, 16 * threads, threads)
+        per_ch = c_secs / (16 * threads)
+        n_ch = int(min(4 * w.Bt * w.Dn, max(16 * threads, 12.0 / max(per_ch, 1e-9))))
         secs, done = oracle_sample(w, a, n_ch, threads)
         cpu = {"value": done / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": "%d channels x L=%d x N=%d (fwd%s) of the same workload, float64, %.1f s"
-                         % (n_ch, L, N, "+bwd" if backward else "", secs)}
+               "sample": "%d channels (wrapping over the %d of the workload) x L=%d x N=%d (fwd%s), "
+                         "float64, %.1f s" % (n_ch, w.Bt * w.Dn, L, N, "+bwd" if backward else "", secs)}
 
     if rank == 0:
         line = {
