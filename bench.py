@@ -252,6 +252,8 @@ def main():
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n-segments", type=int, default=0,
+                    help="split-L for the forward: 0 one pass, k up to k segments, -1 automatic")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -314,6 +316,14 @@ def main():
                                 kw["dt_bias"], kw["conv_w"], kw["conv_b"], True, odt)
     fwd_args.out = out.data_ptr()
     fwd_args.chunk_states = states.data_ptr() if backward else None
+    ws_f = None
+    if args.n_segments:
+        fwd_args.n_segments = args.n_segments
+        need_f = lib.ssm_fwd_workspace_size(ctypes.byref(fwd_args))
+        if need_f:
+            ws_f = torch.empty(need_f + 256, dtype=torch.uint8, device=dev)
+            fwd_args.workspace = (ws_f.data_ptr() + 255) & ~255
+            fwd_args.workspace_bytes = need_f
     fwd_args_fo = _abi.FwdArgs.from_buffer_copy(fwd_args)
     fwd_args_fo.chunk_states = None
     if backward:
@@ -429,7 +439,8 @@ def main():
                 "peak_source": peaks.get("source")}
     else:
         roof = dict(fwd_roof)
-    launches_per_step = 1 + (3 if backward else 0)
+    # a split forward is three launches (segment summaries, carry, segments)
+    launches_per_step = (3 if ws_f is not None else 1) + (3 if backward else 0)
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, compute, D2H results ----
     names_in = ["x", "dt", "z", "B", "C"] + (["dout"] if backward else [])
@@ -488,7 +499,8 @@ def main():
                        "l2": "inputs larger than L2 (per-step working set %.2f GB)"
                              % ((fwd_bytes(Bt, Dn, N, L, s_in, s_out, backward)
                                  + (bwd_bytes(Bt, Dn, N, L, s_in) if backward else 0)) / 1e9),
-                       "parallelism": "replica per GPU" if world > 1 else "single GPU"},
+                       "parallelism": "replica per GPU" if world > 1 else "single GPU",
+                       "n_segments": args.n_segments},
             "roofline": roof,
             "alu_roofline": alu_roof("ssm_bwd_kernel" if backward else "ssm_fwd_kernel",
                                      kern["ssm_bwd_kernel"] if backward else fo_ms),

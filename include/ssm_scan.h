@@ -116,15 +116,37 @@ typedef struct ssm_fwd_args {
   void *conv_hist_out;   /* device (Bt, Dn, K-1) in_dtype or NULL: the K-1 newest pre-conv inputs
                             after this call, newest-first (may alias conv_hist) */
   int32_t discretization;/* ssm_discretization */
+  /* Split-L, for long sequences with few channels ("Sequence and state-space models", the
+   * chunked scan of affine pairs; "Selective Mamba", runArray over consecutive chunks): the
+   * sequence is cut into segments that run in parallel -- (1) every segment but the last runs
+   * from a zero state and keeps its end state and its sum of Delta, (2) the start state of every
+   * segment follows from those in one pass over the segments (the product of a segment's A_bar
+   * is exp(A * its sum of Delta)), (3) every segment runs from its start state, its conv prefix
+   * read from x. The results equal one pass up to fp32 rounding; the arithmetic is about 1.8x,
+   * for up to n_segments times the parallelism. ssm_scan_bwd ignores these three fields. */
+  int32_t n_segments;    /* 0 or 1: one pass. >= 2: up to that many segments, each a multiple of
+                            64 steps long. -1: chosen from the current device's SM count and the
+                            shape (one pass unless even 8 channels per CTA leave fewer than two
+                            CTAs per SM). */
+  void *workspace;       /* device scratch of at least ssm_fwd_workspace_size() bytes, 256-byte
+                            aligned, when the call splits L; may be NULL otherwise */
+  size_t workspace_bytes;
 } ssm_fwd_args;
 
 /*
  * Forward selective scan with the causal depthwise conv1d + SiLU fused in front and the SiLU(z)
  * gate fused behind: computes every output listed in ssm_fwd_args on `stream`.
- * Errors: SSM_ERR_NULL (x, dt, A_log, B, C or out NULL), SSM_ERR_SHAPE, SSM_ERR_ALIGN,
- * SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED (N > 64, K outside 1..4), SSM_ERR_CUDA.
+ * Errors: SSM_ERR_NULL (x, dt, A_log, B, C or out NULL), SSM_ERR_SHAPE (also n_segments < -1),
+ * SSM_ERR_ALIGN, SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED (N > 64, K outside 1..4), SSM_ERR_WORKSPACE
+ * (a split-L call whose workspace is NULL, too small or not 256-byte aligned), SSM_ERR_CUDA.
  */
 ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream);
+
+/* Bytes of workspace ssm_scan_fwd needs for these arguments: 0 when the call runs in one pass
+ * (n_segments 0 or 1, or a split that would leave a single segment), else 2 (n Bt Dn N) + n Bt Dn
+ * floats for n segments (each array rounded up to 256 bytes). With n_segments = -1 the answer
+ * depends on the current device (its SM count is read). Returns 0 for invalid arguments. */
+size_t ssm_fwd_workspace_size(const ssm_fwd_args *args);
 
 /*
  * Backward arguments: the forward's inputs (same meaning and dtypes; out/u_out unused) plus the

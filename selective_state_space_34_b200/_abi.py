@@ -31,6 +31,8 @@ class FwdArgs(ctypes.Structure):
         ("delta_softplus", ctypes.c_int32),
         ("h0", ctypes.c_void_p), ("conv_hist", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
         ("conv_hist_out", ctypes.c_void_p), ("discretization", ctypes.c_int32),
+        ("n_segments", ctypes.c_int32), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -63,6 +65,7 @@ class StepArgs(ctypes.Structure):
 SIGNATURES = [
     ("ssm_num_state_chunks", ctypes.c_int64, [ctypes.c_int64]),
     ("ssm_scan_fwd", ctypes.c_int, [ctypes.POINTER(FwdArgs), ctypes.c_void_p]),
+    ("ssm_fwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(FwdArgs)]),
     ("ssm_bwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(BwdArgs)]),
     ("ssm_scan_bwd", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_bwd_noalloc", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),

@@ -108,11 +108,15 @@ def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
 def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, conv_b=None,
                  delta_softplus: bool = True, out_dtype=None, save_states: bool = False,
                  return_u: bool = False, out: Optional[torch.Tensor] = None,
-                 discretization: str = "zoh", h0=None, conv_hist=None, return_state: bool = False):
+                 discretization: str = "zoh", h0=None, conv_hist=None, return_state: bool = False,
+                 n_segments: int = 0):
     """Fused forward. Returns ``out`` or a dict with ``out`` and, when asked, ``chunk_states``
     ((Bt, Dn, ceil(L/16), N) fp32, for ssm_scan_bwd), ``u`` (the scan input), and ``h_last`` /
     ``conv_hist`` (the state to carry into the next chunk). ``h0`` / ``conv_hist`` carry the state
-    in from a previous chunk; ``discretization`` is "zoh" (exact) or "euler" (Delta * B)."""
+    in from a previous chunk; ``discretization`` is "zoh" (exact) or "euler" (Delta * B).
+    ``n_segments`` splits the sequence across CTAs (0/1: one pass; k >= 2: up to k segments;
+    -1: the library decides from the device and the shape); the scratch it needs is allocated
+    here."""
     a, od = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
                       discretization, h0, conv_hist)
     Bt, Dn, L = x.shape
@@ -140,6 +144,14 @@ def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, 
             a.conv_hist_out = _ptr(ch)
             res["conv_hist"] = ch
     lib = _abi.load()
+    ws = None
+    if n_segments:
+        a.n_segments = int(n_segments)
+        need = lib.ssm_fwd_workspace_size(ctypes.byref(a))
+        if need:
+            ws = torch.empty(need + 256, dtype=torch.uint8, device=x.device)
+            a.workspace = (ws.data_ptr() + 255) & ~255
+            a.workspace_bytes = need
     _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(a), _stream_handle(x.device)))
     return res if (save_states or return_u or return_state) else out
 

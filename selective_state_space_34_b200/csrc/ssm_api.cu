@@ -118,7 +118,24 @@ ssm::FwdParams make_fwd_params(const ssm_fwd_args *a, int vec) {
   p.conv_hist = a->conv_w ? a->conv_hist : nullptr;
   p.h_last = a->h_last;
   p.conv_hist_out = a->conv_w ? a->conv_hist_out : nullptr;
+  p.n_seg = 1;  // one pass unless ssm_scan_fwd plans a split
+  p.seg_len = a->L;
   return p;
+}
+
+int sm_count_or_zero() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// The split-L plan of a forward call (one pass when n_segments asks for none or the device's
+// SM count cannot be read for an automatic choice).
+ssm::SegPlan fwd_plan(const ssm_fwd_args *a) {
+  const int sms = a->n_segments < 0 ? sm_count_or_zero() : 0;
+  if (a->n_segments < 0 && sms <= 0) return ssm::SegPlan{1, a->L, 0};
+  return ssm::plan_segments(a->Bt, a->Dn, a->N, a->L, a->n_segments, sms);
 }
 
 }  // namespace
@@ -150,10 +167,31 @@ ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream) {
   bool empty = false;
   ssm_status st = check_fwd(args, true, &empty);
   if (st != SSM_OK) return st;
+  if (args->n_segments < -1) return SSM_ERR_SHAPE;
   if (empty) return cuda_status(carry_through_empty(args, static_cast<cudaStream_t>(stream)));
-  const ssm::FwdParams p = make_fwd_params(args, vec_ok(args, nullptr, 0));
+  ssm::FwdParams p = make_fwd_params(args, vec_ok(args, nullptr, 0));
+  const ssm::SegPlan plan = fwd_plan(args);
+  if (plan.n_seg > 1) {
+    if (!args->workspace || args->workspace_bytes < plan.workspace_bytes ||
+        (reinterpret_cast<uintptr_t>(args->workspace) & 255))
+      return SSM_ERR_WORKSPACE;
+    auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t bdn = (size_t)plan.n_seg * args->Bt * args->Dn * args->N;
+    char *w = static_cast<char *>(args->workspace);
+    p.n_seg = plan.n_seg;
+    p.seg_len = plan.seg_len;
+    p.seg_hend = reinterpret_cast<float *>(w);
+    p.seg_h0 = reinterpret_cast<float *>(w + rnd(sizeof(float) * bdn));
+    p.seg_sdl = reinterpret_cast<float *>(w + 2 * rnd(sizeof(float) * bdn));
+  }
   return cuda_status(ssm::launch_fwd(p, args->in_dtype == SSM_BF16, args->out_dtype == SSM_BF16,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+size_t ssm_fwd_workspace_size(const ssm_fwd_args *args) {
+  bool empty = false;
+  if (check_fwd(args, false, &empty) != SSM_OK || empty || args->n_segments < -1) return 0;
+  return fwd_plan(args).workspace_bytes;
 }
 
 ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,

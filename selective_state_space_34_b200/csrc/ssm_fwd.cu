@@ -40,7 +40,9 @@ template <int G, int NS, typename Tin, int NT> struct FwdSmem {
   static constexpr size_t bytes = yp_off + sizeof(float) * CH * YC;
 };
 
-template <int G, int NS, typename Tin, typename Tout, int NT, bool EULER>
+// SUMMARY: pass 1 of the split-L forward -- the segment's recurrence from a zero state, keeping
+// only its end state and its sum of Delta (no readout, no outputs).
+template <int G, int NS, typename Tin, typename Tout, int NT, bool EULER, bool SUMMARY>
 __global__ void __launch_bounds__(NT, 512 / NT)
 ssm_fwd_kernel(const FwdParams p) {
   using S = FwdSmem<G, NS, Tin, NT>;
@@ -56,7 +58,9 @@ ssm_fwd_kernel(const FwdParams p) {
   float *yp = reinterpret_cast<float *>(smem + S::yp_off);
 
   const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
-  const int64_t b = blockIdx.x / n_dtiles;
+  const int64_t per_seg = n_dtiles * p.Bt;
+  const int64_t seg = blockIdx.x / per_seg;  // segment of the sequence (0 without split-L)
+  const int64_t b = (blockIdx.x % per_seg) / n_dtiles;
   const int64_t d0 = (blockIdx.x % n_dtiles) * CH;
   const int rows_valid = (int)imin64(CH, p.Dn - d0);
   const int tid = threadIdx.x, c = tid / G, g = tid % G;
@@ -65,14 +69,17 @@ ssm_fwd_kernel(const FwdParams p) {
   const bool has_conv = p.conv_w != nullptr, has_z = p.z != nullptr;
   const bool vec = p.vec != 0;
   const int64_t L = p.L, N = p.N;
+  // this CTA's steps: [ts, te). L stays the row length; steps from te on are padding here.
+  const int64_t ts = seg * p.seg_len, te = imin64(L, ts + p.seg_len);
 
   // per-lane constants: Acoef = A (precise) or A log2(e) (fast), nIA = -1/A; padded states are
   // inert (A_bar = 1, no input, no readout)
   float Acoef[NS], nIA[NS], h[NS];
+  const float *hinit = p.seg_h0 ? p.seg_h0 + (seg * p.Bt * p.Dn) * N : p.h0;  // carried state
 #pragma unroll
   for (int j = 0; j < NS; j++) {
     const int n = g * NS + j;
-    h[j] = (p.h0 && live && n < N) ? p.h0[(b * p.Dn + d) * N + n] : 0.0f;  // carried state or 0
+    h[j] = (!SUMMARY && hinit && live && n < N) ? hinit[(b * p.Dn + d) * N + n] : 0.0f;
     if (live && n < N) {
       const float A = -expf(p.A_log[d * N + n]);
       Acoef[j] = PRECISE ? A : A * kLog2e;
@@ -103,19 +110,24 @@ ssm_fwd_kernel(const FwdParams p) {
   const Tin *gC = static_cast<const Tin *>(p.C) + b * N * L;
   const int n_rows = (int)imin64(NP, N);
 
-  // conv-halo prefixes of both x buffers: the carried history (newest-first) in front of the
-  // first stage, zero where there is none
+  // conv-halo prefixes of both x buffers: the kPre inputs before the first step -- from x itself
+  // for a later segment, else the carried history (newest-first), zero where there is none
   const Tin *hist = (has_conv && p.conv_hist && p.K > 1) ? static_cast<const Tin *>(p.conv_hist) : nullptr;
   for (int i = tid; i < 2 * CH * kPre; i += NT) {
-    const int r = i / kPre, k = i % kPre, j = kPre - 1 - k;  // x_{-1-j}
+    const int r = i / kPre, k = i % kPre, j = kPre - 1 - k;  // x_{ts-1-j}
     Tin v = zero_val<Tin>();
-    if (hist && r < rows_valid && j < p.K - 1) v = hist[(b * p.Dn + d0 + r) * (p.K - 1) + j];
+    if (r < rows_valid) {
+      if (ts > 0)
+        v = gx[(int64_t)r * L + ts - 1 - j];
+      else if (hist && j < p.K - 1)
+        v = hist[(b * p.Dn + d0 + r) * (p.K - 1) + j];
+    }
     xs[r * S::XS + k] = v;
   }
 
-  const int64_t n_stages = (L + kT - 1) / kT;
+  const int64_t n_stages = (te - ts + kT - 1) / kT;
   auto issue = [&](int64_t stage, int buf) {
-    const int64_t t0 = stage * kT;
+    const int64_t t0 = ts + stage * kT;
     stage_rows<Tin, CH, kT, NT>(xs + buf * CH * S::XS + kPre, S::XS, gx, L, rows_valid, t0, L, vec);
     stage_rows<Tin, CH, kT, NT>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
     if (has_z) stage_rows<Tin, CH, kT, NT>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
@@ -123,21 +135,22 @@ ssm_fwd_kernel(const FwdParams p) {
   };
 
   BCStager<Tin, NP, NT> bc;
+  float sdl = 0.0f;  // sum of Delta over the segment (SUMMARY)
   if (n_stages > 0) {
     issue(0, 0);
-    bc.load(gB, gC, n_rows, 0, L, vec);
+    bc.load(gB, gC, n_rows, ts, L, vec);
     bc.store(Bs, Cs, S::BS);
-    if (n_stages > 1) bc.load(gB, gC, n_rows, kT, L, vec);
+    if (n_stages > 1) bc.load(gB, gC, n_rows, ts + kT, L, vec);
   }
   for (int64_t st = 0; st < n_stages; st++) {
     const int buf = (int)(st & 1), nbuf = buf ^ 1;
-    const int64_t t0 = st * kT;
+    const int64_t t0 = ts + st * kT;
     cp_async_wait<0>();
     __syncthreads();  // stage st landed and Bs/Cs[buf] written; stage st-1's buffers are free
     if (st + 1 < n_stages) {
       issue(st + 1, nbuf);
       bc.store(Bs + nbuf * kT * S::BS, Cs + nbuf * kT * S::BS, S::BS);
-      if (st + 2 < n_stages) bc.load(gB, gC, n_rows, (st + 2) * kT, L, vec);
+      if (st + 2 < n_stages) bc.load(gB, gC, n_rows, ts + (st + 2) * kT, L, vec);
     }
     const float *Bst = Bs + buf * kT * S::BS;
     const float *Cst = Cs + buf * kT * S::BS;
@@ -171,7 +184,7 @@ ssm_fwd_kernel(const FwdParams p) {
         float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
         float s = 1.0f;
         if (has_z) s = zw[j] * sigmoid<PRECISE>(zw[j]);
-        if (t0 + t >= L) {  // padded tail: an identity step
+        if (t0 + t >= te) {  // padded tail: an identity step
           u = 0.0f;
           dl = 0.0f;
         }
@@ -181,9 +194,9 @@ ssm_fwd_kernel(const FwdParams p) {
         if (t >= kT - 3)  // carry the conv halo into the next stage's prefix
           xs[(nbuf * CH + c) * S::XS + kPre + t - kT] = xrow[t];
       }
-      if (p.u_out && live)
+      if (!SUMMARY && p.u_out && live)
         store_run<Tout, EPL>(static_cast<Tout *>(p.u_out) + row0 + (int64_t)c * L,
-                             t0 + tb, L, uown, vec);
+                             t0 + tb, te, uown, vec);
       __syncwarp();
 
       // -- the recurrence over the block's kSub steps, in groups of 4 steps: all shared-memory
@@ -198,6 +211,7 @@ ssm_fwd_kernel(const FwdParams p) {
           const float2 du = ud[c * S::US + tq + tt];
           dlq[tt] = du.x;
           uq[tt] = du.y;
+          if (SUMMARY) sdl += du.x;
           load_states<NS>(Bq[tt], Bst + t * S::BS + g * NS);
           load_states<NS>(Cq[tt], Cst + t * S::BS + g * NS);
         }
@@ -274,35 +288,49 @@ ssm_fwd_kernel(const FwdParams p) {
             }
           }
         }
-        *reinterpret_cast<float4 *>(myp + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
+        if (!SUMMARY) *reinterpret_cast<float4 *>(myp + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
       }
       __syncwarp();
+      if constexpr (!SUMMARY) {  // pass 1 keeps only the state
 
-      // -- combine the G partial readouts of the owned steps, D skip, gate, store
-      float o[EPL];
+        // -- combine the G partial readouts of the owned steps, D skip, gate, store
+        float o[EPL];
 #pragma unroll
-      for (int j = 0; j < EPL; j++) o[j] = 0.0f;
+        for (int j = 0; j < EPL; j++) o[j] = 0.0f;
 #pragma unroll
-      for (int gg = 0; gg < G; gg++) {
-        float part[EPL];
-        load_floats<EPL>(part, yp + c * S::YC + gg * S::YG + g * EPL);
+        for (int gg = 0; gg < G; gg++) {
+          float part[EPL];
+          load_floats<EPL>(part, yp + c * S::YC + gg * S::YG + g * EPL);
 #pragma unroll
-        for (int j = 0; j < EPL; j++) o[j] += part[j];
-      }
+          for (int j = 0; j < EPL; j++) o[j] += part[j];
+        }
 #pragma unroll
-      for (int j = 0; j < EPL; j++) o[j] = fmaf(Dd, uown[j], o[j]) * gate[j];
-      if (live && p.out)
-        store_run<Tout, EPL>(static_cast<Tout *>(p.out) + row0 + (int64_t)c * L, t0 + tb, L, o, vec);
-      if (p.chunk_states && live && t0 + sb * kSub < L) {
-        const int64_t kk = (t0 + sb * kSub) / kSub;
-        float *dst = p.chunk_states + ((b * p.Dn + d) * p.n_ck + kk) * N;
+        for (int j = 0; j < EPL; j++) o[j] = fmaf(Dd, uown[j], o[j]) * gate[j];
+        if (live && p.out)
+          store_run<Tout, EPL>(static_cast<Tout *>(p.out) + row0 + (int64_t)c * L, t0 + tb, te, o, vec);
+        if (p.chunk_states && live && t0 + sb * kSub < te) {
+          const int64_t kk = (t0 + sb * kSub) / kSub;
+          float *dst = p.chunk_states + ((b * p.Dn + d) * p.n_ck + kk) * N;
 #pragma unroll
-        for (int j = 0; j < NS; j++)
-          if (g * NS + j < N) dst[g * NS + j] = h[j];
+          for (int j = 0; j < NS; j++)
+            if (g * NS + j < N) dst[g * NS + j] = h[j];
+        }
       }
       __syncwarp();  // ud / yp are rewritten by the next block
     }
   }
+  if (SUMMARY) {
+    // the segment's end state from a zero start, and its sum of Delta
+    if (live) {
+      const int64_t sbd = (seg * p.Bt + b) * p.Dn + d;
+#pragma unroll
+      for (int j = 0; j < NS; j++)
+        if (g * NS + j < N) p.seg_hend[sbd * N + g * NS + j] = h[j];
+      if (g == 0) p.seg_sdl[sbd] = sdl;
+    }
+    return;
+  }
+  if (te != L) return;  // only the last segment hands the state on
   // carried state after step L-1 (padded tail steps are identity steps)
   if (live && p.h_last) {
 #pragma unroll
@@ -367,24 +395,25 @@ int channels_per_cta(const LaneLayout &lay) { return kThreads / lay.G; }
 // 4x4096x16x4096 shape, 64 was no faster).
 constexpr int kFwdThreads = 128;
 
-template <int G, int NS, typename Tin, typename Tout>
-static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
+template <int G, int NS, typename Tin, typename Tout, bool SUMMARY>
+static cudaError_t launch_fwd_t(const FwdParams &p, int n_seg_launch, cudaStream_t stream) {
   constexpr int NT = kFwdThreads;
   using S = FwdSmem<G, NS, Tin, NT>;
-  auto kern = p.euler ? ssm_fwd_kernel<G, NS, Tin, Tout, NT, true> : ssm_fwd_kernel<G, NS, Tin, Tout, NT, false>;
+  auto kern = p.euler ? ssm_fwd_kernel<G, NS, Tin, Tout, NT, true, SUMMARY>
+                      : ssm_fwd_kernel<G, NS, Tin, Tout, NT, false, SUMMARY>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
   if (e != cudaSuccess) return e;
   const int64_t n_dtiles = (p.Dn + S::CH - 1) / S::CH;
-  const int64_t grid = n_dtiles * p.Bt;
+  const int64_t grid = n_dtiles * p.Bt * n_seg_launch;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, NT, S::bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <typename Tin, typename Tout>
-static cudaError_t dispatch_layout(const LaneLayout &lay, const FwdParams &p, cudaStream_t s) {
+template <typename Tin, typename Tout, bool SUMMARY>
+static cudaError_t dispatch_layout(const LaneLayout &lay, const FwdParams &p, int n_seg_launch, cudaStream_t s) {
 #define SSM_FWD_CASE(G_, NS_) \
-  if (lay.G == G_ && lay.NS == NS_) return launch_fwd_t<G_, NS_, Tin, Tout>(p, s);
+  if (lay.G == G_ && lay.NS == NS_) return launch_fwd_t<G_, NS_, Tin, Tout, SUMMARY>(p, n_seg_launch, s);
   SSM_FWD_CASE(4, 1) SSM_FWD_CASE(4, 2) SSM_FWD_CASE(4, 4)
   SSM_FWD_CASE(8, 1) SSM_FWD_CASE(8, 2) SSM_FWD_CASE(8, 4)
   SSM_FWD_CASE(16, 1) SSM_FWD_CASE(16, 2) SSM_FWD_CASE(16, 4)
@@ -392,14 +421,82 @@ static cudaError_t dispatch_layout(const LaneLayout &lay, const FwdParams &p, cu
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream) {
-  const LaneLayout lay = choose_layout(p.N, p.Bt * p.Dn);
+template <bool SUMMARY>
+static cudaError_t dispatch_types(const LaneLayout &lay, const FwdParams &p, int in_bf16, int out_bf16,
+                                  int n_seg_launch, cudaStream_t stream) {
   if (in_bf16) {
-    if (out_bf16) return dispatch_layout<__nv_bfloat16, __nv_bfloat16>(lay, p, stream);
-    return dispatch_layout<__nv_bfloat16, float>(lay, p, stream);
+    if (out_bf16 || SUMMARY) return dispatch_layout<__nv_bfloat16, __nv_bfloat16, SUMMARY>(lay, p, n_seg_launch, stream);
+    return dispatch_layout<__nv_bfloat16, float, SUMMARY>(lay, p, n_seg_launch, stream);
   }
-  if (out_bf16) return dispatch_layout<float, __nv_bfloat16>(lay, p, stream);
-  return dispatch_layout<float, float>(lay, p, stream);
+  if (out_bf16 && !SUMMARY) return dispatch_layout<float, __nv_bfloat16, SUMMARY>(lay, p, n_seg_launch, stream);
+  return dispatch_layout<float, float, SUMMARY>(lay, p, n_seg_launch, stream);
+}
+
+// Pass 2 of the split-L forward: the start state of every segment, walking the segments in order
+// -- h_in[s+1] = exp(A * sum of Delta over s) h_in[s] + (end state of s from a zero start). The
+// product of a segment's A_bar is exp(A * its sum of Delta), for the ZOH and the Euler rule alike.
+__global__ void seg_carry_kernel(const FwdParams p) {
+  const int64_t BDN = p.Bt * p.Dn * p.N;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (b, d, n)
+  if (i >= BDN) return;
+  const int64_t n = i % p.N, bd = i / p.N, d = bd % p.Dn;
+  const float A = -expf(p.A_log[d * p.N + n]);
+  float h = p.h0 ? p.h0[i] : 0.0f;
+  float *hin = const_cast<float *>(p.seg_h0);
+  for (int s = 0; s < p.n_seg; s++) {
+    hin[s * BDN + i] = h;
+    if (s + 1 < p.n_seg) h = fmaf(expf(A * p.seg_sdl[s * p.Bt * p.Dn + bd]), h, p.seg_hend[s * BDN + i]);
+  }
+}
+
+SegPlan plan_segments(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int requested, int sm_count) {
+  SegPlan plan = {1, L, 0};
+  constexpr int64_t kSegAlign = 64;  // a multiple of the stage and of the state chunk
+  int64_t want = requested;
+  if (requested < 0) {
+    // automatic: split only when even the widest lane layout leaves the SMs short of CTAs, then
+    // aim the 4-lane layout's CTAs x segments at one wave of 4 CTAs per SM, with segments of at
+    // least 1024 steps
+    const int64_t widest = Bt * ((Dn + 7) / 8);
+    if (widest >= 2 * (int64_t)sm_count) return plan;
+    const int64_t base = Bt * ((Dn + 31) / 32);
+    want = imin64(4 * (int64_t)sm_count / (base > 0 ? base : 1), L / 1024);
+  }
+  if (want < 2 || L < 2 * kSegAlign) return plan;
+  int64_t len = (L + want - 1) / want;
+  len = (len + kSegAlign - 1) / kSegAlign * kSegAlign;
+  const int64_t n = (L + len - 1) / len;
+  if (n < 2) return plan;
+  auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t bdn = (size_t)(n * Bt * Dn * N);
+  plan.n_seg = (int)n;
+  plan.seg_len = len;
+  plan.workspace_bytes = 2 * rnd(sizeof(float) * bdn) + rnd(sizeof(float) * (size_t)(n * Bt * Dn));
+  return plan;
+}
+
+cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream) {
+  if (p.n_seg <= 1) {
+    FwdParams q = p;
+    q.n_seg = 1;
+    q.seg_len = p.L;
+    q.seg_h0 = nullptr;
+    return dispatch_types<false>(choose_layout(p.N, p.Bt * p.Dn), q, in_bf16, out_bf16, 1, stream);
+  }
+  // split-L: the layout is chosen as if the segments were more channels
+  const LaneLayout lay = choose_layout(p.N, p.Bt * p.Dn * p.n_seg);
+  FwdParams s1 = p;  // pass 1: every segment but the last, from a zero state
+  s1.seg_h0 = nullptr;
+  s1.out = nullptr;
+  s1.u_out = nullptr;
+  s1.chunk_states = nullptr;
+  cudaError_t e = dispatch_types<true>(lay, s1, in_bf16, out_bf16, p.n_seg - 1, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t bdn = p.Bt * p.Dn * p.N;
+  seg_carry_kernel<<<(unsigned)((bdn + 255) / 256), 256, 0, stream>>>(p);  // pass 2
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return dispatch_types<false>(lay, p, in_bf16, out_bf16, p.n_seg, stream);  // pass 3
 }
 
 }  // namespace ssm

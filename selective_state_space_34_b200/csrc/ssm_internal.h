@@ -35,7 +35,22 @@ struct FwdParams {
   const void *conv_hist;  // (Bt, Dn, K-1) in-dtype or null
   float *h_last;          // (Bt, Dn, N) or null
   void *conv_hist_out;    // (Bt, Dn, K-1) in-dtype or null
+  // split-L: the sequence runs as n_seg segments of seg_len steps (n_seg = 1, seg_len = L: one pass)
+  int64_t seg_len;
+  int n_seg;
+  const float *seg_h0;    // (n_seg, Bt, Dn, N): start state of every segment (pass 3), or null
+  float *seg_hend;        // (n_seg, Bt, Dn, N): end state from a zero start (pass 1)
+  float *seg_sdl;         // (n_seg, Bt, Dn): sum of Delta over the segment (pass 1)
 };
+
+// Segmentation of a split-L forward: how many segments of which length, and the scratch it needs.
+struct SegPlan {
+  int n_seg;
+  int64_t seg_len;
+  size_t workspace_bytes;
+};
+// requested: 0/1 one pass, >= 2 up to that many segments, -1 chosen from sm_count and the shape.
+SegPlan plan_segments(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int requested, int sm_count);
 
 struct StepParams {
   const void *x, *dt, *B, *C, *z;

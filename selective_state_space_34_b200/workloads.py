@@ -45,7 +45,8 @@ class Workload:
         return self.Bt * self.Dn * self.L * self.N
 
 
-# The five measured workloads (seeds 1000 + index) and the finite-difference slice.
+# The five measured workloads (seeds 1000 + index), the finite-difference slice and the
+# few-channel long-context case.
 WORKLOADS: Dict[str, Workload] = {
     "tiny_fp32": Workload("tiny_fp32", 1, 16, 4, 64, in_dtype="f32", conv=False, gate=True,
                           dt_std=0.5, delta0=0.05, bc_std=1.0, seed=1000,
@@ -61,6 +62,11 @@ WORKLOADS: Dict[str, Workload] = {
                                  seed=1004, note="forward + backward, bf16 in, fp32 grads"),
     "fd_slice": Workload("fd_slice", 1, 8, 4, 32, in_dtype="f32", backward=True, seed=1005,
                          note="finite-difference slice, fp32"),
+    # the long-context workload's length and Delta distribution with few channels: the shape
+    # class split-L serves (a decode-like batch over a long prompt)
+    "long_fewch_fwd": Workload("long_fewch_fwd", 1, 512, 16, 65536, seed=1006,
+                               delta_loguniform=(1e-3, 1e-1),
+                               note="long-context forward, 512 channels (split-L case)"),
 }
 
 

@@ -46,10 +46,10 @@ def _header_fields(struct):
 
 
 @pytest.mark.parametrize("struct,cls,size", [
-    # 17 pointers, 4 int64, 5 int32 (+4 bytes of tail padding)
-    ("ssm_fwd_args", "FwdArgs", 17 * 8 + 4 * 8 + 5 * 4 + 4),
+    # 18 pointers, 4 int64, 6 int32, one size
+    ("ssm_fwd_args", "FwdArgs", 18 * 8 + 4 * 8 + 6 * 4 + 8),
     # the forward block, 17 pointers and one size
-    ("ssm_bwd_args", "BwdArgs", 192 + 17 * 8 + 8),
+    ("ssm_bwd_args", "BwdArgs", 208 + 17 * 8 + 8),
     # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
     ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
 ])
@@ -152,6 +152,22 @@ def test_state_carry_validation_codes(lib):
     assert _fwd(lib, _args(in_dtype=1, conv_w=0x7000, conv_hist_out=0x7001)) == 3
     # an empty chunk carries the state through without touching NULL pointers
     assert _fwd(lib, _args(L=0, x=None, out=None)) == 0
+
+
+def test_split_l_workspace_and_codes(lib):
+    size = lambda **kw: lib.ssm_fwd_workspace_size(ctypes.byref(_args(**kw)))
+    assert size() == 0 and size(n_segments=1) == 0           # one pass needs no scratch
+    assert size(n_segments=2, L=100) == 0                     # too short to split
+    # L = 1000 in up to 4 segments: 256-step segments -> 4 of them; 2 (4 Bt Dn N) + 4 Bt Dn floats
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert size(n_segments=4, L=1000) == 2 * rnd(4 * 2 * 8 * 4 * 4) + rnd(4 * 2 * 8 * 4)
+    assert size(n_segments=7, L=1000) == 2 * rnd(6 * 2 * 8 * 4 * 4) + rnd(6 * 2 * 8 * 4)  # 192-step segs
+    assert size(n_segments=-2) == 0
+    assert _fwd(lib, _args(n_segments=-2)) == 2
+    assert _fwd(lib, _args(n_segments=4, L=1000)) == 7                  # no workspace
+    assert _fwd(lib, _args(n_segments=4, L=1000, workspace=0x100000, workspace_bytes=16)) == 7
+    need = size(n_segments=4, L=1000)
+    assert _fwd(lib, _args(n_segments=4, L=1000, workspace=0x100010, workspace_bytes=need)) == 7
 
 
 def _step(**kw):
