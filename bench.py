@@ -303,7 +303,7 @@ def main():
                  "dconv_w": torch.empty(tuple(T["conv_w"].shape), **f32),
                  "dconv_b": torch.empty((Dn,), **f32)}
         need = ssm.ssm_bwd_workspace_size(T["dout"], T["x"], T["dt"], T["A_log"], T["B"], T["C"],
-                                          chunk_states=states, **kw)
+                                          chunk_states=states, n_segments=args.n_segments, **kw)
         ws = torch.empty(need + 256, dtype=torch.uint8, device=dev)
 
     import ctypes
@@ -333,6 +333,7 @@ def main():
             setattr(bw_args, k, v.data_ptr())
         bw_args.workspace = (ws.data_ptr() + 255) & ~255
         bw_args.workspace_bytes = need
+        bw_args.fwd.n_segments = args.n_segments
 
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     n_rec = args.steps
@@ -439,8 +440,10 @@ def main():
                 "peak_source": peaks.get("source")}
     else:
         roof = dict(fwd_roof)
-    # a split forward is three launches (segment summaries, carry, segments)
-    launches_per_step = (3 if ws_f is not None else 1) + (3 if backward else 0)
+    # a split forward is three launches (segment summaries, carry, segments); a split backward
+    # adds the adjoint summaries, their carry and the dx fix-up to its kernel and two reductions
+    split = ws_f is not None
+    launches_per_step = (3 if split else 1) + ((6 if split else 3) if backward else 0)
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, compute, D2H results ----
     names_in = ["x", "dt", "z", "B", "C"] + (["dout"] if backward else [])

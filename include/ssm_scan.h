@@ -122,8 +122,15 @@ typedef struct ssm_fwd_args {
    * from a zero state and keeps its end state and its sum of Delta, (2) the start state of every
    * segment follows from those in one pass over the segments (the product of a segment's A_bar
    * is exp(A * its sum of Delta)), (3) every segment runs from its start state, its conv prefix
-   * read from x. The results equal one pass up to fp32 rounding; the arithmetic is about 1.8x,
-   * for up to n_segments times the parallelism. ssm_scan_bwd ignores these three fields. */
+   * read from x. The results equal one pass up to fp32 rounding; the arithmetic is about 1.6x,
+   * for up to n_segments times the parallelism. ssm_scan_bwd splits the same way, from the end:
+   * (1) every segment but the first runs the adjoint backwards from a zero arrival (it needs
+   * only Delta, dy and C) and keeps A_bar_ts lambda_ts, (2) the gradient arriving at every
+   * segment's last state follows in one pass from the end, (3) every segment runs the full
+   * backward from its arrival; then each segment's conv-history gradient is added into the
+   * previous segment's last K-1 steps of dx. The backward reads n_segments from its fwd
+   * block; its scratch comes from the backward workspace (workspace / workspace_bytes below are
+   * the forward's only). */
   int32_t n_segments;    /* 0 or 1: one pass. >= 2: up to that many segments, each a multiple of
                             64 steps long. -1: chosen from the current device's SM count and the
                             shape (one pass unless even 8 channels per CTA leave fewer than two

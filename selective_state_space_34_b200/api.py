@@ -175,9 +175,11 @@ def _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_s
 
 
 def ssm_bwd_workspace_size(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None,
-                           conv_b=None, delta_softplus=True, chunk_states=None) -> int:
+                           conv_b=None, delta_softplus=True, chunk_states=None,
+                           n_segments: int = 0) -> int:
     bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
                      chunk_states)
+    bw.fwd.n_segments = int(n_segments)
     return int(_abi.load().ssm_bwd_workspace_size(ctypes.byref(bw)))
 
 
@@ -185,7 +187,7 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
                  conv_b=None, delta_softplus: bool = True, chunk_states=None,
                  workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None,
                  timing_events=None, discretization: str = "zoh", h0=None, conv_hist=None,
-                 dh_last=None, state_grads: bool = False):
+                 dh_last=None, state_grads: bool = False, n_segments: int = 0):
     """Backward. Returns a dict of fp32 gradients: dx, ddt, dA_log, dB, dC, and dD / ddt_bias /
     dz / dconv_w / dconv_b where the corresponding input exists. ``workspace`` (uint8, at least
     ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call.
@@ -218,6 +220,7 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
         _opt(k, v, torch.float32)
         setattr(bw, k, _ptr(v))
     lib = _abi.load()
+    bw.fwd.n_segments = int(n_segments)  # split-L (see ssm_scan_fwd)
     need = int(lib.ssm_bwd_workspace_size(ctypes.byref(bw)))
     if need > 0:
         if workspace is None or workspace.numel() * workspace.element_size() < need:

@@ -262,8 +262,9 @@ ssm_status ssm_scan_step(const ssm_step_args *a, void *stream) {
 size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {
   if (!args) return 0;
   const ssm_fwd_args *a = &args->fwd;
-  if (a->Bt <= 0 || a->L <= 0 || a->Dn <= 0 || a->N <= 0) return 0;
-  return ssm::bwd_workspace_bytes(a->Bt, a->Dn, a->N, a->L, args->chunk_states == nullptr);
+  if (a->Bt <= 0 || a->L <= 0 || a->Dn <= 0 || a->N <= 0 || a->n_segments < -1) return 0;
+  return ssm::bwd_workspace_bytes(a->Bt, a->Dn, a->N, a->L, args->chunk_states == nullptr,
+                                  fwd_plan(a).n_seg);
 }
 
 ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
@@ -272,6 +273,7 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   ssm_status st = check_fwd(&args->fwd, false, &empty);
   if (st != SSM_OK) return st;
   const ssm_fwd_args *a = &args->fwd;
+  if (a->n_segments < -1) return SSM_ERR_SHAPE;
   if (empty) {
     // nothing flows: parameter gradients are zero, the carried-state gradient passes through
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -331,6 +333,9 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   p.dh_last = args->dh_last;
   p.dh0 = args->dh0;
   p.dconv_hist = (a->conv_w && a->K > 1) ? args->dconv_hist : nullptr;
+  const ssm::SegPlan plan = fwd_plan(a);
+  p.n_seg = plan.n_seg;
+  p.seg_len = plan.seg_len;
   // carve the workspace (layout mirrored by ssm::bwd_workspace_bytes)
   char *ws = static_cast<char *>(args->workspace);
   auto take = [&](size_t bytes) {
@@ -338,19 +343,25 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
     ws += (bytes + 255) & ~size_t(255);
     return r;
   };
-  const ssm::LaneLayout lay = ssm::choose_layout(a->N, a->Bt * a->Dn);
+  const ssm::LaneLayout lay = ssm::choose_layout(a->N, a->Bt * a->Dn * p.n_seg);
   const int64_t ch = ssm::channels_per_cta(lay);
   p.n_dtiles = (a->Dn + ch - 1) / ch;
-  const int64_t BD = a->Bt * a->Dn;
-  p.p_dA_log = reinterpret_cast<float *>(take(sizeof(float) * BD * a->N));
-  p.p_dD = reinterpret_cast<float *>(take(sizeof(float) * BD));
-  p.p_ddt_bias = reinterpret_cast<float *>(take(sizeof(float) * BD));
-  p.p_dconv_w = reinterpret_cast<float *>(take(sizeof(float) * BD * 4));
-  p.p_dconv_b = reinterpret_cast<float *>(take(sizeof(float) * BD));
+  const int64_t BD = a->Bt * a->Dn, PD = BD * p.n_seg;
+  p.p_dA_log = reinterpret_cast<float *>(take(sizeof(float) * PD * a->N));
+  p.p_dD = reinterpret_cast<float *>(take(sizeof(float) * PD));
+  p.p_ddt_bias = reinterpret_cast<float *>(take(sizeof(float) * PD));
+  p.p_dconv_w = reinterpret_cast<float *>(take(sizeof(float) * PD * 4));
+  p.p_dconv_b = reinterpret_cast<float *>(take(sizeof(float) * PD));
   p.p_dB = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
   p.p_dC = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
   if (!args->chunk_states)
     p.f.chunk_states = reinterpret_cast<float *>(take(sizeof(float) * BD * p.f.n_ck * a->N));
+  if (p.n_seg > 1) {
+    p.seg_G = reinterpret_cast<float *>(take(sizeof(float) * PD * a->N));
+    p.seg_gloc = reinterpret_cast<float *>(take(sizeof(float) * PD * a->N));
+    p.seg_sdl = reinterpret_cast<float *>(take(sizeof(float) * PD));
+    p.seg_dxh = reinterpret_cast<float *>(take(sizeof(float) * PD * 4));
+  }
   return cuda_status(ssm::launch_bwd(p, a->in_dtype == SSM_BF16, static_cast<cudaStream_t>(stream)));
 }
 

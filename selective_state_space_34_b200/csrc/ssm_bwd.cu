@@ -83,7 +83,9 @@ template <int NS> __device__ __forceinline__ void store_states(float *dst, const
   }
 }
 
-template <int G, int NS, typename Tin, bool EULER>
+// SEG: split-L pass 3 (a grid of segments x batch x channel tiles); without it the segment is
+// the whole sequence and its bounds are compile-time constants of the one-pass kernel.
+template <int G, int NS, typename Tin, bool EULER, bool SEG>
 __global__ void __launch_bounds__(kThreads, 4)
 ssm_bwd_kernel(const BwdParams P) {
   using S = BwdSmem<G, NS, Tin>;
@@ -116,7 +118,8 @@ ssm_bwd_kernel(const BwdParams P) {
 
   const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
   const int64_t tile = blockIdx.x % n_dtiles;
-  const int64_t b = blockIdx.x / n_dtiles;
+  const int64_t b = SEG ? (blockIdx.x / n_dtiles) % p.Bt : blockIdx.x / n_dtiles;
+  const int64_t seg = SEG ? blockIdx.x / (n_dtiles * p.Bt) : 0;  // segment of the sequence
   const int64_t d0 = tile * CH;
   const int rows_valid = (int)imin64(CH, p.Dn - d0);
   const int tid = threadIdx.x, c = tid / G, g = tid % G;
@@ -125,6 +128,9 @@ ssm_bwd_kernel(const BwdParams P) {
   const bool has_conv = p.conv_w != nullptr, has_z = p.z != nullptr;
   const bool vec = p.vec != 0;
   const int64_t L = p.L, N = p.N;
+  // this CTA's steps: [ts, te). L stays the row length; steps from te on are padding here.
+  const int64_t ts = SEG ? seg * P.seg_len : 0, te = SEG ? imin64(L, ts + P.seg_len) : L;
+  const int64_t sbd = (seg * p.Bt + b) * p.Dn + d;  // row of the per-(segment, b, d) partials
 
   // A, the exp coefficient (A, or A log2 e on the fast path) and -1/A per owned state
   constexpr int NH = (NS + 1) / 2;  // state pairs per lane
@@ -138,7 +144,9 @@ ssm_bwd_kernel(const BwdParams P) {
 #pragma unroll
   for (int j = 0; j < 2 * NH; j++) {
     const int n = g * NS + j;
-    lam[j] = (P.dh_last && j < NS && live && n < N) ? P.dh_last[(b * p.Dn + d) * N + n] : 0.f;
+    // gradient arriving at the last state: from the next segment, or dh_last
+    const float *gin = (SEG && P.seg_G) ? P.seg_G + (seg * p.Bt * p.Dn) * N : P.dh_last;
+    lam[j] = (gin && j < NS && live && n < N) ? gin[(b * p.Dn + d) * N + n] : 0.f;
     aN[j] = 1.f;
     dAl[j] = 0.f;
     if (j < NS && live && n < N) {
@@ -178,9 +186,9 @@ ssm_bwd_kernel(const BwdParams P) {
   // dc of the (non-existent) steps after the sequence end are zero
   for (int i = tid; i < CH * S::DCS; i += kThreads) dcs[i] = 0.f;
 
-  const int64_t n_stages = (L + TS - 1) / TS;
+  const int64_t n_stages = (te - ts + TS - 1) / TS;
   auto issue = [&](int64_t stage, int buf) {
-    const int64_t t0 = stage * TS;
+    const int64_t t0 = ts + stage * TS;
     stage_rows<Tin, CH, kPre + TS>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
     stage_rows<Tin, CH, TS>(dts + buf * CH * TS, TS, gdt, L, rows_valid, t0, L, vec);
     if (has_z) stage_rows<Tin, CH, TS>(zs + buf * CH * TS, TS, gz, L, rows_valid, t0, L, vec);
@@ -192,19 +200,19 @@ ssm_bwd_kernel(const BwdParams P) {
   if (n_stages > 0) {
     const int lbuf = (int)((n_stages - 1) & 1);
     issue(n_stages - 1, lbuf);
-    bc.load(gB, gC, n_rows, (n_stages - 1) * TS, L, vec);
+    bc.load(gB, gC, n_rows, ts + (n_stages - 1) * TS, L, vec);
     bc.store(Bs + lbuf * TS * S::BS, Cs + lbuf * TS * S::BS, S::BS);
-    if (n_stages > 1) bc.load(gB, gC, n_rows, (n_stages - 2) * TS, L, vec);
+    if (n_stages > 1) bc.load(gB, gC, n_rows, ts + (n_stages - 2) * TS, L, vec);
   }
   for (int64_t st = n_stages - 1; st >= 0; st--) {
     const int buf = (int)(st & 1), pbuf = buf ^ 1;
-    const int64_t t0 = st * TS;
+    const int64_t t0 = ts + st * TS;
     cp_async_wait<0>();
     __syncthreads();  // stage st landed; B/C rows of stage st written; stage st+1's buffers free
     if (st > 0) {
       issue(st - 1, pbuf);
       bc.store(Bs + pbuf * TS * S::BS, Cs + pbuf * TS * S::BS, S::BS);
-      if (st > 1) bc.load(gB, gC, n_rows, (st - 2) * TS, L, vec);
+      if (st > 1) bc.load(gB, gC, n_rows, ts + (st - 2) * TS, L, vec);
     }
     const float *Bst = Bs + buf * TS * S::BS;
     const float *Cst = Cs + buf * TS * S::BS;
@@ -212,7 +220,7 @@ ssm_bwd_kernel(const BwdParams P) {
     const Tin *dtrow = dts + (buf * CH + c) * TS;
     const Tin *zrow = zs + (buf * CH + c) * TS;
     const Tin *dorow = dos + (buf * CH + c) * TS;
-    if (st == 0 && has_conv && p.conv_hist && p.K > 1) {
+    if (t0 == 0 && has_conv && p.conv_hist && p.K > 1) {
       // the carried inputs before step 0 (newest-first) replace the zero fill of the prefix
       if (live && g == 0) {
         const Tin *hr = static_cast<const Tin *>(p.conv_hist) + (b * p.Dn + d) * (p.K - 1);
@@ -257,7 +265,7 @@ ssm_bwd_kernel(const BwdParams P) {
           dy *= zw[j] * sz;
           gz = dow[j] * sz * fmaf(zw[j], 1.f - sz, 1.f);
         }
-        if (t0 + tb + j >= L) {  // padded steps are identity steps with no inputs
+        if (t0 + tb + j >= te) {  // padded steps are identity steps with no inputs
           u = 0.f;
           dl = 0.f;
           dy = 0.f;
@@ -281,8 +289,8 @@ ssm_bwd_kernel(const BwdParams P) {
         const int n = g * NS + j;
         h[j] = 0.f;
         if (j < NS && live && n < N) {
-          if (st > 0)
-            h[j] = states[((b * p.Dn + d) * p.n_ck + (st - 1)) * N + n];
+          if (t0 > 0)  // the saved state after the previous chunk of SSM_STATE_CHUNK = TS steps
+            h[j] = states[((b * p.Dn + d) * p.n_ck + (t0 / TS - 1)) * N + n];
           else if (p.h0)
             h[j] = p.h0[(b * p.Dn + d) * N + n];
         }
@@ -512,7 +520,7 @@ ssm_bwd_kernel(const BwdParams P) {
             acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
           }
           const int64_t t = t0 + tq + tt;
-          if (ok && part == 0 && t < L) {
+          if (ok && part == 0 && t < te) {
             float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
             const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
             const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
@@ -575,9 +583,9 @@ ssm_bwd_kernel(const BwdParams P) {
       }
       if (live) {
         const int64_t roff = (b * p.Dn + d) * L;
-        if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, L, dzv, vec);
-        if (P.ddt) store_run<float, EPL>(P.ddt + roff, t0 + tb, L, dtv, vec);
-        if (!has_conv && P.dx) store_run<float, EPL>(P.dx + roff, t0 + tb, L, dcv, vec);
+        if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, te, dzv, vec);
+        if (P.ddt) store_run<float, EPL>(P.ddt + roff, t0 + tb, te, dtv, vec);
+        if (!has_conv && P.dx) store_run<float, EPL>(P.dx + roff, t0 + tb, te, dcv, vec);
       }
     }
 
@@ -595,15 +603,19 @@ ssm_bwd_kernel(const BwdParams P) {
           for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
           dxv[j] = acc;
         }
-        if (live && P.dx) store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + tb, L, dxv, vec);
+        if (live && P.dx) store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + tb, te, dxv, vec);
       }
       __syncwarp();
-      if (st == 0 && live && g == 0 && P.dconv_hist && p.K > 1) {
-        // x_{-1-j} reaches c_t through tap k = t + 1 + j
+      if (st == 0 && live && g == 0 && p.K > 1 && (seg > 0 ? P.seg_dxh != nullptr : P.dconv_hist != nullptr)) {
+        // x_{ts-1-j} reaches c_t through tap k = t - ts + 1 + j: the carried history's gradient
+        // for the first segment, else a term of the previous segment's dx (added afterwards)
         for (int j = 0; j < p.K - 1; j++) {
           float acc = 0.f;
           for (int k = j + 1; k < p.K; k++) acc = fmaf(w4[k], dcs[c * S::DCS + k - j - 1], acc);
-          P.dconv_hist[(b * p.Dn + d) * (p.K - 1) + j] = acc;
+          if (SEG && seg > 0)
+            P.seg_dxh[sbd * 4 + j] = acc;
+          else
+            P.dconv_hist[(b * p.Dn + d) * (p.K - 1) + j] = acc;
         }
       }
       // this stage's first 3 dc values become the halo of the stage before it
@@ -620,8 +632,8 @@ ssm_bwd_kernel(const BwdParams P) {
     for (int j = 0; j < NS; j++) {
       const int n = g * NS + j;
       if (n < N) {
-        P.p_dA_log[(b * p.Dn + d) * N + n] = dAl[j];
-        if (P.dh0) P.dh0[(b * p.Dn + d) * N + n] = aN[j] * lam[j];
+        P.p_dA_log[sbd * N + n] = dAl[j];
+        if (P.dh0 && seg == 0) P.dh0[(b * p.Dn + d) * N + n] = aN[j] * lam[j];
       }
     }
   }
@@ -634,11 +646,10 @@ ssm_bwd_kernel(const BwdParams P) {
     for (int k = 0; k < 4; k++) accW[k] += __shfl_xor_sync(0xffffffffu, accW[k], off);
   }
   if (live && g == 0) {
-    const int64_t bd = b * p.Dn + d;
-    P.p_dD[bd] = accD;
-    P.p_ddt_bias[bd] = accDtb;
-    P.p_dconv_b[bd] = accCb;
-    for (int k = 0; k < 4; k++) P.p_dconv_w[bd * 4 + k] = accW[k];
+    P.p_dD[sbd] = accD;
+    P.p_ddt_bias[sbd] = accDtb;
+    P.p_dconv_b[sbd] = accCb;
+    for (int k = 0; k < 4; k++) P.p_dconv_w[sbd * 4 + k] = accW[k];
   }
   tmem_free_cta(tbase, S::NCOLS);
 }
@@ -657,10 +668,10 @@ __global__ void reduce_tiles_kernel(const float *__restrict__ pdB, const float *
   if (dC) dC[i] = sc;
 }
 
-// per-channel parameters: add the batch partials in batch order.
+// per-channel parameters: add the (segment, batch) partials in order.
 __global__ void reduce_params_kernel(const BwdParams P) {
   const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t Dn = P.f.Dn, N = P.f.N, Bt = P.f.Bt;
+  const int64_t Dn = P.f.Dn, N = P.f.N, Bt = P.f.Bt * P.n_seg;
   if (d >= Dn) return;
   float sD = 0.f, sT = 0.f, sCb = 0.f, sW[4] = {0.f, 0.f, 0.f, 0.f};
   for (int64_t b = 0; b < Bt; b++) {
@@ -682,28 +693,117 @@ __global__ void reduce_params_kernel(const BwdParams P) {
     }
 }
 
-size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states) {
+
+// Split-L pass 1: for every segment but the first, the adjoint run backwards from a zero arrival
+// -- lambda_t = dy_t C_t + A_bar_{t+1} lambda_{t+1} over [ts, te) -- needs only Delta, dy and C
+// (no state recompute). Keeps A_bar_ts lambda_ts (what the segment hands to the one before it
+// when nothing arrives) and the sum of Delta. One thread per (segment, b, d, group of 4 states).
+template <typename Tin>
+__global__ void seg_adjoint_kernel(const BwdParams P) {
+  constexpr bool PRECISE = sizeof(Tin) == 4;
+  const FwdParams &p = P.f;
+  const int64_t L = p.L, N = p.N, NQ = (N + 3) / 4, BD = p.Bt * p.Dn;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)(P.n_seg - 1) * BD * NQ) return;
+  const int64_t q = i % NQ, sb = i / NQ, bd = sb % BD, seg = 1 + sb / BD;
+  const int64_t b = bd / p.Dn, d = bd % p.Dn;
+  const int64_t ts = seg * P.seg_len, te = imin64(L, ts + P.seg_len);
+  float A[4], Ac[4], lam[4], an[4];
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const int64_t n = 4 * q + j;
+    A[j] = n < N ? -expf(p.A_log[d * N + n]) : 0.f;
+    Ac[j] = PRECISE ? A[j] : A[j] * kLog2e;
+    lam[j] = 0.f;
+    an[j] = 1.f;
+  }
+  const float dtb = p.dt_bias ? p.dt_bias[d] : 0.f;
+  const Tin *dtr = static_cast<const Tin *>(p.dt) + bd * L;
+  const Tin *zr = p.z ? static_cast<const Tin *>(p.z) + bd * L : nullptr;
+  const Tin *dor = static_cast<const Tin *>(P.dout) + bd * L;
+  const Tin *Cb = static_cast<const Tin *>(p.C) + b * N * L;
+  float sdl = 0.f;
+  for (int64_t t = te - 1; t >= ts; t--) {
+    const float v = to_f32(dtr[t]) + dtb;
+    const float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
+    float dy = to_f32(dor[t]);
+    if (zr) {
+      const float zz = to_f32(zr[t]);
+      dy *= zz * sigmoid<PRECISE>(zz);
+    }
+    sdl += dl;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int64_t n = 4 * q + j;
+      if (n < N) {
+        lam[j] = fmaf(an[j], lam[j], dy * to_f32(Cb[n * L + t]));
+        an[j] = PRECISE ? expf(dl * A[j]) : ex2_approx(dl * Ac[j]);
+      }
+    }
+  }
+  const int64_t row = (seg * BD + bd) * N;
+#pragma unroll
+  for (int j = 0; j < 4; j++)
+    if (4 * q + j < N) P.seg_gloc[row + 4 * q + j] = an[j] * lam[j];
+  if (q == 0) P.seg_sdl[seg * BD + bd] = sdl;
+}
+
+// Split-L pass 2: the gradient arriving at every segment's last state, from the end --
+// G_last = dh_last, G_{s-1} = A_bar_ts lambda_ts (zero arrival) + exp(A * sum of Delta over s) G_s.
+__global__ void seg_adjoint_carry_kernel(const BwdParams P) {
+  const FwdParams &p = P.f;
+  const int64_t BDN = p.Bt * p.Dn * p.N;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (b, d, n)
+  if (i >= BDN) return;
+  const int64_t n = i % p.N, bd = i / p.N, d = bd % p.Dn;
+  const float A = -expf(p.A_log[d * p.N + n]);
+  float G = P.dh_last ? P.dh_last[i] : 0.f;
+  for (int s = P.n_seg - 1; s >= 0; s--) {
+    P.seg_G[s * BDN + i] = G;
+    if (s > 0) G = fmaf(expf(A * P.seg_sdl[s * p.Bt * p.Dn + bd]), G, P.seg_gloc[s * BDN + i]);
+  }
+}
+
+// After pass 3: each later segment's gradient w.r.t. the K-1 inputs before it belongs to the
+// previous segment's last K-1 steps of dx.
+__global__ void seg_dx_fixup_kernel(const BwdParams P) {
+  const FwdParams &p = P.f;
+  const int64_t BD = p.Bt * p.Dn;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (segment >= 1, b, d)
+  if (i >= (int64_t)(P.n_seg - 1) * BD) return;
+  const int64_t bd = i % BD, seg = 1 + i / BD;
+  const int64_t ts = seg * P.seg_len;
+  for (int j = 0; j < p.K - 1; j++) P.dx[bd * p.L + ts - 1 - j] += P.seg_dxh[(seg * BD + bd) * 4 + j];
+}
+
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg) {
   auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const LaneLayout lay = choose_layout(N, Bt * Dn);
+  const LaneLayout lay = choose_layout(N, Bt * Dn * n_seg);
   const int64_t ch = channels_per_cta(lay);
   const int64_t n_tiles = (Dn + ch - 1) / ch;
-  const int64_t BD = Bt * Dn;
+  const int64_t BD = Bt * Dn, PD = BD * n_seg;  // parameter partials: one row per (segment, b, d)
   size_t s = 0;
-  s += rnd(sizeof(float) * BD * N);
-  s += rnd(sizeof(float) * BD);
-  s += rnd(sizeof(float) * BD);
-  s += rnd(sizeof(float) * BD * 4);
-  s += rnd(sizeof(float) * BD);
+  s += rnd(sizeof(float) * PD * N);
+  s += rnd(sizeof(float) * PD);
+  s += rnd(sizeof(float) * PD);
+  s += rnd(sizeof(float) * PD * 4);
+  s += rnd(sizeof(float) * PD);
   s += rnd(sizeof(float) * n_tiles * Bt * N * L);
   s += rnd(sizeof(float) * n_tiles * Bt * N * L);
   if (need_states) s += rnd(sizeof(float) * BD * ((L + kSub - 1) / kSub) * N);
+  if (n_seg > 1) {
+    s += 2 * rnd(sizeof(float) * PD * N);  // seg_G, seg_gloc
+    s += rnd(sizeof(float) * PD);          // seg_sdl
+    s += rnd(sizeof(float) * PD * 4);      // seg_dxh
+  }
   return s;
 }
 
 template <int G, int NS, typename Tin>
 static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   using S = BwdSmem<G, NS, Tin>;
-  auto kern = P.f.euler ? ssm_bwd_kernel<G, NS, Tin, true> : ssm_bwd_kernel<G, NS, Tin, false>;
+  auto kern = P.n_seg > 1 ? (P.f.euler ? ssm_bwd_kernel<G, NS, Tin, true, true> : ssm_bwd_kernel<G, NS, Tin, false, true>)
+                           : (P.f.euler ? ssm_bwd_kernel<G, NS, Tin, true, false> : ssm_bwd_kernel<G, NS, Tin, false, false>);
   // Each resident CTA holds S::NCOLS of the SM's 512 TMEM columns. Ask for enough shared memory
   // that no more CTAs fit on an SM than the columns allow, so no allocation ever has to wait.
   int dev = 0, smem_sm = 0, reserved = 0;
@@ -719,7 +819,7 @@ static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = P.n_dtiles * P.f.Bt;
+  const int64_t grid = P.n_dtiles * P.f.Bt * P.n_seg;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, kThreads, smem, stream>>>(P);
   return cudaGetLastError();
@@ -746,7 +846,21 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
     e = launch_fwd(f, in_bf16, 0, stream);
     if (e != cudaSuccess) return e;
   }
-  const LaneLayout lay = choose_layout(P.f.N, P.f.Bt * P.f.Dn);
+  const LaneLayout lay = choose_layout(P.f.N, P.f.Bt * P.f.Dn * P.n_seg);
+  if (P.n_seg > 1) {
+    // split-L passes 1 and 2: what arrives at each segment's last state
+    const int64_t n1 = (int64_t)(P.n_seg - 1) * P.f.Bt * P.f.Dn * ((P.f.N + 3) / 4);
+    if (in_bf16)
+      seg_adjoint_kernel<__nv_bfloat16><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
+    else
+      seg_adjoint_kernel<float><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t bdn = P.f.Bt * P.f.Dn * P.f.N;
+    seg_adjoint_carry_kernel<<<(unsigned)((bdn + 255) / 256), 256, 0, stream>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (P.timing_events && P.timing_events[0]) {
     e = cudaEventRecord(static_cast<cudaEvent_t>(P.timing_events[0]), stream);
     if (e != cudaSuccess) return e;
@@ -755,6 +869,12 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (P.timing_events && P.timing_events[1]) {
     e = cudaEventRecord(static_cast<cudaEvent_t>(P.timing_events[1]), stream);
+    if (e != cudaSuccess) return e;
+  }
+  if (P.n_seg > 1 && P.dx && P.f.conv_w && P.f.K > 1) {
+    const int64_t n = (int64_t)(P.n_seg - 1) * P.f.Bt * P.f.Dn;
+    seg_dx_fixup_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(P);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   const int64_t per_tile = P.f.Bt * P.f.N * P.f.L;

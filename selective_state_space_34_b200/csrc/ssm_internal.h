@@ -80,6 +80,15 @@ struct BwdParams {
   const float *dh_last;        // (Bt, Dn, N) or null
   float *dh0;                  // (Bt, Dn, N) or null
   float *dconv_hist;           // (Bt, Dn, K-1) or null
+  // split-L (f stays a one-pass forward for the state recompute): n_seg segments of seg_len steps;
+  // the per-(b, d) parameter partials above then hold n_seg * Bt rows
+  int n_seg;
+  int64_t seg_len;
+  float *seg_G;                // (n_seg, Bt, Dn, N): gradient arriving at each segment's last state
+  float *seg_gloc;             // (n_seg, Bt, Dn, N): A_bar_ts lambda_ts from a zero arrival (pass 1)
+  float *seg_sdl;              // (n_seg, Bt, Dn): sum of Delta over each segment (pass 1)
+  float *seg_dxh;              // (n_seg, Bt, Dn, 4): each segment's gradient w.r.t. the K-1 inputs
+                               // before it, added into the previous segment's dx afterwards
 };
 
 LaneLayout choose_layout(int64_t N, int64_t channels);
@@ -87,7 +96,7 @@ int channels_per_cta(const LaneLayout &lay);
 
 cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
-size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states);
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg);
 cudaError_t launch_step(const StepParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
                                int64_t Dn, int64_t L, int K, int in_bf16, int out_bf16, int vec,

@@ -67,6 +67,9 @@ WORKLOADS: Dict[str, Workload] = {
     "long_fewch_fwd": Workload("long_fewch_fwd", 1, 512, 16, 65536, seed=1006,
                                delta_loguniform=(1e-3, 1e-1),
                                note="long-context forward, 512 channels (split-L case)"),
+    "long_fewch_fwdbwd": Workload("long_fewch_fwdbwd", 1, 512, 16, 65536, seed=1007,
+                                  delta_loguniform=(1e-3, 1e-1), backward=True,
+                                  note="long-context forward + backward, 512 channels (split-L)"),
 }
 
 

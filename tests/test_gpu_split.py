@@ -113,3 +113,58 @@ def test_long_few_channels_sampled():
                                              "conv_w", "conv_b")}
         ref = oracle.fwd(s["x"], s["dt"], s["A_log"], s["B"], s["C"], **oracle_kw(s))
         assert_close("out[%d,%d]" % (b, d), got[b:b + 1, d:d + 1], ref, *TOL[("bf16", "f32")])
+
+
+GRADS = ["dx", "ddt", "dz", "dA_log", "dB", "dC", "dD", "ddt_bias", "dconv_w", "dconv_b",
+         "dh0", "dconv_hist"]
+
+
+def _bwd_case(Bt, Dn, N, L, dtype, nseg, conv=True, gate=True, carried=True, euler=False,
+              saved=True):
+    w = wl.shaped("mamba130m_fwd", Bt=Bt, Dn=Dn, N=N, L=L, in_dtype=dtype, conv=conv, gate=gate,
+                  backward=True)
+    a = wl.generate(w)
+    a.update(wl.carried_state(w))
+    if not carried:
+        a["h0"] = a["conv_hist"] = a["dh_last"] = None
+    t = dev_arrays(a, dtype)
+    kw = param_kw(t, conv=conv, gate=gate)
+    disc = "euler" if euler else "zoh"
+    st = dict(h0=t["h0"], conv_hist=t["conv_hist"] if conv else None, discretization=disc)
+    states = None
+    if saved:
+        states = ssm.ssm_scan_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], save_states=True,
+                                  n_segments=nseg, **st, **kw)["chunk_states"]
+    g = ssm.ssm_scan_bwd(t["dout"], t["x"], t["dt"], t["A_log"], t["B"], t["C"],
+                         chunk_states=states, dh_last=t["dh_last"], state_grads=True,
+                         n_segments=nseg, **st, **kw)
+    g1 = ssm.ssm_scan_bwd(t["dout"], t["x"], t["dt"], t["A_log"], t["B"], t["C"],
+                          chunk_states=states, dh_last=t["dh_last"], state_grads=True, **st, **kw)
+    torch.cuda.synchronize()
+    ok = oracle_kw(a, conv=conv, gate=gate)
+    ref = oracle.bwd(a["x"], a["dt"], a["A_log"], a["B"], a["C"], a["dout"], euler=euler,
+                     h0=a["h0"], conv_hist=a["conv_hist"] if conv else None,
+                     dh_last=a["dh_last"], **ok)
+    from gpu_helpers import assert_grad_close
+    for k in GRADS:
+        if k in ref and k in g:
+            assert_grad_close(k, to_np(g[k]), ref[k])
+            assert_grad_close(k + " vs one pass", to_np(g[k]), to_np(g1[k]))
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 7])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_split_backward(nseg, dtype):
+    _bwd_case(2, 24, 16, 1000, dtype, nseg)
+
+
+@pytest.mark.parametrize("case", ["no_conv", "no_gate", "plain", "euler", "recompute", "N5", "N64"])
+def test_split_backward_variants(case):
+    kw = dict(conv=case != "no_conv", gate=case != "no_gate", carried=case != "plain",
+              euler=case == "euler", saved=case != "recompute")
+    N = {"N5": 5, "N64": 64}.get(case, 16)
+    _bwd_case(1, 16, N, 777, "bf16", 4, **kw)
+
+
+def test_split_backward_long_few_channels():
+    _bwd_case(1, 32, 16, 8192, "bf16", 16, carried=False)
