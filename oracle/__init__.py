@@ -54,6 +54,9 @@ def bind(lib):
     lib.ssm_oracle_fwd.argtypes = common + [_dp] * 5 + [ctypes.c_int]
     lib.ssm_oracle_bwd.restype = ctypes.c_int
     lib.ssm_oracle_bwd.argtypes = common + [_dp] * 2 + [_dp] * 12 + [ctypes.c_int]
+    lib.ssm_oracle_ssd_fwd.restype = ctypes.c_int
+    lib.ssm_oracle_ssd_fwd.argtypes = ([_dp] * 7 + [_i64] * 5 + [ctypes.c_int, ctypes.c_int] +
+                                       [_dp] * 3 + [ctypes.c_int])
     return lib
 
 
@@ -181,3 +184,22 @@ def bwd(x, dt, A_log, B, C, dout, D=None, z=None, dt_bias=None, conv_w=None, con
     if rc != 0:
         raise MemoryError("ssm_oracle_bwd: allocation failed")
     return g
+
+
+def ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, delta_softplus=True, euler=False, h0=None,
+            want_state=False, n_threads=0):
+    """Mamba-2 state-space-duality recurrence ("state-space models", "Mamba-2 and state-space
+    duality"). x: (Bt, H, L, P); dt: (Bt, H, L); B, C: (Bt, L, N); A_log, D, dt_bias: (H,);
+    h0: (Bt, H, N, P). Returns y (Bt, H, L, P), or (y, h_last) with want_state."""
+    x, dt, A_log, B, C = _in(x), _in(dt), _in(A_log), _in(B), _in(C)
+    D, dt_bias, h0 = _in(D), _in(dt_bias), _in(h0)
+    Bt, H, L, P = x.shape
+    N = B.shape[2]
+    y = np.empty_like(x)
+    hl = np.empty((Bt, H, N, P)) if want_state else None
+    rc = _load().ssm_oracle_ssd_fwd(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log), _ptr(B), _ptr(C),
+                                    _ptr(D), Bt, H, L, P, N, int(bool(delta_softplus)),
+                                    int(bool(euler)), _ptr(h0), _ptr(y), _ptr(hl), int(n_threads))
+    if rc != 0:
+        raise MemoryError("ssm_oracle_ssd_fwd: allocation failed")
+    return (y, hl) if want_state else y

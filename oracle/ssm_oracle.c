@@ -45,6 +45,9 @@
  *    objects after this chunk; an empty chunk (L = 0) returns them unchanged.
  *  - euler = 1 selects Mamba's first-order input discretisation B-bar = Delta * B
  *    ([SSMK] mamba_selective_scan_step; [TL] step); A-bar stays exp(Delta * A).
+ *
+ * Also here: the Mamba-2 state-space-duality recurrence ([SSM] "Mamba-2 and state-space
+ * duality"), ssm_oracle_ssd_fwd at the end of the file, with its own readings listed there.
  */
 #include <math.h>
 #include <stdint.h>
@@ -422,5 +425,69 @@ int ssm_oracle_bwd(const double *x, const double *dt, const double *dt_bias, con
 done:
   free(pA); free(pD); free(pdtb); free(pcw); free(pcb);
   (void)n_threads;
+  return failed ? -1 : 0;
+}
+
+
+/* ---- Mamba-2 state-space duality (SSD) ----------------------------------------------------
+ *
+ * [SSM] "Mamba-2 and state-space duality": within a head the transition is a scalar multiple of
+ * the identity, A-bar_t = a_t I, and unrolling gives y_t = sum_{s<=t} (C_t . B-bar_s)
+ * (prod_{k=s+1..t} a_k) x_s, i.e. Y = (L o Q K^T) V with L_ts = prod_{k=s+1..t} a_k (s <= t).
+ * This oracle runs the recurrence that unrolls to that sum, one head at a time:
+ *   h_t = a_t h_{t-1} + B-bar_t x_t^T     (h is N x P: state index n, head-channel index p)
+ *   y_t = h_t^T C_t + D_h x_t
+ * Readings taken where the page leaves a step open:
+ *  - a_t and B-bar_t come from the same discretisation as the selective scan, with one A per
+ *    head: Delta_t = softplus(dt_t + dt_bias[h]) (or dt_t + dt_bias[h] when delta_softplus == 0),
+ *    A_h = -exp(A_log[h]), a_t = exp(Delta_t A_h), B-bar_t = beta_t B_t with beta_t =
+ *    expm1(Delta_t A_h) / A_h (exact zero-order hold) or Delta_t (euler = 1).
+ *  - B_t and C_t (N values) are shared by all heads of a batch element, as the selective scan
+ *    shares them across channels; x_t of a head has P values; D_h is one skip weight per head.
+ *  - h0 (NULL = 0) is the state before step 0; h_last receives the state after step L-1.
+ * Layouts: x, y (Bt, H, L, P); dt (Bt, H, L); B, C (Bt, L, N); A_log, dt_bias, D [H];
+ * h0, h_last (Bt, H, N, P). Returns 0, or -1 if the state buffer cannot be allocated.
+ */
+int ssm_oracle_ssd_fwd(const double *x, const double *dt, const double *dt_bias,
+                       const double *A_log, const double *B, const double *C, const double *D,
+                       int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N, int delta_softplus,
+                       int euler, const double *h0, double *y, double *h_last, int n_threads) {
+  int failed = 0;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+#endif
+  for (int64_t bh = 0; bh < Bt * H; bh++) {
+    const int64_t b = bh / H, hd = bh % H;
+    double *st = (double *)malloc(sizeof(double) * (size_t)(N * P));
+    if (!st) {
+      failed |= 1;
+      continue;
+    }
+    for (int64_t i = 0; i < N * P; i++) st[i] = h0 ? h0[bh * N * P + i] : 0.0;
+    const double A = -exp(A_log[hd]);
+    const double bias = dt_bias ? dt_bias[hd] : 0.0;
+    const double Dh = D ? D[hd] : 0.0;
+    for (int64_t t = 0; t < L; t++) {
+      const double v = dt[bh * L + t] + bias;
+      const double delta = delta_softplus ? ssm_oracle_softplus(v) : v;
+      const double a = exp(delta * A);
+      const double beta = euler ? delta : expm1(delta * A) / A;
+      const double *xt = x + (bh * L + t) * P;
+      const double *Bt_ = B + (b * L + t) * N;
+      const double *Ct = C + (b * L + t) * N;
+      for (int64_t n = 0; n < N; n++)
+        for (int64_t p = 0; p < P; p++) st[n * P + p] = a * st[n * P + p] + beta * Bt_[n] * xt[p];
+      double *yt = y + (bh * L + t) * P;
+      for (int64_t p = 0; p < P; p++) {
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; n++) acc += Ct[n] * st[n * P + p];
+        yt[p] = acc + Dh * xt[p];
+      }
+    }
+    if (h_last)
+      for (int64_t i = 0; i < N * P; i++) h_last[bh * N * P + i] = st[i];
+    free(st);
+  }
   return failed ? -1 : 0;
 }

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_ssd as ssd_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
 
@@ -38,11 +39,24 @@ MUTATIONS = [
     ("dh0_missing_decay", "? a[(size_t)n] * lam[n] : lam[n];", "? lam[n] : lam[n];"),
     ("dh_last_decayed", "a[i + (size_t)N] : 1.0;", "a[i + (size_t)N] : 0.0;"),
     ("bwd_euler_dB", "dBb[n * L + t] += lam[n] * u[t] * dl[t];", "dBb[n * L + t] += lam[n] * u[t];"),
+    # the state-space-duality recurrence
+    ("ssd_dropped_decay", "st[n * P + p] = a * st[n * P + p] + beta * Bt_[n] * xt[p];",
+     "st[n * P + p] = st[n * P + p] + beta * Bt_[n] * xt[p];"),
+    ("ssd_euler_ignored", "const double beta = euler ? delta : expm1(delta * A) / A;",
+     "const double beta = expm1(delta * A) / A;"),
+    ("ssd_zoh_as_euler", "const double beta = euler ? delta : expm1(delta * A) / A;",
+     "const double beta = delta;"),
+    ("ssd_readout_with_B", "acc += Ct[n] * st[n * P + p];", "acc += Bt_[n] * st[n * P + p];"),
+    ("ssd_dropped_skip", "yt[p] = acc + Dh * xt[p];", "yt[p] = acc;"),
+    ("ssd_bias_ignored", "const double bias = dt_bias ? dt_bias[hd] : 0.0;", "const double bias = 0.0;"),
+    ("ssd_A_sign", "const double A = -exp(A_log[hd]);", "const double A = -exp(-A_log[hd]);"),
+    ("ssd_h0_ignored", "st[i] = h0 ? h0[bh * N * P + i] : 0.0;", "st[i] = 0.0;"),
 ]
 
 
 def _pin_functions():
-    return [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+    return ([getattr(pins, n) for n in dir(pins) if n.startswith("test_")] +
+            [getattr(ssd_pins, n) for n in dir(ssd_pins) if n.startswith("test_")])
 
 
 def _param_sets(fn):
