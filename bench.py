@@ -240,6 +240,61 @@ def reference_arm(args, w):
     return 0
 
 
+# ---- the state-space-duality leg (Mamba-2 heads, tensor cores) ---------------------------------
+
+def ssd_bench(args, cfg, name):
+    import torch
+    import selective_state_space_34_b200 as ssm
+    from selective_state_space_34_b200 import workloads as wl
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Bt, H, L, P, N = cfg["Bt"], cfg["H"], cfg["L"], cfg["P"], cfg["N"]
+    a = wl.generate_ssd(Bt, H, L, P, N, seed=cfg["seed"] + rank)
+    T = {k: torch.from_numpy(v).to(dev, torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    run = lambda: ssm.ssm_ssd_fwd(T["x"], T["dt"], T["A_log"], T["B"], T["C"], D=T["D"],
+                                  dt_bias=T["dt_bias"])
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(args.steps):
+        run()
+    s1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(s0.elapsed_time(s1), world, dev) / args.steps
+    es = Bt * H * P * L * N
+    nC = (L + 127) // 128
+    # algorithmic bytes: x, dt, B, C in, y out (bf16); the chunk states are intermediates
+    ab = Bt * H * L * P * 2 * 2 + Bt * H * L * 2 + 2 * Bt * L * N * 2
+    # tensor-core work as issued: C B^T (Q x Q x N), C H (Q x N x P), G' X (Q x Q x P), state (N x Q x P)
+    flops = 2 * Bt * H * nC * (128 * 128 * 128 + 128 * 128 * P + 128 * 128 * P + 128 * 128 * P)
+    peaks = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = {
+        "metric": METRIC, "value": job_throughput(es, world, 1, ms), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": name, "Bt": Bt, "H": H, "P": P, "N": N, "L": L, "chunk": 128,
+                   "step": "ssd forward (3 launches)", "l2": "inputs larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": ab / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": ab / (ms * 1e-3) / 1e9 / hbm, "traffic": None, "algorithmic_bytes": ab},
+        "tensor": {"achieved": flops / (ms * 1e-3) / 1e12, "peak": bf16, "unit": "TFLOP/s",
+                   "frac": flops / (ms * 1e-3) / 1e12 / bf16},
+        "gpu_launches": 3 * args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---- our arm ----------------------------------------------------------------------------------
 
 def main():
@@ -258,6 +313,12 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     from selective_state_space_34_b200 import workloads as wl
+    if args.workload in wl.SSD_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the state-space-duality leg has no "
+                              "CPU reference arm; its parity is in tests/test_gpu_ssd.py"}))
+            return 0
+        return ssd_bench(args, wl.SSD_WORKLOADS[args.workload], args.workload)
     w = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
         return reference_arm(args, w)

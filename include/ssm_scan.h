@@ -149,6 +149,53 @@ typedef struct ssm_fwd_args {
  */
 ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream);
 
+/*
+ * Mamba-2 state-space duality (SSD) forward ("state-space models", "Mamba-2 and state-space
+ * duality"). Within a head h the transition is a scalar multiple of the identity, A_bar_t = a_t I:
+ *
+ *   Delta_t = softplus(dt_t + dt_bias[h])   (or dt_t + dt_bias[h] when delta_softplus = 0, which
+ *             must then be >= 0: a step size; a negative one makes a_t > 1 and the chunk-local
+ *             decay factors e^{cum_t - cum_s} can overflow fp32)
+ *   a_t     = exp(Delta_t A_h),  A_h = -exp(A_log[h])
+ *   B_bar_t = beta_t B_t,  beta_t = (a_t - 1) / A_h (exact ZOH) or Delta_t (SSM_EULER)
+ *   h_t     = a_t h_{t-1} + B_bar_t x_t^T       (N x P per head; h_{-1} = h0 or 0)
+ *   y_t     = h_t^T C_t + D[h] x_t
+ *
+ * i.e. y_t = sum_{s<=t} (C_t . B_bar_s) (prod_{k=s+1..t} a_k) x_s + D x_t = (L o C B_bar^T) X.
+ * Computed in chunks of 128 steps: matrix products within a chunk on the tensor cores (bf16
+ * operands, fp32 accumulation), the N x P state carried between chunks in fp32. B and C are
+ * shared by all heads of a batch element (one group). Supported: bf16 inputs, P (head dim) 64 or
+ * 128, N (state) 64 or 128 (SSM_ERR_UNSUPPORTED otherwise).
+ */
+typedef struct ssm_ssd_args {
+  const void *x;         /* device (Bt, H, L, P) bf16, 16-byte aligned */
+  const void *dt;        /* device (Bt, H, L) bf16 */
+  const float *dt_bias;  /* device [H] or NULL (= 0) */
+  const float *A_log;    /* device [H] */
+  const void *B;         /* device (Bt, L, N) bf16, 16-byte aligned */
+  const void *C;         /* device (Bt, L, N) bf16, 16-byte aligned */
+  const float *D;        /* device [H] or NULL (= 0) */
+  const float *h0;       /* device (Bt, H, N, P) fp32 or NULL (= 0) */
+  void *y;               /* device (Bt, H, L, P) out_dtype, 16-byte aligned */
+  float *h_last;         /* device (Bt, H, N, P) fp32 or NULL: the state after step L-1 */
+  int64_t Bt, H, L, P, N;
+  int32_t in_dtype;      /* must be SSM_BF16 */
+  int32_t out_dtype;     /* SSM_BF16 or SSM_F32 */
+  int32_t delta_softplus;
+  int32_t discretization;/* ssm_discretization */
+  void *workspace;       /* device scratch of ssm_ssd_workspace_size() bytes, 256-byte aligned */
+  size_t workspace_bytes;
+} ssm_ssd_args;
+
+/* Scratch bytes ssm_ssd_fwd needs: the chunk states (fp32), the state entering every chunk
+ * (bf16), one log-decay per chunk, and an error word; 0 for an empty or invalid problem. */
+size_t ssm_ssd_workspace_size(const ssm_ssd_args *args);
+
+/* Errors: SSM_ERR_NULL, SSM_ERR_SHAPE (negative sizes, H/P/N = 0), SSM_ERR_ALIGN,
+ * SSM_ERR_DTYPE (codes), SSM_ERR_UNSUPPORTED (in_dtype not bf16, P not 64/128, N not 64/128),
+ * SSM_ERR_WORKSPACE, SSM_ERR_CUDA. Bt = 0 or L = 0: nothing to do (h_last = h0 or 0). */
+ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream);
+
 /* Bytes of workspace ssm_scan_fwd needs for these arguments: 0 when the call runs in one pass
  * (n_segments 0 or 1, or a split that would leave a single segment), else 2 (n Bt Dn N) + n Bt Dn
  * floats for n segments (each array rounded up to 256 bytes). With n_segments = -1 the answer

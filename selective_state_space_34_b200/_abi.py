@@ -62,6 +62,20 @@ class StepArgs(ctypes.Structure):
 
 
 # (name, restype, argtypes) of every exported function in include/ssm_scan.h
+class SsdArgs(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+        ("A_log", ctypes.c_void_p), ("B", ctypes.c_void_p), ("C", ctypes.c_void_p),
+        ("D", ctypes.c_void_p), ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p),
+        ("h_last", ctypes.c_void_p),
+        ("Bt", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64), ("P", ctypes.c_int64),
+        ("N", ctypes.c_int64),
+        ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+        ("delta_softplus", ctypes.c_int32), ("discretization", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 SIGNATURES = [
     ("ssm_num_state_chunks", ctypes.c_int64, [ctypes.c_int64]),
     ("ssm_scan_fwd", ctypes.c_int, [ctypes.POINTER(FwdArgs), ctypes.c_void_p]),
@@ -70,6 +84,8 @@ SIGNATURES = [
     ("ssm_scan_bwd", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_bwd_noalloc", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_step", ctypes.c_int, [ctypes.POINTER(StepArgs), ctypes.c_void_p]),
+    ("ssm_ssd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(SsdArgs)]),
+    ("ssm_ssd_fwd", ctypes.c_int, [ctypes.POINTER(SsdArgs), ctypes.c_void_p]),
     ("ssm_conv1d_silu", ctypes.c_int,
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
       ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,

@@ -296,3 +296,44 @@ def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = 
         _ptr(x), _ptr(out), _ptr(w), _ptr(b), Bt, Dn, L, int(w.shape[1]), _DT[x.dtype], _DT[od],
         _stream_handle(x.device)))
     return out
+
+
+def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplus: bool = True,
+                out_dtype=None, discretization: str = "zoh", return_state: bool = False):
+    """Mamba-2 state-space duality forward. x: (Bt, H, L, P) bf16; dt: (Bt, H, L) bf16; B, C:
+    (Bt, L, N) bf16 shared by the heads; A_log, D, dt_bias: (H,) fp32; h0: (Bt, H, N, P) fp32.
+    P and N must be 64 or 128. Returns y (Bt, H, L, P), or (y, h_last) with return_state."""
+    for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
+        _need_cuda(n, t)
+    for n, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("%s must be bfloat16" % n)
+    for n, t in (("A_log", A_log), ("D", D), ("dt_bias", dt_bias), ("h0", h0)):
+        _opt(n, t, torch.float32)
+    Bt, H, L, P = x.shape
+    N = B.shape[2]
+    if tuple(dt.shape) != (Bt, H, L) or tuple(B.shape) != (Bt, L, N) or tuple(C.shape) != (Bt, L, N):
+        raise ValueError("dt must be (Bt, H, L); B, C (Bt, L, N)")
+    if h0 is not None and tuple(h0.shape) != (Bt, H, N, P):
+        raise ValueError("h0 must be (Bt, H, N, P)")
+    od = torch.bfloat16 if out_dtype is None else out_dtype
+    y = torch.empty((Bt, H, L, P), dtype=od, device=x.device)
+    hl = torch.empty((Bt, H, N, P), dtype=torch.float32, device=x.device) if return_state else None
+    a = _abi.SsdArgs()
+    a.x, a.dt, a.dt_bias, a.A_log, a.B, a.C = _ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A_log), _ptr(B), _ptr(C)
+    a.D, a.h0, a.y, a.h_last = _ptr(D), _ptr(h0), _ptr(y), _ptr(hl)
+    a.Bt, a.H, a.L, a.P, a.N = Bt, H, L, P, N
+    a.in_dtype, a.out_dtype = _abi.SSM_BF16, _DT[od]
+    a.delta_softplus = 1 if delta_softplus else 0
+    if discretization not in _DISC:
+        raise ValueError("discretization must be 'zoh' or 'euler'")
+    a.discretization = _DISC[discretization]
+    lib = _abi.load()
+    need = int(lib.ssm_ssd_workspace_size(ctypes.byref(a)))
+    ws = None
+    if need:
+        ws = torch.empty(need + 256, dtype=torch.uint8, device=x.device)
+        a.workspace = (ws.data_ptr() + 255) & ~255
+        a.workspace_bytes = need
+    _abi.check("ssm_ssd_fwd", lib.ssm_ssd_fwd(ctypes.byref(a), _stream_handle(x.device)))
+    return (y, hl) if return_state else y

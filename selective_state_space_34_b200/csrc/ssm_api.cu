@@ -365,4 +365,89 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   return cuda_status(ssm::launch_bwd(p, a->in_dtype == SSM_BF16, static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {
+  if (!a) return SSM_ERR_NULL;
+  if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
+  if (a->discretization != SSM_ZOH && a->discretization != SSM_EULER) return SSM_ERR_UNSUPPORTED;
+  if (a->Bt < 0 || a->H < 0 || a->L < 0 || a->P < 0 || a->N < 0) return SSM_ERR_SHAPE;
+  if (a->H == 0 || a->P == 0 || a->N == 0) return SSM_ERR_SHAPE;
+  if (a->in_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if ((a->P != 64 && a->P != 128) || (a->N != 64 && a->N != 128)) return SSM_ERR_UNSUPPORTED;
+  int64_t bh, rows, elems;
+  if (!mul_ok(a->Bt, a->H, &bh) || !mul_ok(bh, a->L, &rows) || !mul_ok(rows, a->P, &elems) ||
+      elems > (INT64_C(1) << 50) || (bh > 0 && (a->L + 127) / 128 > (INT64_C(1) << 31) / bh))
+    return SSM_ERR_SHAPE;
+  *empty = (a->Bt == 0 || a->L == 0);
+  if (*empty) return SSM_OK;
+  if (!a->x || !a->dt || !a->A_log || !a->B || !a->C || !a->y) return SSM_ERR_NULL;
+  const void *v16[4] = {a->x, a->B, a->C, a->y};
+  for (const void *p : v16)
+    if (!aligned(p, 16)) return SSM_ERR_ALIGN;
+  if (!aligned(a->dt, 2)) return SSM_ERR_ALIGN;
+  const void *f32[5] = {a->dt_bias, a->A_log, a->D, a->h0, a->h_last};
+  for (const void *p : f32)
+    if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  return SSM_OK;
+}
+}  // namespace
+
+size_t ssm_ssd_workspace_size(const ssm_ssd_args *args) {
+  bool empty = false;
+  if (check_ssd(args, &empty) != SSM_OK || empty) return 0;
+  return ssm::ssd_workspace_bytes(args->Bt, args->H, args->L, args->P, args->N);
+}
+
+ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream) {
+  bool empty = false;
+  ssm_status st = check_ssd(args, &empty);
+  if (st != SSM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (empty) {
+    // nothing to run: the state passes through
+    if (args->h_last && args->Bt > 0) {
+      const size_t nb = sizeof(float) * (size_t)(args->Bt * args->H * args->N * args->P);
+      return cuda_status(args->h0 ? cudaMemcpyAsync(args->h_last, args->h0, nb, cudaMemcpyDeviceToDevice, s)
+                                  : cudaMemsetAsync(args->h_last, 0, nb, s));
+    }
+    return SSM_OK;
+  }
+  const size_t need = ssm::ssd_workspace_bytes(args->Bt, args->H, args->L, args->P, args->N);
+  if (!args->workspace || args->workspace_bytes < need || !aligned(args->workspace, 256))
+    return SSM_ERR_WORKSPACE;
+  auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int64_t nC = (args->L + 127) / 128;
+  const size_t chunks = (size_t)(args->Bt * args->H * nC), np = (size_t)(args->N * args->P);
+  char *w = static_cast<char *>(args->workspace);
+  ssm::SsdParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = args->x;
+  p.dt = args->dt;
+  p.B = args->B;
+  p.C = args->C;
+  p.dt_bias = args->dt_bias;
+  p.A_log = args->A_log;
+  p.D = args->D;
+  p.h0 = args->h0;
+  p.y = args->y;
+  p.h_last = args->h_last;
+  p.Bt = args->Bt;
+  p.H = args->H;
+  p.L = args->L;
+  p.P = args->P;
+  p.N = args->N;
+  p.delta_softplus = args->delta_softplus ? 1 : 0;
+  p.euler = args->discretization == SSM_EULER ? 1 : 0;
+  p.S = reinterpret_cast<float *>(w);
+  w += rnd(sizeof(float) * chunks * np);
+  p.Hin = reinterpret_cast<__nv_bfloat16 *>(w);
+  w += rnd(sizeof(__nv_bfloat16) * chunks * np);
+  p.cum_end = reinterpret_cast<float *>(w);
+  w += rnd(sizeof(float) * chunks);
+  p.error = reinterpret_cast<int *>(w);
+  cudaError_t e = cudaMemsetAsync(p.error, 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(ssm::launch_ssd(p, args->out_dtype == SSM_BF16, s));
+}
+
 }  // extern "C"

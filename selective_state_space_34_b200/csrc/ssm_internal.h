@@ -2,6 +2,7 @@
 // the C-ABI layer. Host/device plain data only; no torch types anywhere in the library.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -42,6 +43,23 @@ struct FwdParams {
   float *seg_hend;        // (n_seg, Bt, Dn, N): end state from a zero start (pass 1)
   float *seg_sdl;         // (n_seg, Bt, Dn): sum of Delta over the segment (pass 1)
 };
+
+// Mamba-2 state-space duality forward (ssm_ssd.cu).
+struct SsdParams {
+  const void *x, *dt, *B, *C;  // bf16: x (Bt, H, L, P), dt (Bt, H, L), B / C (Bt, L, N)
+  const float *dt_bias, *A_log, *D;  // [H]
+  const float *h0;             // (Bt, H, N, P) or null
+  void *y;                     // (Bt, H, L, P), bf16 or fp32
+  float *h_last;               // (Bt, H, N, P) or null
+  int64_t Bt, H, L, P, N;
+  int delta_softplus, euler;
+  float *S;                    // workspace: chunk states (Bt, H, n_chunks, N, P) fp32
+  __nv_bfloat16 *Hin;          // workspace: state entering each chunk, same shape, bf16
+  float *cum_end;              // workspace: log-decay of each chunk (Bt, H, n_chunks)
+  int *error;                  // workspace: set to 1 if a tensor-core wait timed out
+};
+cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream);
+size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);
 
 // Segmentation of a split-L forward: how many segments of which length, and the scratch it needs.
 struct SegPlan {

@@ -1,0 +1,435 @@
+// ssm_ssd.cu -- Mamba-2 state-space duality (SSD) forward on the sm_100a tensor cores.
+//
+// "state-space models" (aarnphm.xyz), "Mamba-2 and state-space duality": within a head the
+// transition is a_t I, so y_t = sum_{s<=t} (C_t . B-bar_s)(prod_{k=s+1..t} a_k) x_s, i.e.
+// Y = (L o Q K^T) V, computed by matrix products within chunks while a state is carried between
+// chunks. With cum_t the running sum of log a over a chunk of Q steps and B-bar_s = beta_s B_s:
+//
+//   S_c      = sum_s e^{cum_end - cum_s} beta_s B_s x_s^T                  (N x P, chunk state)
+//   H_c      = e^{cum_end} H_{c-1} + S_c                                   (state after chunk c)
+//   Y_c[t]   = sum_{s<=t} (C_t . B_s) e^{cum_t - cum_s} beta_s x_s  +  e^{cum_t} C_t H_{c-1}
+//              + D x_t
+//
+// Three kernels: ssd_state_kernel (S_c, one tcgen05 product per chunk and head), ssd_pass_kernel
+// (the carry over chunks, fp32, CUDA cores), ssd_out_kernel (C B^T and C H_{c-1} on the tensor
+// cores, the masked decay applied to C B^T in registers, then the product with X). Operands are
+// bf16 in shared memory in the canonical no-swizzle layouts (8 x 16-byte core matrices);
+// accumulators are fp32 in tensor memory with M = 128, so accumulator row i is TMEM lane i and
+// thread i of the 128-thread CTA owns it. One elected thread issues the MMAs; completion is
+// signalled through an mbarrier whose wait is bounded (on a timeout the kernel records an error
+// and still frees its tensor memory).
+#include "ssm_common.cuh"
+#include "ssm_internal.h"
+#include "ssm_stage.cuh"
+#include "ssm_tmem.cuh"
+#include "ssm_umma.cuh"
+
+namespace ssm {
+
+namespace {
+
+constexpr int kQ = 128;   // chunk length (steps)
+constexpr int kNP = 128;  // padded state dimension (N = 64 runs with zero rows)
+
+// ---- tcgen05 plumbing ----------------------------------------------------------------------
+
+// Shared-memory matrix descriptor of a no-swizzle operand tile (bit layout in ssm_umma.cuh).
+__device__ __forceinline__ uint64_t smem_desc(const void *p, uint32_t lbo, uint32_t sbo) {
+  return umma_smem_desc_bits(static_cast<uint32_t>(__cvta_generic_to_shared(p)), lbo, sbo);
+}
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, int a_mn_major, int b_mn_major) {
+  return umma_instr_desc_bf16_f32(M, N, a_mn_major, b_mn_major);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(a)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");  // visible to the async proxy
+}
+
+// Wait for the phase with parity `phase`; gives up after ~2^22 polls. Returns false on timeout.
+// The result is made warp-uniform by the caller before any warp-collective tcgen05 access.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+  for (int i = 0; i < (1 << 22); i++) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(phase)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, float *v) {
+  float a[16], b[16];
+  tmem_ld2<16>(addr, a, addr + 16, b);
+#pragma unroll
+  for (int i = 0; i < 16; i++) {
+    v[i] = a[i];
+    v[16 + i] = b[i];
+  }
+}
+
+// Byte offset of element (mn, k) in a no-swizzle operand tile with R rows along M/N; core
+// matrices are laid out K-group-major: group (i, j) at (j * R/8 + i) * 128, so sbo = 128 and
+// lbo = R / 8 * 128. K-major rows hold 8 consecutive k; MN-major rows hold 8 consecutive mn.
+__device__ __forceinline__ uint32_t kmaj_off(int R, int mn, int k) {
+  return (uint32_t)(((k >> 3) * (R >> 3) + (mn >> 3)) * 128 + (mn & 7) * 16 + (k & 7) * 2);
+}
+__device__ __forceinline__ uint32_t mnmaj_off(int R, int mn, int k) {
+  return (uint32_t)(((k >> 3) * (R >> 3) + (mn >> 3)) * 128 + (k & 7) * 16 + (mn & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Delta, log a = Delta A and beta of step t of the chunk (0 past the sequence end: an identity
+// step), and the inclusive running sum of log a over the chunk (block-wide scan, 128 threads).
+struct StepCoefs {
+  float la, beta, cum;
+};
+__device__ __forceinline__ StepCoefs chunk_coefs(const SsdParams &p, int64_t bh, int64_t t_glob,
+                                                 float A, float bias, float *scan_buf) {
+  float la = 0.f, beta = 0.f;
+  if (t_glob < p.L) {
+    const float v = to_f32(static_cast<const __nv_bfloat16 *>(p.dt)[bh * p.L + t_glob]) + bias;
+    const float dl = p.delta_softplus ? softplus<false>(v) : v;
+    la = dl * A;
+    beta = p.euler ? dl : expm1f(la) / A;
+  }
+  // inclusive scan of la over the 128 threads
+  float s = la;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float o = __shfl_up_sync(0xffffffffu, s, off);
+    if (lane >= off) s += o;
+  }
+  if (lane == 31) scan_buf[w] = s;
+  __syncthreads();
+  float base = 0.f;
+  for (int i = 0; i < w; i++) base += scan_buf[i];
+  __syncthreads();
+  return StepCoefs{la, beta, s + base};
+}
+
+}  // namespace
+
+// ---- kernel 1: chunk states S_c = (w beta B)^T X -------------------------------------------
+template <int P>
+__global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char *sA = smem;                       // (w beta B)^T: M = n (128), K = s (128), MN-major
+  unsigned char *sX = smem + kNP * kQ * 2;        // X: N = p (P), K = s (128), MN-major
+  float *scan_buf = reinterpret_cast<float *>(sX + P * kQ * 2);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(scan_buf + 8);
+  uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 1);
+
+  const int64_t nC = (p.L + kQ - 1) / kQ;
+  const int64_t c = blockIdx.x % nC, bh = blockIdx.x / nC, b = bh / p.H, h = bh % p.H;
+  const int t = threadIdx.x;
+  const int64_t tg = c * kQ + t;
+
+  const uint32_t tbase = tmem_alloc_cta(slot, (uint32_t)P);
+  if (t == 0) mbar_init(bar, 1);
+
+  const float A = -expf(p.A_log[h]);
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);
+  // total log-decay of the chunk = the last thread's inclusive sum
+  if (t == kQ - 1) scan_buf[4] = k.cum;
+  __syncthreads();
+  const float cum_end = scan_buf[4];
+  const float scale = k.beta * __expf(cum_end - k.cum);  // e^{cum_end - cum_s} beta_s
+
+  // stage row s = t of both operands
+  {
+    const __nv_bfloat16 *Brow = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + tg) * p.N;
+#pragma unroll 4
+    for (int n0 = 0; n0 < kNP; n0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; e++) v[e] = (tg < p.L && n0 + e < p.N) ? to_f32(Brow[n0 + e]) * scale : 0.f;
+      uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+      *reinterpret_cast<uint4 *>(sA + mnmaj_off(kNP, n0, t)) = pk;
+    }
+    const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + tg) * P;
+#pragma unroll 4
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+      if (tg < p.L) pk = *reinterpret_cast<const uint4 *>(xrow + p0);
+      *reinterpret_cast<uint4 *>(sX + mnmaj_off(P, p0, t)) = pk;
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+  tc_fence_after();
+  if (t == 0) {
+    constexpr uint32_t idesc = instr_desc(128, P, 1, 1);
+#pragma unroll
+    for (int ks = 0; ks < kQ / 16; ks++) {
+      const uint64_t da = smem_desc(sA + ks * 2 * (kNP / 8) * 128, (kNP / 8) * 128, 128);
+      const uint64_t db = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+      mma_bf16(tbase, da, db, idesc, ks > 0);
+    }
+    mma_commit(bar);
+  }
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
+  tc_fence_after();
+  if (!ok) {
+    if ((t & 31) == 0) atomicExch(p.error, 1);
+  } else if (t < p.N) {
+    // row n = t of S_c
+    float *dst = p.S + ((bh * nC + c) * p.N + t) * P;
+    const uint32_t lane_addr = tmem_lane_addr(tbase);
+#pragma unroll
+    for (int q = 0; q < P; q += 32) {
+      float v[32];
+      tmem_ld32(lane_addr + q, v);
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(dst + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
+  } else {
+    // lanes past N still take part in the warp-collective loads
+    const uint32_t lane_addr = tmem_lane_addr(tbase);
+#pragma unroll
+    for (int q = 0; q < P; q += 32) {
+      float v[32];
+      tmem_ld32(lane_addr + q, v);
+    }
+  }
+  if (t == 0) p.cum_end[bh * nC + c] = cum_end;
+  tc_fence_before();
+  tmem_free_cta(tbase, (uint32_t)P);
+}
+
+// ---- kernel 2: carry over chunks ------------------------------------------------------------
+// H_in[c] = state entering chunk c (bf16, the MMA operand of kernel 3); H_c = e^{cum_end} H + S_c.
+template <int P>
+__global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
+  const int64_t nC = (p.L + kQ - 1) / kQ;
+  const int64_t bh = blockIdx.x;
+  const int64_t NPs = p.N * P;
+  for (int64_t e = threadIdx.x; e < NPs; e += blockDim.x) {
+    float hcur = p.h0 ? p.h0[bh * NPs + e] : 0.f;
+    for (int64_t c = 0; c < nC; c++) {
+      p.Hin[(bh * nC + c) * NPs + e] = __float2bfloat16_rn(hcur);
+      hcur = fmaf(__expf(p.cum_end[bh * nC + c]), hcur, p.S[(bh * nC + c) * NPs + e]);
+    }
+    if (p.h_last) p.h_last[bh * NPs + e] = hcur;
+  }
+}
+
+// ---- kernel 3: chunk outputs ------------------------------------------------------------------
+template <int P, typename Tout>
+__global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char *sC = smem;                        // C: M = t (128), K = n (128), K-major
+  unsigned char *sB = sC + kQ * kNP * 2;           // B: N = s (128), K = n (128), K-major; then G'
+  unsigned char *sX = sB + kQ * kNP * 2;           // X: N = p (P), K = s (128), MN-major
+  unsigned char *sH = sX + P * kQ * 2;             // H_in: N = p (P), K = n (128), MN-major
+  float *cum_s = reinterpret_cast<float *>(sH + P * kNP * 2);
+  float *beta_s = cum_s + kQ;
+  float *scan_buf = beta_s + kQ;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(scan_buf + 8);  // two barriers
+  uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 2);
+
+  constexpr uint32_t kCols = (128 + 2 * P <= 256) ? 256u : 512u;  // G (128) + Y (P) + C H (P)
+  const int64_t nC = (p.L + kQ - 1) / kQ;
+  const int64_t c = blockIdx.x % nC, bh = blockIdx.x / nC, b = bh / p.H, h = bh % p.H;
+  const int t = threadIdx.x;
+  const int64_t tg = c * kQ + t;
+
+  const uint32_t tbase = tmem_alloc_cta(slot, kCols);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+  }
+  const float A = -expf(p.A_log[h]);
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);
+  cum_s[t] = k.cum;
+  beta_s[t] = k.beta;
+
+  // stage C, B (row t), X (row s = t), H_in (row n = t)
+  {
+    const __nv_bfloat16 *Crow = static_cast<const __nv_bfloat16 *>(p.C) + (b * p.L + tg) * p.N;
+    const __nv_bfloat16 *Brow = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + tg) * p.N;
+#pragma unroll 4
+    for (int n0 = 0; n0 < kNP; n0 += 8) {
+      uint4 pc = make_uint4(0u, 0u, 0u, 0u), pb = pc;
+      if (tg < p.L && n0 < p.N) {
+        pc = *reinterpret_cast<const uint4 *>(Crow + n0);
+        pb = *reinterpret_cast<const uint4 *>(Brow + n0);
+      }
+      *reinterpret_cast<uint4 *>(sC + kmaj_off(kQ, t, n0)) = pc;
+      *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, n0)) = pb;
+    }
+    const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + tg) * P;
+#pragma unroll 4
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+      if (tg < p.L) pk = *reinterpret_cast<const uint4 *>(xrow + p0);
+      *reinterpret_cast<uint4 *>(sX + mnmaj_off(P, p0, t)) = pk;
+    }
+    const __nv_bfloat16 *hrow = p.Hin + ((bh * nC + c) * p.N + t) * P;
+#pragma unroll 4
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+      if (t < p.N) pk = *reinterpret_cast<const uint4 *>(hrow + p0);
+      *reinterpret_cast<uint4 *>(sH + mnmaj_off(P, p0, t)) = pk;
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tG = tbase, tY = tbase + 128, tCH = tbase + 128 + P;
+  if (t == 0) {
+    // G = C B^T (t x s), and C H_in (t x p)
+#pragma unroll
+    for (int ks = 0; ks < kNP / 16; ks++) {
+      const uint64_t dc = smem_desc(sC + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
+      const uint64_t dbm = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
+      const uint64_t dh = smem_desc(sH + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+      mma_bf16(tG, dc, dbm, instr_desc(128, 128, 0, 0), ks > 0);
+      mma_bf16(tCH, dc, dh, instr_desc(128, P, 0, 1), ks > 0);
+    }
+    mma_commit(bar);
+  }
+  bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
+  tc_fence_after();
+  // G'[t][s] = G[t][s] e^{cum_t - cum_s} beta_s for s <= t, written over B as the A operand of
+  // the next product (row t, K = s, K-major); B is no longer read once the barrier fired
+  {
+    const uint32_t lane_addr = tmem_lane_addr(tbase);
+    const float ct = k.cum;
+#pragma unroll 1
+    for (int s0 = 0; s0 < kQ; s0 += 32) {
+      float g[32];
+      tmem_ld32(lane_addr + s0, g);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          const int s = s0 + e + j;
+          v[j] = (s <= t) ? g[e + j] * __expf(ct - cum_s[s]) * beta_s[s] : 0.f;
+        }
+        uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, s0 + e)) = pk;
+      }
+    }
+  }
+  tc_fence_before();
+  fence_async_smem();
+  __syncthreads();
+  tc_fence_after();
+  if (t == 0) {
+#pragma unroll
+    for (int ks = 0; ks < kQ / 16; ks++) {
+      const uint64_t dg = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
+      const uint64_t dx = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+      mma_bf16(tY, dg, dx, instr_desc(128, P, 0, 1), ks > 0);
+    }
+    mma_commit(bar + 1);
+  }
+  ok = __all_sync(0xffffffffu, mbar_wait(bar + 1, 0)) && ok;
+  tc_fence_after();
+  {
+    const uint32_t lane_addr = tmem_lane_addr(tbase);
+    const float et = __expf(k.cum);
+    const float Dh = p.D ? p.D[h] : 0.f;
+    Tout *yrow = static_cast<Tout *>(p.y) + (bh * p.L + tg) * P;
+#pragma unroll 1
+    for (int q = 0; q < P; q += 32) {
+      float yv[32], cv[32];
+      tmem_ld32(lane_addr + 128 + q, yv);
+      tmem_ld32(lane_addr + 128 + P + q, cv);
+      if (ok && tg < p.L) {
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+          const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sX + mnmaj_off(P, q + j, t)));
+          o[j] = fmaf(et, cv[j], yv[j]) + Dh * xv;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) VecStore<Tout, 4>::run(yrow + q + j, o + j);
+      }
+    }
+  }
+  if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
+  tc_fence_before();
+  tmem_free_cta(tbase, kCols);
+}
+
+// ---- host ------------------------------------------------------------------------------------
+
+size_t ssd_smem_state(int P) { return (size_t)kNP * kQ * 2 + (size_t)P * kQ * 2 + 64; }
+size_t ssd_smem_out(int P) { return (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2 + 2 * kQ * 4 + 64; }
+
+template <int P, typename Tout>
+static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
+  const int64_t nC = (p.L + kQ - 1) / kQ;
+  const int64_t grid = p.Bt * p.H * nC;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const size_t s1 = ssd_smem_state(P), s3 = ssd_smem_out(P);
+  cudaError_t e = cudaFuncSetAttribute(ssd_state_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(ssd_out_kernel<P, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+  if (e != cudaSuccess) return e;
+  ssd_state_kernel<P><<<(unsigned)grid, 128, s1, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ssd_out_kernel<P, Tout><<<(unsigned)grid, 128, s3, s>>>(p);
+  return cudaGetLastError();
+}
+
+size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N) {
+  auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int64_t nC = (L + kQ - 1) / kQ;
+  const size_t chunks = (size_t)(Bt * H * nC);
+  return rnd(sizeof(float) * chunks * N * P)               // S
+         + rnd(sizeof(__nv_bfloat16) * chunks * N * P)     // H_in
+         + rnd(sizeof(float) * chunks)                     // cum_end
+         + 256;                                            // error flag
+}
+
+cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream) {
+  if (p.P == 64) return out_bf16 ? launch_ssd_t<64, __nv_bfloat16>(p, stream) : launch_ssd_t<64, float>(p, stream);
+  if (p.P == 128) return out_bf16 ? launch_ssd_t<128, __nv_bfloat16>(p, stream) : launch_ssd_t<128, float>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ssm

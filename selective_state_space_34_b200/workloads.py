@@ -144,6 +144,29 @@ def carried_state(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional
     }
 
 
+def generate_ssd(Bt: int, H: int, L: int, P: int, N: int, seed: int = 1008) -> Dict[str, np.ndarray]:
+    """Inputs of a Mamba-2 state-space-duality layer (the pages give no SSD shapes or
+    distributions; these follow the selective-scan workloads): x ~ N(0, 1) (Bt, H, L, P),
+    dt ~ N(0, 1) (Bt, H, L), B, C ~ N(0, 1/sqrt(N)) (Bt, L, N), all bf16-rounded; per head
+    A_log = ln(1..H spread over [1, 16]), dt_bias = softplus^-1 of a log-uniform step in
+    [1e-3, 1e-1], D = 1."""
+    out: Dict[str, np.ndarray] = {}
+    out["x"] = round_to_bf16(_normal(seed, 21, (Bt, H, L, P), 1.0))
+    out["dt"] = round_to_bf16(_normal(seed, 22, (Bt, H, L), 1.0))
+    std = 1.0 / math.sqrt(N)
+    out["B"] = round_to_bf16(_normal(seed, 23, (Bt, L, N), std))
+    out["C"] = round_to_bf16(_normal(seed, 24, (Bt, L, N), std))
+    out["A_log"] = np.log(np.linspace(1.0, 16.0, H)).astype(np.float32)
+    lu = _rng(seed, 25).uniform(math.log(1e-3), math.log(1e-1), size=H)
+    out["dt_bias"] = softplus_inverse(np.exp(lu)).astype(np.float32)
+    out["D"] = np.ones(H, dtype=np.float32)
+    return out
+
+
+# Mamba-2-style layer on the 1.4B-shaped block: d_inner 4096 as 64 heads of 64, d_state 128.
+SSD_WORKLOADS = {"ssd_fwd": dict(Bt=4, H=64, L=4096, P=64, N=128, seed=1008)}
+
+
 def shaped(base: str, **overrides) -> Workload:
     """A named workload with some fields replaced (e.g. smaller Bt/Dn/L for a parity case)."""
     return replace(WORKLOADS[base], **overrides)

@@ -52,6 +52,8 @@ def _header_fields(struct):
     ("ssm_bwd_args", "BwdArgs", 208 + 17 * 8 + 8),
     # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
     ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
+    # 10 pointers, 5 int64, 4 int32, workspace pointer and size
+    ("ssm_ssd_args", "SsdArgs", 10 * 8 + 5 * 8 + 4 * 4 + 8 + 8),
 ])
 def test_struct_layout_matches_header_field_order(struct, cls, size):
     ct = [f[0] for f in getattr(_abi, cls)._fields_]
@@ -194,6 +196,37 @@ def test_step_validation_codes(lib):
     assert f(_step(conv_w=0x8000, K=4, conv_hist=0x9001)) == 3
     assert f(_step(h=0x6002)) == 3
     assert f(_step(Bt=0, x=None, h=None)) == 0        # no rows: nothing to do
+
+
+def _ssd(**kw):
+    a = _abi.SsdArgs()
+    a.x, a.dt, a.A_log, a.B, a.C, a.y = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000
+    a.Bt, a.H, a.L, a.P, a.N = 2, 4, 300, 64, 128
+    a.in_dtype, a.out_dtype, a.delta_softplus = 1, 1, 1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_ssd_validation_codes(lib):
+    f = lambda a: lib.ssm_ssd_fwd(ctypes.byref(a), None)
+    size = lambda a: lib.ssm_ssd_workspace_size(ctypes.byref(a))
+    assert lib.ssm_ssd_fwd(None, None) == 1
+    assert f(_ssd(x=None)) == 1
+    assert f(_ssd(in_dtype=0)) == 5            # fp32 inputs: tensor-core path is bf16 only
+    assert f(_ssd(out_dtype=3)) == 4
+    assert f(_ssd(P=32)) == 5 and f(_ssd(N=16)) == 5
+    assert f(_ssd(H=0)) == 2 and f(_ssd(L=-1)) == 2
+    assert f(_ssd(discretization=2)) == 5
+    assert f(_ssd(x=0x10008)) == 3             # 16-byte alignment of the tile loads
+    assert f(_ssd(dt=0x20001)) == 3
+    assert f(_ssd(Bt=0, x=None)) == 0          # empty: nothing launched
+    assert f(_ssd()) == 7                      # no workspace
+    need = size(_ssd())
+    # 2 x 4 heads x 3 chunks: S (fp32) + H_in (bf16) of 128 x 64, one log-decay each, error word
+    rnd = lambda v: (v + 255) // 256 * 256
+    assert need == rnd(24 * 128 * 64 * 4) + rnd(24 * 128 * 64 * 2) + rnd(24 * 4) + 256
+    assert f(_ssd(workspace=0x100010, workspace_bytes=need)) == 7
 
 
 def test_conv_validation_codes(lib):

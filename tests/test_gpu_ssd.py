@@ -1,0 +1,99 @@
+"""Parity of the Mamba-2 state-space-duality forward on the tensor cores ("state-space models",
+"Mamba-2 and state-space duality") against the float64 recurrence of the oracle.
+
+Tolerance, from the arithmetic: three bf16 roundings reach an output -- beta_s e^{cum_end-cum_s}
+B_s as an operand of the chunk-state product, the state entering a chunk, and the masked scores
+(C_t . B_s) e^{cum_t-cum_s} beta_s -- each a relative error of at most 2^-9 per term, with fp32
+accumulation. So |y - y_ref| <= 3 * 2^-9 * Y_abs where Y_abs bounds the sum of the terms' magnitudes:
+the oracle run on |x|, |B|, |C|, |D| (|C_t . B_s| <= |C_t| . |B_s|; beta, the decays and the state
+recursion are non-negative maps of non-negative inputs). The tests allow 2^-6 * Y_abs, plus 2^-8 |y|
+for a bf16 output."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_34_b200 as ssm
+from selective_state_space_34_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(Bt, H, L, P, N, out_dtype=torch.float32, euler=False, softplus=True, carry=False, D=True,
+         seed=7):
+    a = wl.generate_ssd(Bt, H, L, P, N, seed=seed)
+    if not softplus:
+        # without softplus dt + dt_bias is Delta itself: a step size, so non-negative
+        a["dt"] = wl.round_to_bf16(np.abs(a["dt"]) * np.float32(0.05))
+        a["dt_bias"] = np.zeros_like(a["dt_bias"])
+    dev = "cuda"
+    t = {k: torch.from_numpy(v).to(dev, torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    h0 = None
+    if carry:
+        h0_np = np.random.default_rng(seed).standard_normal((Bt, H, N, P)).astype(np.float32) * 0.3
+        h0 = torch.from_numpy(h0_np).to(dev)
+    r = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"] if D else None,
+                        dt_bias=t["dt_bias"], h0=h0, delta_softplus=softplus, out_dtype=out_dtype,
+                        discretization="euler" if euler else "zoh", return_state=carry)
+    torch.cuda.synchronize()
+    y = (r[0] if carry else r).float().cpu().numpy()
+    kw = dict(dt_bias=a["dt_bias"], delta_softplus=softplus, euler=euler)
+    ref = oracle.ssd_fwd(a["x"], a["dt"], a["A_log"], a["B"], a["C"], D=a["D"] if D else None,
+                         h0=None if h0 is None else h0.cpu().numpy(), want_state=carry, **kw)
+    yref = ref[0] if carry else ref
+    yabs = oracle.ssd_fwd(np.abs(a["x"]), a["dt"], a["A_log"], np.abs(a["B"]), np.abs(a["C"]),
+                          D=np.abs(a["D"]) if D else None,
+                          h0=None if h0 is None else np.abs(h0.cpu().numpy()), **kw)
+    tol = 2.0 ** -6 * yabs + (2.0 ** -8 * np.abs(yref) if out_dtype == torch.bfloat16 else 0.0) + 1e-6
+    err = np.abs(y - yref)
+    bad = err > tol
+    assert np.all(np.isfinite(y))
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - tol), err.shape)
+        raise AssertionError("%d/%d outside the bound; worst at %s: gpu %r oracle %r bound %r"
+                             % (bad.sum(), bad.size, i, y[i], yref[i], tol[i]))
+    if carry:
+        hl = r[1].cpu().numpy()
+        # the final state is fp32 throughout except the chunk-state products' bf16 operands
+        habs = oracle.ssd_fwd(np.abs(a["x"]), a["dt"], a["A_log"], np.abs(a["B"]), np.abs(a["C"]),
+                              h0=np.abs(h0.cpu().numpy()), want_state=True, **kw)[1]
+        assert np.all(np.abs(hl - ref[1]) <= 2.0 ** -7 * habs + 1e-6)
+    return y, yref
+
+
+@pytest.mark.parametrize("P,N", [(64, 128), (64, 64), (128, 128), (128, 64)])
+@pytest.mark.parametrize("L", [128, 300, 1])
+def test_ssd_shapes(P, N, L):
+    _run(2, 3, L, P, N)
+
+
+@pytest.mark.parametrize("variant", ["euler", "no_softplus", "bf16_out", "no_D", "carried_state"])
+def test_ssd_variants(variant):
+    _run(1, 2, 257, 64, 128, euler=variant == "euler", softplus=variant != "no_softplus",
+         out_dtype=torch.bfloat16 if variant == "bf16_out" else torch.float32,
+         D=variant != "no_D", carry=variant == "carried_state")
+
+
+def test_ssd_longer_sequence():
+    """16 chunks: the carried state crosses many chunk boundaries."""
+    _run(1, 4, 2048, 64, 128)
+
+
+def test_ssd_matches_selective_scan_for_one_channel_semantics():
+    """Cross-check of the two CUDA paths' shared discretisation: with one head, the SSD of a
+    sequence whose x is the same in all P channels equals P copies of the per-channel result, and
+    the result is linear in x (doubling x doubles y)."""
+    a = wl.generate_ssd(1, 2, 200, 64, 64, seed=3)
+    x1 = a["x"].copy()
+    x1[...] = a["x"][..., :1]
+    t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    xs = torch.from_numpy(x1).to("cuda", torch.bfloat16)
+    y = ssm.ssm_ssd_fwd(xs, t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
+                        out_dtype=torch.float32)
+    y2 = ssm.ssm_ssd_fwd(xs * 2, t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
+                         out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(y, y[..., :1].expand_as(y), rtol=1e-6, atol=1e-7)  # same per channel
+    assert torch.equal(y2, 2 * y)     # exact: scaling by 2 commutes with every rounding on the way
