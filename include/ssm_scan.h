@@ -175,9 +175,10 @@ typedef struct ssm_ssd_args {
   const void *B;         /* device (Bt, L, N) bf16, 16-byte aligned */
   const void *C;         /* device (Bt, L, N) bf16, 16-byte aligned */
   const float *D;        /* device [H] or NULL (= 0) */
-  const float *h0;       /* device (Bt, H, N, P) fp32 or NULL (= 0) */
+  const float *h0;       /* device (Bt, H, N, P) fp32, 16-byte aligned, or NULL (= 0) */
   void *y;               /* device (Bt, H, L, P) out_dtype, 16-byte aligned */
-  float *h_last;         /* device (Bt, H, N, P) fp32 or NULL: the state after step L-1 */
+  float *h_last;         /* device (Bt, H, N, P) fp32, 16-byte aligned, or NULL: the state after
+                            step L-1 */
   int64_t Bt, H, L, P, N;
   int32_t in_dtype;      /* must be SSM_BF16 */
   int32_t out_dtype;     /* SSM_BF16 or SSM_F32 */

@@ -385,9 +385,10 @@ ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {
   for (const void *p : v16)
     if (!aligned(p, 16)) return SSM_ERR_ALIGN;
   if (!aligned(a->dt, 2)) return SSM_ERR_ALIGN;
-  const void *f32[5] = {a->dt_bias, a->A_log, a->D, a->h0, a->h_last};
+  const void *f32[3] = {a->dt_bias, a->A_log, a->D};
   for (const void *p : f32)
     if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
+  if ((a->h0 && !aligned(a->h0, 16)) || (a->h_last && !aligned(a->h_last, 16))) return SSM_ERR_ALIGN;
   return SSM_OK;
 }
 }  // namespace

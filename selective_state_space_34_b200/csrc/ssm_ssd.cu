@@ -30,6 +30,7 @@ namespace {
 
 constexpr int kQ = 128;   // chunk length (steps)
 constexpr int kNP = 128;  // padded state dimension (N = 64 runs with zero rows)
+constexpr int kSsdHeader = 2048;  // bytes of small per-CTA data in front of the tiles
 
 // ---- tcgen05 plumbing ----------------------------------------------------------------------
 
@@ -115,6 +116,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Cooperative copy of a tile of R rows x VPR 16-byte vectors (8 bf16 each) from a row-major
+// source into an operand tile: vector (row, v) goes to smem_off(row, v). Row r of the source
+// starts at src + r * rs elements; rows with valid(r) false, and vectors past vmax, read as zero.
+// A warp takes 8 rows x 4 vectors: 64 contiguous bytes per row from global memory, and the 8
+// lanes of each shared-memory phase write 8 different core-matrix rows (distinct banks).
+template <int R, int VPR, typename Off, typename Valid, typename Xform>
+__device__ __forceinline__ void coop_tile(unsigned char *tile, const __nv_bfloat16 *src, int64_t rs,
+                                          int vmax, Off smem_off, Valid valid, Xform xform) {
+  static_assert(R % 8 == 0 && (R * VPR) % 128 == 0, "tile shape");
+#pragma unroll 4
+  for (int it = 0; it < R * VPR / 128; it++) {
+    const int idx = it * 128 + threadIdx.x;
+    const int r8 = idx & 7, v = (idx >> 3) % VPR, rg = (idx >> 3) / VPR;
+    const int row = rg * 8 + r8;
+    uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+    if (valid(row) && v < vmax) pk = *reinterpret_cast<const uint4 *>(src + (int64_t)row * rs + v * 8);
+    *reinterpret_cast<uint4 *>(tile + smem_off(row, v)) = xform(row, pk);
+  }
+}
+struct NoXform {
+  __device__ __forceinline__ uint4 operator()(int, uint4 v) const { return v; }
+};
+
 // Delta, log a = Delta A and beta of step t of the chunk (0 past the sequence end: an identity
 // step), and the inclusive running sum of log a over the chunk (block-wide scan, 128 threads).
 struct StepCoefs {
@@ -151,11 +175,13 @@ __device__ __forceinline__ StepCoefs chunk_coefs(const SsdParams &p, int64_t bh,
 template <int P>
 __global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char *sA = smem;                       // (w beta B)^T: M = n (128), K = s (128), MN-major
-  unsigned char *sX = smem + kNP * kQ * 2;        // X: N = p (P), K = s (128), MN-major
-  float *scan_buf = reinterpret_cast<float *>(sX + P * kQ * 2);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(scan_buf + 8);
-  uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 1);
+  // header (scan scratch, per-row scales, barrier, TMEM address), then the operand tiles; the
+  // tiles' region is reused afterwards to stage the result rows
+  float *scan_buf = reinterpret_cast<float *>(smem);                 // 8 + kQ floats
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSsdHeader - 16);
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + kSsdHeader - 8);
+  unsigned char *sA = smem + kSsdHeader;          // (w beta B)^T: M = n (128), K = s (128), MN-major
+  unsigned char *sX = sA + kNP * kQ * 2;          // X: N = p (P), K = s (128), MN-major
 
   const int64_t nC = (p.L + kQ - 1) / kQ;
   const int64_t c = blockIdx.x % nC, bh = blockIdx.x / nC, b = bh / p.H, h = bh % p.H;
@@ -174,24 +200,32 @@ __global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
   const float cum_end = scan_buf[4];
   const float scale = k.beta * __expf(cum_end - k.cum);  // e^{cum_end - cum_s} beta_s
 
-  // stage row s = t of both operands
+  // stage both operands: row s of B scaled by e^{cum_end - cum_s} beta_s (A operand, MN-major
+  // along n), row s of X (B operand, MN-major along p)
+  float *row_scale = scan_buf + 8;  // kQ floats after the scan scratch
+  row_scale[t] = scale;
+  __syncthreads();
   {
-    const __nv_bfloat16 *Brow = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + tg) * p.N;
-#pragma unroll 4
-    for (int n0 = 0; n0 < kNP; n0 += 8) {
-      float v[8];
+    const int64_t rows_left = p.L - c * kQ;
+    auto valid = [&](int r) { return r < rows_left; };
+    const __nv_bfloat16 *Bsrc = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + c * kQ) * p.N;
+    coop_tile<kQ, kNP / 8>(sA, Bsrc, p.N, (int)(p.N / 8),
+                           [](int r, int v) { return mnmaj_off(kNP, v * 8, r); }, valid,
+                           [&](int r, uint4 pk) {
+                             const float sc = row_scale[r];
+                             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&pk);
+                             uint4 o;
+                             uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
-      for (int e = 0; e < 8; e++) v[e] = (tg < p.L && n0 + e < p.N) ? to_f32(Brow[n0 + e]) * scale : 0.f;
-      uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-      *reinterpret_cast<uint4 *>(sA + mnmaj_off(kNP, n0, t)) = pk;
-    }
-    const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + tg) * P;
-#pragma unroll 4
-    for (int p0 = 0; p0 < P; p0 += 8) {
-      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-      if (tg < p.L) pk = *reinterpret_cast<const uint4 *>(xrow + p0);
-      *reinterpret_cast<uint4 *>(sX + mnmaj_off(P, p0, t)) = pk;
-    }
+                             for (int i = 0; i < 4; i++) {
+                               const float2 f = __bfloat1622float2(h2[i]);
+                               ow[i] = pack_bf16(f.x * sc, f.y * sc);
+                             }
+                             return o;
+                           });
+    const __nv_bfloat16 *Xsrc = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
+    coop_tile<kQ, P / 8>(sX, Xsrc, P, P / 8, [](int r, int v) { return mnmaj_off(P, v * 8, r); },
+                         valid, NoXform());
   }
   fence_async_smem();
   __syncthreads();
@@ -208,26 +242,28 @@ __global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
   }
   const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
   tc_fence_after();
-  if (!ok) {
-    if ((t & 31) == 0) atomicExch(p.error, 1);
-  } else if (t < p.N) {
-    // row n = t of S_c
-    float *dst = p.S + ((bh * nC + c) * p.N + t) * P;
+  if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
+  // row n = t of S_c: TMEM -> registers -> shared (padded rows, over the consumed A tile) ->
+  // coalesced global stores
+  constexpr int SR = P + 4;  // padded row, floats
+  float *stage = reinterpret_cast<float *>(sA);
+  {
     const uint32_t lane_addr = tmem_lane_addr(tbase);
 #pragma unroll
     for (int q = 0; q < P; q += 32) {
       float v[32];
       tmem_ld32(lane_addr + q, v);
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(dst + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4 *>(stage + t * SR + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     }
-  } else {
-    // lanes past N still take part in the warp-collective loads
-    const uint32_t lane_addr = tmem_lane_addr(tbase);
-#pragma unroll
-    for (int q = 0; q < P; q += 32) {
-      float v[32];
-      tmem_ld32(lane_addr + q, v);
+  }
+  __syncthreads();
+  if (ok) {
+    float *dst = p.S + (bh * nC + c) * p.N * P;
+    for (int i = t; i < p.N * P / 4; i += 128) {
+      const int r = i / (P / 4), q = (i % (P / 4)) * 4;
+      *reinterpret_cast<float4 *>(dst + r * P + q) = *reinterpret_cast<const float4 *>(stage + r * SR + q);
     }
   }
   if (t == 0) p.cum_end[bh * nC + c] = cum_end;
@@ -239,32 +275,42 @@ __global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
 // H_in[c] = state entering chunk c (bf16, the MMA operand of kernel 3); H_c = e^{cum_end} H + S_c.
 template <int P>
 __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
+  // grid: (batch x head) x (N P / 1024); each thread carries 4 consecutive state entries
   const int64_t nC = (p.L + kQ - 1) / kQ;
-  const int64_t bh = blockIdx.x;
   const int64_t NPs = p.N * P;
-  for (int64_t e = threadIdx.x; e < NPs; e += blockDim.x) {
-    float hcur = p.h0 ? p.h0[bh * NPs + e] : 0.f;
-    for (int64_t c = 0; c < nC; c++) {
-      p.Hin[(bh * nC + c) * NPs + e] = __float2bfloat16_rn(hcur);
-      hcur = fmaf(__expf(p.cum_end[bh * nC + c]), hcur, p.S[(bh * nC + c) * NPs + e]);
-    }
-    if (p.h_last) p.h_last[bh * NPs + e] = hcur;
+  const int64_t per = NPs / 1024;
+  const int64_t bh = blockIdx.x / per;
+  const int64_t e = (blockIdx.x % per) * 1024 + threadIdx.x * 4;
+  float4 hcur = p.h0 ? *reinterpret_cast<const float4 *>(p.h0 + bh * NPs + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float *S = p.S + bh * nC * NPs + e;
+  __nv_bfloat16 *Hin = p.Hin + bh * nC * NPs + e;
+  const float *ce = p.cum_end + bh * nC;
+#pragma unroll 4
+  for (int64_t c = 0; c < nC; c++) {
+    const float4 sv = *reinterpret_cast<const float4 *>(S + c * NPs);
+    const float a = __expf(ce[c]);
+    uint2 pk;
+    pk.x = pack_bf16(hcur.x, hcur.y);
+    pk.y = pack_bf16(hcur.z, hcur.w);
+    *reinterpret_cast<uint2 *>(Hin + c * NPs) = pk;
+    hcur = make_float4(fmaf(a, hcur.x, sv.x), fmaf(a, hcur.y, sv.y), fmaf(a, hcur.z, sv.z), fmaf(a, hcur.w, sv.w));
   }
+  if (p.h_last) *reinterpret_cast<float4 *>(p.h_last + bh * NPs + e) = hcur;
 }
 
 // ---- kernel 3: chunk outputs ------------------------------------------------------------------
 template <int P, typename Tout>
 __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char *sC = smem;                        // C: M = t (128), K = n (128), K-major
+  float *cum_s = reinterpret_cast<float *>(smem);  // header: 2 kQ + 8 floats, 2 barriers, slot
+  float *beta_s = cum_s + kQ;
+  float *scan_buf = beta_s + kQ;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSsdHeader - 24);  // two barriers
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + kSsdHeader - 8);
+  unsigned char *sC = smem + kSsdHeader;           // C: M = t (128), K = n (128), K-major
   unsigned char *sB = sC + kQ * kNP * 2;           // B: N = s (128), K = n (128), K-major; then G'
   unsigned char *sX = sB + kQ * kNP * 2;           // X: N = p (P), K = s (128), MN-major
   unsigned char *sH = sX + P * kQ * 2;             // H_in: N = p (P), K = n (128), MN-major
-  float *cum_s = reinterpret_cast<float *>(sH + P * kNP * 2);
-  float *beta_s = cum_s + kQ;
-  float *scan_buf = beta_s + kQ;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(scan_buf + 8);  // two barriers
-  uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 2);
 
   constexpr uint32_t kCols = (128 + 2 * P <= 256) ? 256u : 512u;  // G (128) + Y (P) + C H (P)
   const int64_t nC = (p.L + kQ - 1) / kQ;
@@ -283,34 +329,18 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
   cum_s[t] = k.cum;
   beta_s[t] = k.beta;
 
-  // stage C, B (row t), X (row s = t), H_in (row n = t)
+  // stage C and B (rows t / s, K = n, K-major), X (rows s, MN-major along p), H_in (rows n)
   {
-    const __nv_bfloat16 *Crow = static_cast<const __nv_bfloat16 *>(p.C) + (b * p.L + tg) * p.N;
-    const __nv_bfloat16 *Brow = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + tg) * p.N;
-#pragma unroll 4
-    for (int n0 = 0; n0 < kNP; n0 += 8) {
-      uint4 pc = make_uint4(0u, 0u, 0u, 0u), pb = pc;
-      if (tg < p.L && n0 < p.N) {
-        pc = *reinterpret_cast<const uint4 *>(Crow + n0);
-        pb = *reinterpret_cast<const uint4 *>(Brow + n0);
-      }
-      *reinterpret_cast<uint4 *>(sC + kmaj_off(kQ, t, n0)) = pc;
-      *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, n0)) = pb;
-    }
-    const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + tg) * P;
-#pragma unroll 4
-    for (int p0 = 0; p0 < P; p0 += 8) {
-      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-      if (tg < p.L) pk = *reinterpret_cast<const uint4 *>(xrow + p0);
-      *reinterpret_cast<uint4 *>(sX + mnmaj_off(P, p0, t)) = pk;
-    }
-    const __nv_bfloat16 *hrow = p.Hin + ((bh * nC + c) * p.N + t) * P;
-#pragma unroll 4
-    for (int p0 = 0; p0 < P; p0 += 8) {
-      uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-      if (t < p.N) pk = *reinterpret_cast<const uint4 *>(hrow + p0);
-      *reinterpret_cast<uint4 *>(sH + mnmaj_off(P, p0, t)) = pk;
-    }
+    const int64_t rows_left = p.L - c * kQ;
+    auto valid = [&](int r) { return r < rows_left; };
+    const int64_t off = (b * p.L + c * kQ) * p.N;
+    const auto kmaj = [](int r, int v) { return kmaj_off(kQ, r, v * 8); };
+    coop_tile<kQ, kNP / 8>(sC, static_cast<const __nv_bfloat16 *>(p.C) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
+    coop_tile<kQ, kNP / 8>(sB, static_cast<const __nv_bfloat16 *>(p.B) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
+    const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
+    coop_tile<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid, NoXform());
+    const int64_t nrows = p.N;
+    coop_tile<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; }, NoXform());
   }
   fence_async_smem();
   __syncthreads();
@@ -367,26 +397,40 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
   }
   ok = __all_sync(0xffffffffu, mbar_wait(bar + 1, 0)) && ok;
   tc_fence_after();
+  // y row t = G'X + e^{cum_t} C H_in (fp32) -> shared (padded rows, over the consumed tiles)
+  constexpr int SR = P + 4;
+  float *stage = reinterpret_cast<float *>(sC);
   {
     const uint32_t lane_addr = tmem_lane_addr(tbase);
     const float et = __expf(k.cum);
-    const float Dh = p.D ? p.D[h] : 0.f;
-    Tout *yrow = static_cast<Tout *>(p.y) + (bh * p.L + tg) * P;
 #pragma unroll 1
     for (int q = 0; q < P; q += 32) {
       float yv[32], cv[32];
       tmem_ld32(lane_addr + 128 + q, yv);
       tmem_ld32(lane_addr + 128 + P + q, cv);
-      if (ok && tg < p.L) {
-        float o[32];
 #pragma unroll
-        for (int j = 0; j < 32; j++) {
-          const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sX + mnmaj_off(P, q + j, t)));
-          o[j] = fmaf(et, cv[j], yv[j]) + Dh * xv;
-        }
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) VecStore<Tout, 4>::run(yrow + q + j, o + j);
-      }
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(stage + t * SR + q + j) =
+            make_float4(fmaf(et, cv[j], yv[j]), fmaf(et, cv[j + 1], yv[j + 1]),
+                        fmaf(et, cv[j + 2], yv[j + 2]), fmaf(et, cv[j + 3], yv[j + 3]));
+    }
+  }
+  __syncthreads();
+  // coalesced: + D x (x from global), one rounding to the output type
+  if (ok) {
+    const float Dh = p.D ? p.D[h] : 0.f;
+    const int64_t rows_left = p.L - c * kQ;
+    const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
+    Tout *ys = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ) * P;
+    for (int i = t; i < kQ * P / 4; i += 128) {
+      const int r = i / (P / 4), q = (i % (P / 4)) * 4;
+      if (r >= rows_left) continue;
+      const float4 v = *reinterpret_cast<const float4 *>(stage + r * SR + q);
+      const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (int64_t)r * P + q);
+      const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
+      const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
+      const float o[4] = {fmaf(Dh, x01.x, v.x), fmaf(Dh, x01.y, v.y), fmaf(Dh, x23.x, v.z), fmaf(Dh, x23.y, v.w)};
+      VecStore<Tout, 4>::run(ys + (int64_t)r * P + q, o);
     }
   }
   if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
@@ -396,8 +440,16 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
 
 // ---- host ------------------------------------------------------------------------------------
 
-size_t ssd_smem_state(int P) { return (size_t)kNP * kQ * 2 + (size_t)P * kQ * 2 + 64; }
-size_t ssd_smem_out(int P) { return (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2 + 2 * kQ * 4 + 64; }
+// header + operand tiles, or header + the padded fp32 result rows staged over them
+size_t ssd_smem_state(int P) {
+  const size_t tiles = (size_t)kNP * kQ * 2 + (size_t)P * kQ * 2, stage = (size_t)kNP * (P + 4) * 4;
+  return kSsdHeader + (tiles > stage ? tiles : stage);
+}
+size_t ssd_smem_out(int P) {
+  const size_t tiles = (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2;
+  const size_t stage = (size_t)kQ * (P + 4) * 4;
+  return kSsdHeader + (tiles > stage ? tiles : stage);
+}
 
 template <int P, typename Tout>
 static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
@@ -410,7 +462,7 @@ static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   ssd_state_kernel<P><<<(unsigned)grid, 128, s1, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H), 256, 0, s>>>(p);
+  ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H * (p.N * P / 1024)), 256, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ssd_out_kernel<P, Tout><<<(unsigned)grid, 128, s3, s>>>(p);
   return cudaGetLastError();

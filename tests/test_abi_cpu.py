@@ -220,6 +220,7 @@ def test_ssd_validation_codes(lib):
     assert f(_ssd(discretization=2)) == 5
     assert f(_ssd(x=0x10008)) == 3             # 16-byte alignment of the tile loads
     assert f(_ssd(dt=0x20001)) == 3
+    assert f(_ssd(h0=0x70004)) == 3 and f(_ssd(h_last=0x70008)) == 3
     assert f(_ssd(Bt=0, x=None)) == 0          # empty: nothing launched
     assert f(_ssd()) == 7                      # no workspace
     need = size(_ssd())
