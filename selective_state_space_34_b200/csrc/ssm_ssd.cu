@@ -299,8 +299,10 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
 }
 
 // ---- kernel 3: chunk outputs ------------------------------------------------------------------
+// One CTA per (batch, chunk, group of HG heads): C and B are shared by the heads, so they are
+// staged once and G = C B^T is formed once; each head then applies its own decays to G.
 template <int P, typename Tout>
-__global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int HG) {
   extern __shared__ __align__(1024) unsigned char smem[];
   float *cum_s = reinterpret_cast<float *>(smem);  // header: 2 kQ + 8 floats, 2 barriers, slot
   float *beta_s = cum_s + kQ;
@@ -308,130 +310,136 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p) {
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSsdHeader - 24);  // two barriers
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + kSsdHeader - 8);
   unsigned char *sC = smem + kSsdHeader;           // C: M = t (128), K = n (128), K-major
-  unsigned char *sB = sC + kQ * kNP * 2;           // B: N = s (128), K = n (128), K-major; then G'
+  unsigned char *sB = sC + kQ * kNP * 2;           // B: N = s, K = n, K-major; then each head's G'
   unsigned char *sX = sB + kQ * kNP * 2;           // X: N = p (P), K = s (128), MN-major
   unsigned char *sH = sX + P * kQ * 2;             // H_in: N = p (P), K = n (128), MN-major
+  float *stage = reinterpret_cast<float *>(sB);    // result rows, over G' and X once consumed
 
   constexpr uint32_t kCols = (128 + 2 * P <= 256) ? 256u : 512u;  // G (128) + Y (P) + C H (P)
   const int64_t nC = (p.L + kQ - 1) / kQ;
-  const int64_t c = blockIdx.x % nC, bh = blockIdx.x / nC, b = bh / p.H, h = bh % p.H;
+  const int64_t ngrp = p.H / HG;
+  const int64_t c = blockIdx.x % nC, rest = blockIdx.x / nC;
+  const int64_t hgrp = rest % ngrp, b = rest / ngrp;
   const int t = threadIdx.x;
   const int64_t tg = c * kQ + t;
+  const int64_t rows_left = p.L - c * kQ;
+  auto valid = [&](int r) { return r < rows_left; };
 
   const uint32_t tbase = tmem_alloc_cta(slot, kCols);
   if (t == 0) {
     mbar_init(bar, 1);
     mbar_init(bar + 1, 1);
   }
-  const float A = -expf(p.A_log[h]);
-  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
-  const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);
-  cum_s[t] = k.cum;
-  beta_s[t] = k.beta;
-
-  // stage C and B (rows t / s, K = n, K-major), X (rows s, MN-major along p), H_in (rows n)
   {
-    const int64_t rows_left = p.L - c * kQ;
-    auto valid = [&](int r) { return r < rows_left; };
     const int64_t off = (b * p.L + c * kQ) * p.N;
     const auto kmaj = [](int r, int v) { return kmaj_off(kQ, r, v * 8); };
     coop_tile<kQ, kNP / 8>(sC, static_cast<const __nv_bfloat16 *>(p.C) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
     coop_tile<kQ, kNP / 8>(sB, static_cast<const __nv_bfloat16 *>(p.B) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
-    const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
-    coop_tile<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid, NoXform());
-    const int64_t nrows = p.N;
-    coop_tile<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; }, NoXform());
   }
   fence_async_smem();
   __syncthreads();
   tc_fence_after();
   const uint32_t tG = tbase, tY = tbase + 128, tCH = tbase + 128 + P;
   if (t == 0) {
-    // G = C B^T (t x s), and C H_in (t x p)
 #pragma unroll
     for (int ks = 0; ks < kNP / 16; ks++) {
       const uint64_t dc = smem_desc(sC + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
       const uint64_t dbm = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
-      const uint64_t dh = smem_desc(sH + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
       mma_bf16(tG, dc, dbm, instr_desc(128, 128, 0, 0), ks > 0);
-      mma_bf16(tCH, dc, dh, instr_desc(128, P, 0, 1), ks > 0);
     }
     mma_commit(bar);
   }
   bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
-  tc_fence_after();
-  // G'[t][s] = G[t][s] e^{cum_t - cum_s} beta_s for s <= t, written over B as the A operand of
-  // the next product (row t, K = s, K-major); B is no longer read once the barrier fired
-  {
-    const uint32_t lane_addr = tmem_lane_addr(tbase);
-    const float ct = k.cum;
+  uint32_t phase = 0;  // of bar + 1, one completion per head
+  const uint32_t lane_addr = tmem_lane_addr(tbase);
+  for (int hi = 0; hi < HG; hi++) {
+    const int64_t h = hgrp * HG + hi, bh = b * p.H + h;
+    const float A = -expf(p.A_log[h]);
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+    const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);  // (synchronises the CTA)
+    cum_s[t] = k.cum;
+    beta_s[t] = k.beta;
+    {
+      const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
+      coop_tile<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid, NoXform());
+      const int64_t nrows = p.N;
+      coop_tile<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; }, NoXform());
+    }
+    __syncthreads();  // cum_s / beta_s of this head
+    tc_fence_after();
+    // G'[t][s] = G[t][s] e^{cum_t - cum_s} beta_s for s <= t -> the A operand of G' X
+    {
+      const float ct = k.cum;
 #pragma unroll 1
-    for (int s0 = 0; s0 < kQ; s0 += 32) {
-      float g[32];
-      tmem_ld32(lane_addr + s0, g);
+      for (int s0 = 0; s0 < kQ; s0 += 32) {
+        float g[32];
+        tmem_ld32(lane_addr + s0, g);
 #pragma unroll
-      for (int e = 0; e < 32; e += 8) {
-        float v[8];
+        for (int e = 0; e < 32; e += 8) {
+          float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-          const int s = s0 + e + j;
-          v[j] = (s <= t) ? g[e + j] * __expf(ct - cum_s[s]) * beta_s[s] : 0.f;
+          for (int j = 0; j < 8; j++) {
+            const int s = s0 + e + j;
+            v[j] = (s <= t) ? g[e + j] * __expf(ct - cum_s[s]) * beta_s[s] : 0.f;
+          }
+          uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, s0 + e)) = pk;
         }
-        uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-        *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, s0 + e)) = pk;
       }
     }
-  }
-  tc_fence_before();
-  fence_async_smem();
-  __syncthreads();
-  tc_fence_after();
-  if (t == 0) {
+    tc_fence_before();
+    fence_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
 #pragma unroll
-    for (int ks = 0; ks < kQ / 16; ks++) {
-      const uint64_t dg = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
-      const uint64_t dx = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
-      mma_bf16(tY, dg, dx, instr_desc(128, P, 0, 1), ks > 0);
+      for (int ks = 0; ks < kQ / 16; ks++) {
+        const uint64_t dg = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
+        const uint64_t dx = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+        const uint64_t dc = smem_desc(sC + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
+        const uint64_t dh = smem_desc(sH + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+        mma_bf16(tY, dg, dx, instr_desc(128, P, 0, 1), ks > 0);
+        mma_bf16(tCH, dc, dh, instr_desc(128, P, 0, 1), ks > 0);
+      }
+      mma_commit(bar + 1);
     }
-    mma_commit(bar + 1);
-  }
-  ok = __all_sync(0xffffffffu, mbar_wait(bar + 1, 0)) && ok;
-  tc_fence_after();
-  // y row t = G'X + e^{cum_t} C H_in (fp32) -> shared (padded rows, over the consumed tiles)
-  constexpr int SR = P + 4;
-  float *stage = reinterpret_cast<float *>(sC);
-  {
-    const uint32_t lane_addr = tmem_lane_addr(tbase);
-    const float et = __expf(k.cum);
+    ok = __all_sync(0xffffffffu, mbar_wait(bar + 1, phase)) && ok;
+    phase ^= 1u;
+    tc_fence_after();
+    // y row t = G'X + e^{cum_t} C H_in -> shared (padded) -> coalesced stores with + D x
+    constexpr int SR = P + 4;
+    {
+      const float et = __expf(k.cum);
 #pragma unroll 1
-    for (int q = 0; q < P; q += 32) {
-      float yv[32], cv[32];
-      tmem_ld32(lane_addr + 128 + q, yv);
-      tmem_ld32(lane_addr + 128 + P + q, cv);
+      for (int q = 0; q < P; q += 32) {
+        float yv[32], cv[32];
+        tmem_ld32(lane_addr + 128 + q, yv);
+        tmem_ld32(lane_addr + 128 + P + q, cv);
 #pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4 *>(stage + t * SR + q + j) =
-            make_float4(fmaf(et, cv[j], yv[j]), fmaf(et, cv[j + 1], yv[j + 1]),
-                        fmaf(et, cv[j + 2], yv[j + 2]), fmaf(et, cv[j + 3], yv[j + 3]));
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4 *>(stage + t * SR + q + j) =
+              make_float4(fmaf(et, cv[j], yv[j]), fmaf(et, cv[j + 1], yv[j + 1]),
+                          fmaf(et, cv[j + 2], yv[j + 2]), fmaf(et, cv[j + 3], yv[j + 3]));
+      }
     }
-  }
-  __syncthreads();
-  // coalesced: + D x (x from global), one rounding to the output type
-  if (ok) {
-    const float Dh = p.D ? p.D[h] : 0.f;
-    const int64_t rows_left = p.L - c * kQ;
-    const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
-    Tout *ys = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ) * P;
-    for (int i = t; i < kQ * P / 4; i += 128) {
-      const int r = i / (P / 4), q = (i % (P / 4)) * 4;
-      if (r >= rows_left) continue;
-      const float4 v = *reinterpret_cast<const float4 *>(stage + r * SR + q);
-      const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (int64_t)r * P + q);
-      const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
-      const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
-      const float o[4] = {fmaf(Dh, x01.x, v.x), fmaf(Dh, x01.y, v.y), fmaf(Dh, x23.x, v.z), fmaf(Dh, x23.y, v.w)};
-      VecStore<Tout, 4>::run(ys + (int64_t)r * P + q, o);
+    tc_fence_before();
+    __syncthreads();
+    if (ok) {
+      const float Dh = p.D ? p.D[h] : 0.f;
+      const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
+      Tout *ys = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ) * P;
+      for (int i = t; i < kQ * P / 4; i += 128) {
+        const int r = i / (P / 4), q = (i % (P / 4)) * 4;
+        if (r >= rows_left) continue;
+        const float4 v = *reinterpret_cast<const float4 *>(stage + r * SR + q);
+        const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (int64_t)r * P + q);
+        const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
+        const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
+        const float o[4] = {fmaf(Dh, x01.x, v.x), fmaf(Dh, x01.y, v.y), fmaf(Dh, x23.x, v.z), fmaf(Dh, x23.y, v.w)};
+        VecStore<Tout, 4>::run(ys + (int64_t)r * P + q, o);
+      }
     }
+    __syncthreads();  // the staged rows, G' and X are rewritten by the next head
   }
   if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
   tc_fence_before();
@@ -446,9 +454,10 @@ size_t ssd_smem_state(int P) {
   return kSsdHeader + (tiles > stage ? tiles : stage);
 }
 size_t ssd_smem_out(int P) {
+  // C, B / G', X, H_in; the staged result rows overlay G' and X (kQ x (P + 4) floats)
   const size_t tiles = (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2;
-  const size_t stage = (size_t)kQ * (P + 4) * 4;
-  return kSsdHeader + (tiles > stage ? tiles : stage);
+  const size_t stage_end = (size_t)kQ * kNP * 2 + (size_t)kQ * (P + 4) * 4;
+  return kSsdHeader + (tiles > stage_end ? tiles : stage_end);
 }
 
 template <int P, typename Tout>
@@ -464,7 +473,13 @@ static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H * (p.N * P / 1024)), 256, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ssd_out_kernel<P, Tout><<<(unsigned)grid, 128, s3, s>>>(p);
+  int HG = 1;  // heads per CTA: C, B and C B^T are shared by them
+  for (int cand : {8, 4, 2})
+    if (p.H % cand == 0) {
+      HG = cand;
+      break;
+    }
+  ssd_out_kernel<P, Tout><<<(unsigned)(grid / HG), 128, s3, s>>>(p, HG);
   return cudaGetLastError();
 }
 
