@@ -138,6 +138,24 @@ __device__ __forceinline__ void coop_tile(unsigned char *tile, const __nv_bfloat
 struct NoXform {
   __device__ __forceinline__ uint4 operator()(int, uint4 v) const { return v; }
 };
+// Same placement, copied asynchronously (cp.async, 16 bytes) with no transform; invalid rows are
+// zero-filled with plain stores. The caller commits, waits and fences before the tile is read.
+template <int R, int VPR, typename Off, typename Valid>
+__device__ __forceinline__ void coop_tile_async(unsigned char *tile, const __nv_bfloat16 *src,
+                                                int64_t rs, int vmax, Off smem_off, Valid valid) {
+  static_assert(R % 8 == 0 && (R * VPR) % 128 == 0, "tile shape");
+#pragma unroll 4
+  for (int it = 0; it < R * VPR / 128; it++) {
+    const int idx = it * 128 + threadIdx.x;
+    const int r8 = idx & 7, v = (idx >> 3) % VPR, rg = (idx >> 3) / VPR;
+    const int row = rg * 8 + r8;
+    unsigned char *dst = tile + smem_off(row, v);
+    if (valid(row) && v < vmax)
+      cp_async16(dst, src + (int64_t)row * rs + v * 8);
+    else
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
 
 // Delta, log a = Delta A and beta of step t of the chunk (0 past the sequence end: an identity
 // step), and the inclusive running sum of log a over the chunk (block-wide scan, 128 threads).
@@ -354,17 +372,19 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
   const uint32_t lane_addr = tmem_lane_addr(tbase);
   for (int hi = 0; hi < HG; hi++) {
     const int64_t h = hgrp * HG + hi, bh = b * p.H + h;
+    // this head's X and H_in tiles travel while the decays and G' are computed
+    {
+      const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
+      coop_tile_async<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid);
+      const int64_t nrows = p.N;
+      coop_tile_async<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; });
+      cp_async_commit();
+    }
     const float A = -expf(p.A_log[h]);
     const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
     const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);  // (synchronises the CTA)
     cum_s[t] = k.cum;
     beta_s[t] = k.beta;
-    {
-      const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
-      coop_tile<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid, NoXform());
-      const int64_t nrows = p.N;
-      coop_tile<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; }, NoXform());
-    }
     __syncthreads();  // cum_s / beta_s of this head
     tc_fence_after();
     // G'[t][s] = G[t][s] e^{cum_t - cum_s} beta_s for s <= t -> the A operand of G' X
@@ -387,6 +407,7 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
         }
       }
     }
+    cp_async_wait<0>();  // this thread's X / H_in copies landed
     tc_fence_before();
     fence_async_smem();
     __syncthreads();
