@@ -168,3 +168,42 @@ def test_split_backward_variants(case):
 
 def test_split_backward_long_few_channels():
     _bwd_case(1, 32, 16, 8192, "bf16", 16, carried=False)
+
+
+@pytest.mark.slow
+def test_full_few_channel_long_split_sampled():
+    """The split-L workload at full size (1 x 512 x 16 x 65536, bf16) in the benchmark's launch
+    configuration (automatic split), forward and backward, on sampled channels; dB / dC with a dout
+    that is zero outside the sampled channels, so every other channel contributes exactly zero."""
+    from gpu_helpers import assert_grad_close, channel_slice
+    w = wl.WORKLOADS["long_fewch_fwdbwd"]
+    a = wl.generate(w)
+    picks = wl.sample_channels(w.Bt, w.Dn, 6)
+    mask = np.zeros((w.Bt, w.Dn, 1), dtype=np.float32)
+    for b, d in picks:
+        mask[b, d] = 1.0
+    a["dout"] = a["dout"] * mask
+    t = dev_arrays(a, "bf16")
+    kw = param_kw(t)
+    r = ssm.ssm_scan_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], out_dtype=torch.float32,
+                         save_states=True, n_segments=-1, **kw)
+    g = ssm.ssm_scan_bwd(t["dout"], t["x"], t["dt"], t["A_log"], t["B"], t["C"],
+                         chunk_states=r["chunk_states"], n_segments=-1, **kw)
+    torch.cuda.synchronize()
+    out = to_np(r["out"])
+    got = {k: to_np(v) for k, v in g.items()}
+    dB_ref = np.zeros((w.Bt, w.N, w.L))
+    dC_ref = np.zeros((w.Bt, w.N, w.L))
+    for b, d in picks:
+        s = channel_slice(a, b, d)
+        ref = oracle.fwd(s["x"], s["dt"], s["A_log"], s["B"], s["C"], **oracle_kw(s))
+        assert_close("out (b=%d,d=%d)" % (b, d), out[b:b + 1, d:d + 1], ref, *TOL[("bf16", "f32")])
+        rg = oracle.bwd(s["x"], s["dt"], s["A_log"], s["B"], s["C"], s["dout"], **oracle_kw(s))
+        for k in ("dx", "ddt", "dz"):
+            assert_grad_close("%s (b=%d,d=%d)" % (k, b, d), got[k][b:b + 1, d:d + 1], rg[k])
+        for k in ("dA_log", "dD", "ddt_bias", "dconv_w", "dconv_b"):
+            assert_grad_close("%s (d=%d)" % (k, d), got[k][d:d + 1], rg[k])   # Bt = 1
+        dB_ref[b] += rg["dB"][0]
+        dC_ref[b] += rg["dC"][0]
+    assert_grad_close("dB (masked)", got["dB"], dB_ref)
+    assert_grad_close("dC (masked)", got["dC"], dC_ref)

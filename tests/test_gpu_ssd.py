@@ -97,3 +97,27 @@ def test_ssd_matches_selective_scan_for_one_channel_semantics():
     torch.cuda.synchronize()
     torch.testing.assert_close(y, y[..., :1].expand_as(y), rtol=1e-6, atol=1e-7)  # same per channel
     assert torch.equal(y2, 2 * y)     # exact: scaling by 2 commutes with every rounding on the way
+
+
+@pytest.mark.slow
+def test_full_ssd_layer_sampled_heads():
+    """The benchmarked SSD layer at full size (4 x 64 heads x 64 x 4096, N = 128, bf16 out), on
+    sampled (batch, head) pairs over the whole sequence, within the derived bound."""
+    cfg = wl.SSD_WORKLOADS["ssd_fwd"]
+    Bt, H, L, P, N = cfg["Bt"], cfg["H"], cfg["L"], cfg["P"], cfg["N"]
+    a = wl.generate_ssd(Bt, H, L, P, N, seed=cfg["seed"])
+    t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    y = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    y = y.float().cpu().numpy()
+    for (b, h) in wl.sample_channels(Bt, H, 8):
+        sl = dict(x=a["x"][b:b + 1, h:h + 1], dt=a["dt"][b:b + 1, h:h + 1], B=a["B"][b:b + 1],
+                  C=a["C"][b:b + 1], A_log=a["A_log"][h:h + 1], D=a["D"][h:h + 1],
+                  dt_bias=a["dt_bias"][h:h + 1])
+        ref = oracle.ssd_fwd(sl["x"], sl["dt"], sl["A_log"], sl["B"], sl["C"], D=sl["D"], dt_bias=sl["dt_bias"])
+        yabs = oracle.ssd_fwd(np.abs(sl["x"]), sl["dt"], sl["A_log"], np.abs(sl["B"]), np.abs(sl["C"]),
+                              D=np.abs(sl["D"]), dt_bias=sl["dt_bias"])
+        got = y[b:b + 1, h:h + 1]
+        tol = 2.0 ** -6 * yabs + 2.0 ** -8 * np.abs(ref) + 1e-6
+        assert np.all(np.abs(got - ref) <= tol), "head (%d, %d): worst excess %g" % (b, h, (np.abs(got - ref) - tol).max())
