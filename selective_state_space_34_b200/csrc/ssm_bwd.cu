@@ -697,21 +697,22 @@ __global__ void reduce_params_kernel(const BwdParams P) {
 // Split-L pass 1: for every segment but the first, the adjoint run backwards from a zero arrival
 // -- lambda_t = dy_t C_t + A_bar_{t+1} lambda_{t+1} over [ts, te) -- needs only Delta, dy and C
 // (no state recompute). Keeps A_bar_ts lambda_ts (what the segment hands to the one before it
-// when nothing arrives) and the sum of Delta. One thread per (segment, b, d, group of 4 states).
-template <typename Tin>
+// when nothing arrives) and the sum of Delta. One thread per (segment, b, d, group of SG states);
+// the sequence is walked in 8-step blocks read as 16-byte vectors when rows are aligned.
+template <typename Tin, int SG>
 __global__ void seg_adjoint_kernel(const BwdParams P) {
   constexpr bool PRECISE = sizeof(Tin) == 4;
   const FwdParams &p = P.f;
-  const int64_t L = p.L, N = p.N, NQ = (N + 3) / 4, BD = p.Bt * p.Dn;
+  const int64_t L = p.L, N = p.N, NQ = (N + SG - 1) / SG, BD = p.Bt * p.Dn;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)(P.n_seg - 1) * BD * NQ) return;
   const int64_t q = i % NQ, sb = i / NQ, bd = sb % BD, seg = 1 + sb / BD;
   const int64_t b = bd / p.Dn, d = bd % p.Dn;
   const int64_t ts = seg * P.seg_len, te = imin64(L, ts + P.seg_len);
-  float A[4], Ac[4], lam[4], an[4];
+  float A[SG], Ac[SG], lam[SG], an[SG];
 #pragma unroll
-  for (int j = 0; j < 4; j++) {
-    const int64_t n = 4 * q + j;
+  for (int j = 0; j < SG; j++) {
+    const int64_t n = SG * q + j;
     A[j] = n < N ? -expf(p.A_log[d * N + n]) : 0.f;
     Ac[j] = PRECISE ? A[j] : A[j] * kLog2e;
     lam[j] = 0.f;
@@ -721,30 +722,71 @@ __global__ void seg_adjoint_kernel(const BwdParams P) {
   const Tin *dtr = static_cast<const Tin *>(p.dt) + bd * L;
   const Tin *zr = p.z ? static_cast<const Tin *>(p.z) + bd * L : nullptr;
   const Tin *dor = static_cast<const Tin *>(P.dout) + bd * L;
-  const Tin *Cb = static_cast<const Tin *>(p.C) + b * N * L;
+  const Tin *Cb = static_cast<const Tin *>(p.C) + (b * N + SG * q) * L;
+  const int nv = (int)imin64(SG, N - SG * q);  // valid states of this group
   float sdl = 0.f;
-  for (int64_t t = te - 1; t >= ts; t--) {
-    const float v = to_f32(dtr[t]) + dtb;
+  // one step t with the group's C_t values in cv
+  auto step = [&](float dtv, float zv, float dov, const float *cv) {
+    const float v = dtv + dtb;
     const float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
-    float dy = to_f32(dor[t]);
-    if (zr) {
-      const float zz = to_f32(zr[t]);
-      dy *= zz * sigmoid<PRECISE>(zz);
-    }
+    float dy = dov;
+    if (zr) dy *= zv * sigmoid<PRECISE>(zv);
     sdl += dl;
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const int64_t n = 4 * q + j;
-      if (n < N) {
-        lam[j] = fmaf(an[j], lam[j], dy * to_f32(Cb[n * L + t]));
-        an[j] = PRECISE ? expf(dl * A[j]) : ex2_approx(dl * Ac[j]);
+    for (int j = 0; j < SG; j++) {
+      lam[j] = fmaf(an[j], lam[j], dy * cv[j]);
+      an[j] = PRECISE ? expf(dl * A[j]) : ex2_approx(dl * Ac[j]);
+    }
+  };
+  int64_t t = te - 1;
+  // the ragged end first (te - ts need not be a multiple of 8), one step at a time
+  for (int64_t k = 0; k < (te - ts) % 8; k++, t--) {
+    float cv[SG];
+#pragma unroll
+    for (int j = 0; j < SG; j++) cv[j] = j < nv ? to_f32(Cb[(int64_t)j * L + t]) : 0.f;
+    step(to_f32(dtr[t]), zr ? to_f32(zr[t]) : 0.f, to_f32(dor[t]), cv);
+  }
+  // then whole 8-step blocks [t - 7, t], ts a multiple of 64 so t - 7 is a multiple of 8
+  for (; t >= ts; t -= 8) {
+    const int64_t t0 = t - 7;
+    float dtw[8], zw[8], dow[8], cw[SG][8];
+    if (p.vec) {
+      load_window<Tin, 8>(dtw, dtr + t0);
+      load_window<Tin, 8>(dow, dor + t0);
+      if (zr) load_window<Tin, 8>(zw, zr + t0);
+#pragma unroll
+      for (int j = 0; j < SG; j++) {
+        if (j < nv)
+          load_window<Tin, 8>(cw[j], Cb + (int64_t)j * L + t0);
+        else
+#pragma unroll
+          for (int e = 0; e < 8; e++) cw[j][e] = 0.f;
       }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        dtw[e] = to_f32(dtr[t0 + e]);
+        dow[e] = to_f32(dor[t0 + e]);
+        zw[e] = zr ? to_f32(zr[t0 + e]) : 0.f;
+#pragma unroll
+        for (int j = 0; j < SG; j++) cw[j][e] = j < nv ? to_f32(Cb[(int64_t)j * L + t0 + e]) : 0.f;
+      }
+    }
+    if (!zr)
+#pragma unroll
+      for (int e = 0; e < 8; e++) zw[e] = 0.f;
+#pragma unroll
+    for (int e = 7; e >= 0; e--) {
+      float cv[SG];
+#pragma unroll
+      for (int j = 0; j < SG; j++) cv[j] = cw[j][e];
+      step(dtw[e], zw[e], dow[e], cv);
     }
   }
   const int64_t row = (seg * BD + bd) * N;
 #pragma unroll
-  for (int j = 0; j < 4; j++)
-    if (4 * q + j < N) P.seg_gloc[row + 4 * q + j] = an[j] * lam[j];
+  for (int j = 0; j < SG; j++)
+    if (j < nv) P.seg_gloc[row + SG * q + j] = an[j] * lam[j];
   if (q == 0) P.seg_sdl[seg * BD + bd] = sdl;
 }
 
@@ -849,11 +891,12 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
   const LaneLayout lay = choose_layout(P.f.N, P.f.Bt * P.f.Dn * P.n_seg);
   if (P.n_seg > 1) {
     // split-L passes 1 and 2: what arrives at each segment's last state
-    const int64_t n1 = (int64_t)(P.n_seg - 1) * P.f.Bt * P.f.Dn * ((P.f.N + 3) / 4);
+    constexpr int SG = 8;  // states per thread
+    const int64_t n1 = (int64_t)(P.n_seg - 1) * P.f.Bt * P.f.Dn * ((P.f.N + SG - 1) / SG);
     if (in_bf16)
-      seg_adjoint_kernel<__nv_bfloat16><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
+      seg_adjoint_kernel<__nv_bfloat16, SG><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
     else
-      seg_adjoint_kernel<float><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
+      seg_adjoint_kernel<float, SG><<<(unsigned)((n1 + 127) / 128), 128, 0, stream>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t bdn = P.f.Bt * P.f.Dn * P.f.N;
