@@ -207,3 +207,15 @@ def test_full_few_channel_long_split_sampled():
         dC_ref[b] += rg["dC"][0]
     assert_grad_close("dB (masked)", got["dB"], dB_ref)
     assert_grad_close("dC (masked)", got["dC"], dC_ref)
+
+
+def test_split_backward_deterministic():
+    w = wl.shaped("mamba130m_fwd", Bt=1, Dn=32, N=16, L=2048, backward=True)
+    a = wl.generate(w)
+    t = dev_arrays(a, "bf16")
+    kw = param_kw(t)
+    g1 = ssm.ssm_scan_bwd(t["dout"], t["x"], t["dt"], t["A_log"], t["B"], t["C"], n_segments=8, **kw)
+    g2 = ssm.ssm_scan_bwd(t["dout"], t["x"], t["dt"], t["A_log"], t["B"], t["C"], n_segments=8, **kw)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k

@@ -121,3 +121,21 @@ def test_full_ssd_layer_sampled_heads():
         got = y[b:b + 1, h:h + 1]
         tol = 2.0 ** -6 * yabs + 2.0 ** -8 * np.abs(ref) + 1e-6
         assert np.all(np.abs(got - ref) <= tol), "head (%d, %d): worst excess %g" % (b, h, (np.abs(got - ref) - tol).max())
+
+
+def test_ssd_deterministic_and_empty():
+    a = wl.generate_ssd(2, 8, 300, 64, 128, seed=11)
+    t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    kw = dict(D=t["D"], dt_bias=t["dt_bias"], return_state=True)
+    y1, h1 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], **kw)
+    y2, h2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(h1, h2)   # no atomics: bitwise run to run
+    # an empty sequence hands the state through
+    h0 = torch.randn(2, 8, 128, 64, device="cuda")
+    e = lambda v, shape: torch.empty(shape, dtype=v.dtype, device="cuda")
+    y0, hl = ssm.ssm_ssd_fwd(e(t["x"], (2, 8, 0, 64)), e(t["dt"], (2, 8, 0)), t["A_log"],
+                             e(t["B"], (2, 0, 128)), e(t["C"], (2, 0, 128)), h0=h0, **kw)
+    torch.cuda.synchronize()
+    assert y0.numel() == 0 and torch.equal(hl, h0)
