@@ -1,6 +1,7 @@
 // ssm_api.cu -- the extern "C" boundary declared in include/ssm_scan.h: host-side validation
-// (synchronous, before any launch) and dispatch to the kernel launchers. No exception crosses the
-// ABI and the library allocates no device memory.
+// (synchronous, before any launch), workspace carving, and dispatch to the kernel launchers. No
+// exception crosses the ABI and these entry points allocate no device memory (scratch comes from
+// the caller's workspace; ssm_noalloc.cu is the one entry point with a library-owned array).
 #include <stdint.h>
 #include <string.h>
 

@@ -5,7 +5,7 @@
 // "Sequence and state-space models", state_space_models).
 //
 // Work decomposition. One CTA owns CH = 128 / G channels of one batch element and walks the whole
-// sequence in stages of kT time steps. Inside a warp, the G lanes of a channel each hold NS of its
+// sequence (or, with split-L, one segment of it) in stages of kT time steps. Inside a warp, the G lanes of a channel each hold NS of its
 // states in fp32 registers and run the recurrence sequentially in time; B_t and C_t are shared by
 // all channels, so every lane reads them as shared-memory broadcasts. Per-element work (conv,
 // SiLU, softplus, gate, the D skip and the store) is split over the G lanes of a channel so that
