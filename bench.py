@@ -532,7 +532,7 @@ def main():
             if k in T2:
                 setattr(ba2.fwd, k, T2[k].data_ptr())
         ba2.dout = T2["dout"].data_ptr()
-    sets = [(T, fwd_args, bw_args), (T2, fa2, ba2)]
+    sets = [(T, fwd_args, bw_args if backward else None), (T2, fa2, ba2)]
     h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_ready, ev_free, ev_comp, ev_back = [E(), E()], [E(), E()], E(), E()
 

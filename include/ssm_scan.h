@@ -133,8 +133,8 @@ typedef struct ssm_fwd_args {
    * the forward's only). */
   int32_t n_segments;    /* 0 or 1: one pass. >= 2: up to that many segments, each a multiple of
                             64 steps long. -1: chosen from the current device's SM count and the
-                            shape (one pass unless even 8 channels per CTA leave fewer than two
-                            CTAs per SM). */
+                            shape (one pass when the one-pass grid fills the SMs once; else enough
+                            segments for one wave (very few channels) or about two). */
   void *workspace;       /* device scratch of at least ssm_fwd_workspace_size() bytes, 256-byte
                             aligned, when the call splits L; may be NULL otherwise */
   size_t workspace_bytes;

@@ -454,13 +454,19 @@ SegPlan plan_segments(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int requeste
   constexpr int64_t kSegAlign = 64;  // a multiple of the stage and of the state chunk
   int64_t want = requested;
   if (requested < 0) {
-    // automatic: split only when even the widest lane layout leaves the SMs short of CTAs, then
-    // aim the 4-lane layout's CTAs x segments at one wave of 4 CTAs per SM, with segments of at
-    // least 1024 steps
-    const int64_t widest = Bt * ((Dn + 7) / 8);
-    if (widest >= 2 * (int64_t)sm_count) return plan;
+    // automatic, from measurements on B200 (4 CTAs per SM): the one-pass 4-lane grid has
+    // base = Bt ceil(Dn / 32) CTAs. From three quarters of a wave up, no split. When even the widest lane
+    // layout leaves fewer than two CTAs per SM, aim the segments at one wave (1x512x16x65536:
+    // 37 segments, 7.1x); otherwise at about 2.2 waves (1x5120x16x65536: 8 segments, -10%;
+    // 2x1536x16x2048: 4-8 segments, -12 to -16%). Segments of at least 1024 resp. 256 steps.
+    const int64_t slots = 4 * (int64_t)sm_count;
     const int64_t base = Bt * ((Dn + 31) / 32);
-    want = imin64(4 * (int64_t)sm_count / (base > 0 ? base : 1), L / 1024);
+    if (4 * base >= 3 * slots) return plan;  // three quarters of a wave or more (1.4B shape: 86%)
+    const int64_t widest = Bt * ((Dn + 7) / 8);
+    if (widest < 2 * (int64_t)sm_count)
+      want = imin64(slots / (base > 0 ? base : 1), L / 1024);
+    else
+      want = imin64((22 * slots / (base > 0 ? base : 1) + 5) / 10, L / 256);
   }
   if (want < 2 || L < 2 * kSegAlign) return plan;
   int64_t len = (L + want - 1) / want;

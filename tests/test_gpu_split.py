@@ -95,8 +95,8 @@ def test_split_bf16_output_and_auto():
     from selective_state_space_34_b200 import _abi
     args.n_segments = -1
     assert _abi.load().ssm_fwd_workspace_size(ctypes.byref(args)) > 0   # it splits
-    args.Dn = 8192
-    assert _abi.load().ssm_fwd_workspace_size(ctypes.byref(args)) == 0  # enough channels
+    args.Dn = 32768
+    assert _abi.load().ssm_fwd_workspace_size(ctypes.byref(args)) == 0  # a full wave without it
 
 
 def test_long_few_channels_sampled():
