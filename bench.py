@@ -170,6 +170,49 @@ class ClockSampler:
 
 # ---- CPU baseline: the float64 oracle on a bounded sample of the same workload ------------------
 
+def _channel_slice(a, b, lo, hi):
+    """Inputs of channels lo..hi-1 of batch element b (the oracle runs channels independently;
+    B and C are the batch element's own)."""
+    sl = slice(lo, hi)
+    kw = dict(D=a["D"][sl], z=None if a["z"] is None else a["z"][b:b + 1, sl],
+              dt_bias=a["dt_bias"][sl], conv_w=None if a["conv_w"] is None else a["conv_w"][sl],
+              conv_b=None if a["conv_b"] is None else a["conv_b"][sl])
+    dout = a["dout"][b:b + 1, sl] if a.get("dout") is not None else None
+    return (a["x"][b:b + 1, sl], a["dt"][b:b + 1, sl], a["A_log"][sl], a["B"][b:b + 1],
+            a["C"][b:b + 1], dout, kw)
+
+
+def oracle_parity(w, a, picks, out_bf16):
+    """Errors of the benchmarked kernels' own results on sampled channels against the oracle, with
+    the parity tests' tolerances: output rtol 2e-3 (+2^-8 for a bf16 output), atol 1e-4 for bf16
+    inputs (1e-5 / 1e-6 for fp32); dx rtol 1e-2, atol 1e-4 max|dx_ref|. tol_ratio <= 1 passes."""
+    import oracle
+    rtol, atol = (2e-3, 1e-4) if w.in_dtype == "bf16" else (1e-5, 1e-6)
+    if out_bf16:
+        rtol += 2.0 ** -8
+    res = {"channels": ["b%d:d%d-%d" % (b, d, d + g.shape[0]) for b, d, g, _ in picks]}
+
+    def stats(name, got, ref, rt, at):
+        err = np.abs(got - ref)
+        big = np.abs(ref) > 1e-3 * max(np.abs(ref).max(), 1e-30)
+        res[name] = {"max_abs_err": float(err.max()),
+                     "max_rel_err": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+                     "tol_ratio": float((err / (at + rt * np.abs(ref))).max())}
+
+    outs, dxs = [], []
+    for b, d, g_out, g_dx in picks:
+        x, dt, Al, B, C, dout, kw = _channel_slice(a, b, d, d + g_out.shape[0])
+        outs.append((g_out, oracle.fwd(x, dt, Al, B, C, n_threads=1, **kw)[0]))
+        if g_dx is not None:
+            dxs.append((g_dx, oracle.bwd(x, dt, Al, B, C, dout, n_threads=1, **kw)["dx"][0]))
+    stats("out", np.concatenate([o[0] for o in outs]), np.concatenate([o[1] for o in outs]), rtol, atol)
+    if dxs:
+        ref = np.concatenate([o[1] for o in dxs])
+        stats("dx", np.concatenate([o[0] for o in dxs]), ref, 1e-2, 1e-4 * np.abs(ref).max())
+    res["ok"] = all(v["tol_ratio"] <= 1.0 for k, v in res.items() if isinstance(v, dict))
+    return res
+
+
 def oracle_sample(w, a, n_channels, threads):
     """Run the oracle's forward + backward on n_channels channels of the workload, spread over a
     thread pool (the C oracle releases the GIL); returns (seconds, elem_states)."""
@@ -187,15 +230,10 @@ def oracle_sample(w, a, n_channels, threads):
 
     def run(group):
         b, lo, hi = group
-        sl = slice(lo, hi)
-        kw = dict(D=a["D"][sl], z=None if a["z"] is None else a["z"][b:b + 1, sl],
-                  dt_bias=a["dt_bias"][sl], conv_w=None if a["conv_w"] is None else a["conv_w"][sl],
-                  conv_b=None if a["conv_b"] is None else a["conv_b"][sl])
-        x, dt = a["x"][b:b + 1, sl], a["dt"][b:b + 1, sl]
-        B, C, Al = a["B"][b:b + 1], a["C"][b:b + 1], a["A_log"][sl]
+        x, dt, Al, B, C, dout, kw = _channel_slice(a, b, lo, hi)
         oracle.fwd(x, dt, Al, B, C, n_threads=1, **kw)
         if w.backward:
-            oracle.bwd(x, dt, Al, B, C, a["dout"][b:b + 1, sl], n_threads=1, **kw)
+            oracle.bwd(x, dt, Al, B, C, dout, n_threads=1, **kw)
         return (hi - lo) * w.L * w.N
 
     oracle.build()
@@ -449,6 +487,17 @@ def main():
     ms_step = max_ms / args.steps
     value = job_throughput(es, world, args.steps, max_ms)
 
+    step_end = ev_b1 if backward else ev_f1
+    per_step = np.array([ev_f0[i].elapsed_time(step_end[i]) for i in range(args.steps)])
+    step_dist = {"median": float(np.median(per_step)), "p10": float(np.percentile(per_step, 10)),
+                 "p90": float(np.percentile(per_step, 90)),
+                 "of": "rank 0, CUDA events around each timed step"}
+    # the timed steps' own results on a few sampled channels, for the parity check below
+    picks = []
+    for i in range(4):
+        b, d = i % Bt, (i * 997) % max(1, Dn - 4)
+        picks.append((b, d, out[b, d:d + 4].float().cpu().numpy(),
+                      grads["dx"][b, d:d + 4].cpu().numpy() if backward else None))
     fwd_ms = float(np.mean([ev_f0[i].elapsed_time(ev_f1[i]) for i in range(args.steps)]))
     kern = {"ssm_fwd_kernel": fwd_ms}
     if backward:
@@ -590,12 +639,14 @@ def main():
         secs, done = oracle_sample(w, a, n_ch, threads)
         cpu = {"value": done / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": "%d channels (wrapping over the %d of the workload) x L=%d x N=%d (fwd%s), "
-                         "float64, %.1f s" % (n_ch, w.Bt * w.Dn, L, N, "+bwd" if backward else "", secs)}
+                         "float64, %.1f s" % (n_ch, w.Bt * w.Dn, L, N, "+bwd" if backward else "", secs),
+               "parity": oracle_parity(w, a, picks, odt == torch.bfloat16)}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": ms_step, "step_ms": step_dist,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "Bt": Bt, "Dn": Dn, "N": N, "L": L,
                        "in_dtype": w.in_dtype, "out_dtype": args.out_dtype,

@@ -63,7 +63,8 @@ typedef enum ssm_status {
   SSM_ERR_UNSUPPORTED = 5, /* d_state > 64 or K > 4 */
   SSM_ERR_CUDA = 6,        /* a CUDA call or launch failed; see ssm_last_cuda_error() */
   SSM_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssm_*_workspace_size() */
-  SSM_ERR_TIMEOUT = 8      /* reserved for bounded device-side waits; not returned today */
+  SSM_ERR_TIMEOUT = 8      /* a bounded device-side wait ran out (ssm_ssd_check,
+                              ssm_wait_selftest); the CUDA context stays usable */
 } ssm_status;
 
 typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
@@ -196,6 +197,25 @@ size_t ssm_ssd_workspace_size(const ssm_ssd_args *args);
  * SSM_ERR_DTYPE (codes), SSM_ERR_UNSUPPORTED (in_dtype not bf16, P not 64/128, N not 64/128),
  * SSM_ERR_WORKSPACE, SSM_ERR_CUDA. Bt = 0 or L = 0: nothing to do (h_last = h0 or 0). */
 ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream);
+
+/* Failure detection for ssm_ssd_fwd. Its kernels wait for every tensor-core product through an
+ * mbarrier, polling a bounded number of times (2^18, about one second on B200, where a failed poll
+ * takes about 4 us); a wait that runs out sets an error word in
+ * the workspace (zeroed at the start of every ssm_ssd_fwd), and the kernel still releases its
+ * tensor memory and exits, so the context stays usable. This call SYNCHRONISES `stream`, reads the
+ * word of the latest ssm_ssd_fwd that used args->workspace, and returns SSM_ERR_TIMEOUT when it is
+ * set, SSM_OK otherwise. Same argument checks as ssm_ssd_fwd (plus SSM_ERR_WORKSPACE); SSM_ERR_CUDA
+ * when the copy or the synchronisation fails. */
+ssm_status ssm_ssd_check(const ssm_ssd_args *args, void *stream);
+
+/* Self-test of that timeout path on the current device: one CTA of 128 threads waits, polling at
+ * most `polls` times (1..2^22), on a shared-memory mbarrier that expects one arrival. With arrive
+ * != 0 one thread arrives first and the wait succeeds (SSM_OK); with arrive = 0 nothing arrives, the
+ * wait runs out and the kernel sets *error_word (device int32, 4-byte aligned, zeroed here first)
+ * through the same bounded wait the SSD kernels use; the call then returns SSM_ERR_TIMEOUT.
+ * Synchronises `stream`. Errors: SSM_ERR_NULL, SSM_ERR_ALIGN, SSM_ERR_SHAPE (polls out of range),
+ * SSM_ERR_CUDA. */
+ssm_status ssm_wait_selftest(int32_t arrive, int32_t polls, int32_t *error_word, void *stream);
 
 /* Bytes of workspace ssm_scan_fwd needs for these arguments: 0 when the call runs in one pass
  * (n_segments 0 or 1, or a split that would leave a single segment), else 2 (n Bt Dn N) + n Bt Dn

@@ -18,7 +18,7 @@ parameters are fp32.
 from __future__ import annotations
 
 from .api import (ssm_conv1d_silu, ssm_scan_bwd, ssm_scan_fwd, ssm_scan_step, ssm_ssd_fwd,
-                  ssm_bwd_workspace_size, ssm_num_state_chunks)
+                  ssm_bwd_workspace_size, ssm_num_state_chunks, ssm_wait_selftest)
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_step", "ssm_ssd_fwd", "ssm_conv1d_silu",
-           "ssm_bwd_workspace_size", "ssm_num_state_chunks"]
+           "ssm_bwd_workspace_size", "ssm_num_state_chunks", "ssm_wait_selftest"]

@@ -12,6 +12,7 @@ SSM_F32, SSM_BF16 = 0, 1
 SSM_ZOH, SSM_EULER = 0, 1
 SSM_STATE_CHUNK = 16
 SSM_NOALLOC_SCRATCH_BYTES = 64 << 20
+SSM_ERR_TIMEOUT = 8
 
 STATUS = {
     0: "SSM_OK", 1: "SSM_ERR_NULL", 2: "SSM_ERR_SHAPE", 3: "SSM_ERR_ALIGN", 4: "SSM_ERR_DTYPE",
@@ -61,7 +62,6 @@ class StepArgs(ctypes.Structure):
     ]
 
 
-# (name, restype, argtypes) of every exported function in include/ssm_scan.h
 class SsdArgs(ctypes.Structure):
     _fields_ = [
         ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
@@ -76,6 +76,7 @@ class SsdArgs(ctypes.Structure):
     ]
 
 
+# (name, restype, argtypes) of every exported function in include/ssm_scan.h
 SIGNATURES = [
     ("ssm_num_state_chunks", ctypes.c_int64, [ctypes.c_int64]),
     ("ssm_scan_fwd", ctypes.c_int, [ctypes.POINTER(FwdArgs), ctypes.c_void_p]),
@@ -86,6 +87,8 @@ SIGNATURES = [
     ("ssm_scan_step", ctypes.c_int, [ctypes.POINTER(StepArgs), ctypes.c_void_p]),
     ("ssm_ssd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(SsdArgs)]),
     ("ssm_ssd_fwd", ctypes.c_int, [ctypes.POINTER(SsdArgs), ctypes.c_void_p]),
+    ("ssm_ssd_check", ctypes.c_int, [ctypes.POINTER(SsdArgs), ctypes.c_void_p]),
+    ("ssm_wait_selftest", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     ("ssm_conv1d_silu", ctypes.c_int,
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
       ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,

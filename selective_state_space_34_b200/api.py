@@ -299,10 +299,13 @@ def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = 
 
 
 def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplus: bool = True,
-                out_dtype=None, discretization: str = "zoh", return_state: bool = False):
+                out_dtype=None, discretization: str = "zoh", return_state: bool = False,
+                check: bool = False):
     """Mamba-2 state-space duality forward. x: (Bt, H, L, P) bf16; dt: (Bt, H, L) bf16; B, C:
     (Bt, L, N) bf16 shared by the heads; A_log, D, dt_bias: (H,) fp32; h0: (Bt, H, N, P) fp32.
-    P and N must be 64 or 128. Returns y (Bt, H, L, P), or (y, h_last) with return_state."""
+    P and N must be 64 or 128. Returns y (Bt, H, L, P), or (y, h_last) with return_state.
+    check=True synchronises the stream afterwards and raises SSMError (code SSM_ERR_TIMEOUT) if a
+    bounded wait for the tensor cores ran out."""
     for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
         _need_cuda(n, t)
     for n, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
@@ -336,4 +339,22 @@ def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplu
         a.workspace = (ws.data_ptr() + 255) & ~255
         a.workspace_bytes = need
     _abi.check("ssm_ssd_fwd", lib.ssm_ssd_fwd(ctypes.byref(a), _stream_handle(x.device)))
+    if check:
+        _abi.check("ssm_ssd_check", lib.ssm_ssd_check(ctypes.byref(a), _stream_handle(x.device)))
     return (y, hl) if return_state else y
+
+
+def ssm_wait_selftest(arrive: bool, polls: int = 4096, device=None) -> bool:
+    """Run the bounded-wait self-test on a CUDA device: one CTA waits, at most `polls` times, on an
+    mbarrier that receives its arrival only when `arrive` is true. Returns True when the wait
+    completed and False when it ran out (the library answered SSM_ERR_TIMEOUT); any other failure
+    raises SSMError. Synchronises the device's current stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if dev.type != "cuda":
+        raise ValueError("ssm_wait_selftest needs a CUDA device")
+    word = torch.empty(1, dtype=torch.int32, device=dev)
+    code = _abi.load().ssm_wait_selftest(1 if arrive else 0, int(polls), _ptr(word), _stream_handle(dev))
+    if code == _abi.SSM_ERR_TIMEOUT:
+        return False
+    _abi.check("ssm_wait_selftest", code)
+    return True

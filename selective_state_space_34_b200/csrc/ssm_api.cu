@@ -5,10 +5,21 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/ssm_scan.h"
 #include "ssm_internal.h"
 
 namespace {
+
+// An NVTX range named after the entry point around its host work and launches, so a profiler's
+// timeline groups each call's kernels under the API call that issued them. Header-only NVTX v3:
+// without an attached tool a push or pop is one predictable branch.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define SSM_RANGE(name) NvtxRange ssm_nvtx_range_(name)
 
 thread_local int g_last_cuda_error = 0;
 
@@ -165,6 +176,7 @@ const char *ssm_status_string(ssm_status s) {
 int ssm_last_cuda_error(void) { return g_last_cuda_error; }
 
 ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream) {
+  SSM_RANGE("ssm_scan_fwd");
   bool empty = false;
   ssm_status st = check_fwd(args, true, &empty);
   if (st != SSM_OK) return st;
@@ -198,6 +210,7 @@ size_t ssm_fwd_workspace_size(const ssm_fwd_args *args) {
 ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
                            int64_t Dn, int64_t L, int32_t K, int32_t in_dtype, int32_t out_dtype,
                            void *stream) {
+  SSM_RANGE("ssm_conv1d_silu");
   if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return SSM_ERR_DTYPE;
   if (Bt < 0 || Dn < 0 || L < 0) return SSM_ERR_SHAPE;
   if (Dn == 0 || K <= 0) return SSM_ERR_SHAPE;
@@ -216,6 +229,7 @@ ssm_status ssm_conv1d_silu(const void *x, void *u, const float *w, const float *
 }
 
 ssm_status ssm_scan_step(const ssm_step_args *a, void *stream) {
+  SSM_RANGE("ssm_scan_step");
   if (!a) return SSM_ERR_NULL;
   if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
   if (a->discretization != SSM_ZOH && a->discretization != SSM_EULER) return SSM_ERR_UNSUPPORTED;
@@ -269,6 +283,7 @@ size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {
 }
 
 ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
+  SSM_RANGE("ssm_scan_bwd");
   if (!args) return SSM_ERR_NULL;
   bool empty = false;
   ssm_status st = check_fwd(&args->fwd, false, &empty);
@@ -366,6 +381,8 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   return cuda_status(ssm::launch_bwd(p, a->in_dtype == SSM_BF16, static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
 namespace {
 ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {
   if (!a) return SSM_ERR_NULL;
@@ -392,7 +409,18 @@ ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {
   if ((a->h0 && !aligned(a->h0, 16)) || (a->h_last && !aligned(a->h_last, 16))) return SSM_ERR_ALIGN;
   return SSM_OK;
 }
+
+// Synchronise `s`, then read a device error word: non-zero means a bounded wait ran out.
+ssm_status read_error_word(const void *word, cudaStream_t s) {
+  int32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, word, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return host ? SSM_ERR_TIMEOUT : SSM_OK;
+}
 }  // namespace
+
+extern "C" {
 
 size_t ssm_ssd_workspace_size(const ssm_ssd_args *args) {
   bool empty = false;
@@ -401,6 +429,7 @@ size_t ssm_ssd_workspace_size(const ssm_ssd_args *args) {
 }
 
 ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream) {
+  SSM_RANGE("ssm_ssd_fwd");
   bool empty = false;
   ssm_status st = check_ssd(args, &empty);
   if (st != SSM_OK) return st;
@@ -446,10 +475,37 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream) {
   w += rnd(sizeof(__nv_bfloat16) * chunks * np);
   p.cum_end = reinterpret_cast<float *>(w);
   w += rnd(sizeof(float) * chunks);
-  p.error = reinterpret_cast<int *>(w);
+  p.error = reinterpret_cast<int *>(static_cast<char *>(args->workspace) +
+                                     ssm::ssd_error_offset(args->Bt, args->H, args->L, args->P, args->N));
   cudaError_t e = cudaMemsetAsync(p.error, 0, sizeof(int), s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(ssm::launch_ssd(p, args->out_dtype == SSM_BF16, s));
+}
+
+ssm_status ssm_ssd_check(const ssm_ssd_args *args, void *stream) {
+  SSM_RANGE("ssm_ssd_check");
+  bool empty = false;
+  ssm_status st = check_ssd(args, &empty);
+  if (st != SSM_OK) return st;
+  if (empty) return SSM_OK;  // nothing ran, nothing to report
+  if (!args->workspace || !aligned(args->workspace, 256) ||
+      args->workspace_bytes < ssm::ssd_workspace_bytes(args->Bt, args->H, args->L, args->P, args->N))
+    return SSM_ERR_WORKSPACE;
+  return read_error_word(static_cast<const char *>(args->workspace) +
+                             ssm::ssd_error_offset(args->Bt, args->H, args->L, args->P, args->N),
+                         static_cast<cudaStream_t>(stream));
+}
+
+ssm_status ssm_wait_selftest(int32_t arrive, int32_t polls, int32_t *error_word, void *stream) {
+  SSM_RANGE("ssm_wait_selftest");
+  if (!error_word) return SSM_ERR_NULL;
+  if (!aligned(error_word, 4)) return SSM_ERR_ALIGN;
+  if (polls < 1 || polls > (1 << 22)) return SSM_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(error_word, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = ssm::launch_wait_selftest(arrive ? 1 : 0, polls, error_word, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return read_error_word(error_word, s);
 }
 
 }  // extern "C"

@@ -60,6 +60,10 @@ struct SsdParams {
 };
 cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream);
 size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);
+// Byte offset of the SSD error word inside the workspace (its last 256-byte block).
+size_t ssd_error_offset(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);
+// One CTA waiting, with a bound of `polls`, on an mbarrier that gets one arrival iff `arrive`.
+cudaError_t launch_wait_selftest(int arrive, int polls, int *error, cudaStream_t stream);
 
 // Segmentation of a split-L forward: how many segments of which length, and the scratch it needs.
 struct SegPlan {

@@ -63,11 +63,14 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");  // visible to the async proxy
 }
 
-// Wait for the phase with parity `phase`; gives up after ~2^22 polls. Returns false on timeout.
-// The result is made warp-uniform by the caller before any warp-collective tcgen05 access.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase) {
+// Wait for the phase with parity `phase`; gives up after max_polls polls. Returns false on timeout.
+// A failed poll suspends the thread for a hardware-chosen time (about 4 us on B200, measured by
+// the wait self-test), so the default bound of 2^18 polls gives up after about one second; a
+// product completes in microseconds. The result is made warp-uniform by the caller before any
+// warp-collective tcgen05 access.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int max_polls = 1 << 18) {
   const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
-  for (int i = 0; i < (1 << 22); i++) {
+  for (int i = 0; i < max_polls; i++) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -467,6 +470,23 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
   tmem_free_cta(tbase, kCols);
 }
 
+// The timeout path of the bounded wait above, on its own: one CTA waits on an mbarrier that
+// expects one arrival; with arrive = 0 nothing arrives, every poll fails, and the CTA records the
+// same error word the SSD kernels record. No tensor memory or MMA is involved.
+__global__ void __launch_bounds__(128) wait_selftest_kernel(int arrive, int polls, int *error) {
+  __shared__ __align__(8) uint64_t bar;
+  const int t = threadIdx.x;
+  if (t == 0) mbar_init(&bar, 1);
+  __syncthreads();
+  if (arrive && t == 0) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(a)
+                 : "memory");
+  }
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, polls));
+  if (!ok && (t & 31) == 0) atomicExch(error, 1);
+}
+
 // ---- host ------------------------------------------------------------------------------------
 
 // header + operand tiles, or header + the padded fp32 result rows staged over them
@@ -512,6 +532,15 @@ size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t 
          + rnd(sizeof(__nv_bfloat16) * chunks * N * P)     // H_in
          + rnd(sizeof(float) * chunks)                     // cum_end
          + 256;                                            // error flag
+}
+
+size_t ssd_error_offset(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N) {
+  return ssd_workspace_bytes(Bt, H, L, P, N) - 256;
+}
+
+cudaError_t launch_wait_selftest(int arrive, int polls, int *error, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 128, 0, stream>>>(arrive, polls, error);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream) {

@@ -230,6 +230,23 @@ def test_ssd_validation_codes(lib):
     assert f(_ssd(workspace=0x100010, workspace_bytes=need)) == 7
 
 
+def test_failure_detection_validation_codes(lib):
+    # Error paths only: each returns before any CUDA call.
+    chk = lambda a: lib.ssm_ssd_check(ctypes.byref(a), None)
+    assert lib.ssm_ssd_check(None, None) == 1
+    assert chk(_ssd(P=32)) == 5                 # same argument checks as ssm_ssd_fwd
+    assert chk(_ssd(Bt=0, x=None)) == 0         # empty: nothing ran, nothing to read
+    assert chk(_ssd()) == 7                     # the error word lives in the workspace
+    need = lib.ssm_ssd_workspace_size(ctypes.byref(_ssd()))
+    assert chk(_ssd(workspace=0x100100, workspace_bytes=need - 1)) == 7
+    assert chk(_ssd(workspace=0x100010, workspace_bytes=need)) == 7
+    st = lib.ssm_wait_selftest
+    assert st(0, 16, None, None) == 1
+    assert st(0, 16, 0x1002, None) == 3
+    assert st(0, 0, 0x1000, None) == 2 and st(0, (1 << 22) + 1, 0x1000, None) == 2
+    assert lib.ssm_status_string(8).decode().startswith("SSM_ERR_TIMEOUT")
+
+
 def test_conv_validation_codes(lib):
     f = lib.ssm_conv1d_silu
     assert f(0x1000, 0x2000, 0x3000, None, 2, 4, 8, 4, 9, 0, None) == 4
