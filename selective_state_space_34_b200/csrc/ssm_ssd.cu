@@ -31,6 +31,8 @@ namespace {
 constexpr int kQ = 128;   // chunk length (steps)
 constexpr int kNP = 128;  // padded state dimension (N = 64 runs with zero rows)
 constexpr int kSsdHeader = 2048;  // bytes of small per-CTA data in front of the tiles
+constexpr int kHGMax = 8;         // heads per CTA at most (they share B, C and C B^T)
+constexpr int kCoefBytes = 3 * kHGMax * kQ * 4;  // output kernel: q, ct, e^{cum} of every head
 
 // ---- tcgen05 plumbing ----------------------------------------------------------------------
 
@@ -119,37 +121,33 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Cooperative copy of a tile of R rows x VPR 16-byte vectors (8 bf16 each) from a row-major
-// source into an operand tile: vector (row, v) goes to smem_off(row, v). Row r of the source
-// starts at src + r * rs elements; rows with valid(r) false, and vectors past vmax, read as zero.
-// A warp takes 8 rows x 4 vectors: 64 contiguous bytes per row from global memory, and the 8
-// lanes of each shared-memory phase write 8 different core-matrix rows (distinct banks).
-template <int R, int VPR, typename Off, typename Valid, typename Xform>
-__device__ __forceinline__ void coop_tile(unsigned char *tile, const __nv_bfloat16 *src, int64_t rs,
-                                          int vmax, Off smem_off, Valid valid, Xform xform) {
-  static_assert(R % 8 == 0 && (R * VPR) % 128 == 0, "tile shape");
-#pragma unroll 4
-  for (int it = 0; it < R * VPR / 128; it++) {
-    const int idx = it * 128 + threadIdx.x;
-    const int r8 = idx & 7, v = (idx >> 3) % VPR, rg = (idx >> 3) / VPR;
-    const int row = rg * 8 + r8;
-    uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-    if (valid(row) && v < vmax) pk = *reinterpret_cast<const uint4 *>(src + (int64_t)row * rs + v * 8);
-    *reinterpret_cast<uint4 *>(tile + smem_off(row, v)) = xform(row, pk);
-  }
+// Eight consecutive outputs (16-byte aligned destination): one 16-byte store for bf16, two for fp32.
+__device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                               pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
-struct NoXform {
-  __device__ __forceinline__ uint4 operator()(int, uint4 v) const { return v; }
-};
-// Same placement, copied asynchronously (cp.async, 16 bytes) with no transform; invalid rows are
-// zero-filled with plain stores. The caller commits, waits and fences before the tile is read.
+__device__ __forceinline__ void store8(float *dst, const float *v) {
+  *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Threads per CTA of the chunk-state and output kernels: two threads per tensor-memory lane (warps
+// w and w + 4 reach the same 32 lanes), each taking half of the row's columns.
+constexpr int kThr = 256;
+
+// Cooperative asynchronous copy (cp.async, 16 bytes) of a tile of R rows x VPR 16-byte vectors
+// (8 bf16 each) from a row-major source into an operand tile: vector (row, v) goes to
+// smem_off(row, v). Row r of the source starts at src + r * rs elements; rows with valid(r) false,
+// and vectors past vmax, are zero-filled with plain stores. A warp takes 8 rows x 4 vectors: 64
+// contiguous bytes per row from global memory, and the 8 lanes of each shared-memory phase write 8
+// different core-matrix rows (distinct banks). The caller commits, waits and fences.
 template <int R, int VPR, typename Off, typename Valid>
 __device__ __forceinline__ void coop_tile_async(unsigned char *tile, const __nv_bfloat16 *src,
                                                 int64_t rs, int vmax, Off smem_off, Valid valid) {
-  static_assert(R % 8 == 0 && (R * VPR) % 128 == 0, "tile shape");
+  static_assert(R % 8 == 0 && (R * VPR) % kThr == 0, "tile shape");
 #pragma unroll 4
-  for (int it = 0; it < R * VPR / 128; it++) {
-    const int idx = it * 128 + threadIdx.x;
+  for (int it = 0; it < R * VPR / kThr; it++) {
+    const int idx = it * kThr + threadIdx.x;
     const int r8 = idx & 7, v = (idx >> 3) % VPR, rg = (idx >> 3) / VPR;
     const int row = rg * 8 + r8;
     unsigned char *dst = tile + smem_off(row, v);
@@ -160,136 +158,176 @@ __device__ __forceinline__ void coop_tile_async(unsigned char *tile, const __nv_
   }
 }
 
-// Delta, log a = Delta A and beta of step t of the chunk (0 past the sequence end: an identity
-// step), and the inclusive running sum of log a over the chunk (block-wide scan, 128 threads).
-struct StepCoefs {
-  float la, beta, cum;
-};
-__device__ __forceinline__ StepCoefs chunk_coefs(const SsdParams &p, int64_t bh, int64_t t_glob,
-                                                 float A, float bias, float *scan_buf) {
-  float la = 0.f, beta = 0.f;
-  if (t_glob < p.L) {
-    const float v = to_f32(static_cast<const __nv_bfloat16 *>(p.dt)[bh * p.L + t_glob]) + bias;
-    const float dl = p.delta_softplus ? softplus<false>(v) : v;
-    la = dl * A;
-    beta = p.euler ? dl : expm1f(la) / A;
-  }
-  // inclusive scan of la over the 128 threads
-  float s = la;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float o = __shfl_up_sync(0xffffffffu, s, off);
-    if (lane >= off) s += o;
-  }
-  if (lane == 31) scan_buf[w] = s;
-  __syncthreads();
-  float base = 0.f;
-  for (int i = 0; i < w; i++) base += scan_buf[i];
-  __syncthreads();
-  return StepCoefs{la, beta, s + base};
+// This thread's lane of the CTA's tensor memory: row (threadIdx.x mod 128), column 0.
+__device__ __forceinline__ uint32_t ssd_lane_addr(uint32_t tbase) {
+  return tbase + (static_cast<uint32_t>(threadIdx.x & 96) << 16);
 }
 
 }  // namespace
 
 // ---- kernel 1: chunk states S_c = (w beta B)^T X -------------------------------------------
+// One CTA per (batch, chunk, group of HG <= 8 heads). B_c is shared by the heads: every thread
+// keeps its share of the raw tile in registers and, per head, writes it scaled by that head's
+// row weights e^{cum_end - cum_s} beta_s as the A operand. X of the next head is copied into a
+// second buffer while the current head's product runs. Thread t owns accumulator row t mod 128
+// (state n) and half of its P columns.
 template <int P>
-__global__ void __launch_bounds__(128, 1) ssd_state_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThr, 2) ssd_state_kernel(const SsdParams p, int HG) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  // header (scan scratch, per-row scales, barrier, TMEM address), then the operand tiles; the
-  // tiles' region is reused afterwards to stage the result rows
-  float *scan_buf = reinterpret_cast<float *>(smem);                 // 8 + kQ floats
+  float *scan_buf = reinterpret_cast<float *>(smem);  // header: kHGMax x 4 warp sums, cum_end per head
+  float *cend_s = scan_buf + kHGMax * 4;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSsdHeader - 16);
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + kSsdHeader - 8);
-  unsigned char *sA = smem + kSsdHeader;          // (w beta B)^T: M = n (128), K = s (128), MN-major
-  unsigned char *sX = sA + kNP * kQ * 2;          // X: N = p (P), K = s (128), MN-major
+  float *scale_s = reinterpret_cast<float *>(smem + kSsdHeader);       // [head][step]
+  unsigned char *sA = smem + kSsdHeader + kHGMax * kQ * 4;             // M = n (128), K = s, MN-major
+  unsigned char *sX0 = sA + kNP * kQ * 2;                              // N = p (P), K = s, MN-major; x2
 
+  constexpr uint32_t kCols = P < 32 ? 32u : (uint32_t)P;
+  constexpr int VPR = kNP / 8;                   // 16-byte vectors per row of B
+  constexpr int NV = kQ * VPR / kThr;            // vectors of B per thread
+  constexpr int HH = kHGMax / 2;                 // heads per thread in the coefficient pass
   const int64_t nC = (p.L + kQ - 1) / kQ;
-  const int64_t c = blockIdx.x % nC, bh = blockIdx.x / nC, b = bh / p.H, h = bh % p.H;
-  const int t = threadIdx.x;
-  const int64_t tg = c * kQ + t;
+  const int64_t ngrp = p.H / HG;
+  const int64_t c = blockIdx.x % nC, rest = blockIdx.x / nC;
+  const int64_t hgrp = rest % ngrp, b = rest / ngrp;
+  const int t = threadIdx.x, r = t & 127, hf = t >> 7, wq = (t >> 5) & 3;
+  const int64_t rows_left = p.L - c * kQ;
+  auto valid = [&](int row) { return row < rows_left; };
+  auto load_x = [&](int hi) {
+    const int64_t bh = b * p.H + hgrp * HG + hi;
+    coop_tile_async<kQ, P / 8>(sX0 + (hi & 1) * P * kQ * 2,
+                               static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8,
+                               [](int row, int v) { return mnmaj_off(P, v * 8, row); }, valid);
+    cp_async_commit();
+  };
 
-  const uint32_t tbase = tmem_alloc_cta(slot, (uint32_t)P);
+  const uint32_t tbase = tmem_alloc_cta(slot, kCols);
   if (t == 0) mbar_init(bar, 1);
-
-  const float A = -expf(p.A_log[h]);
-  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
-  const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);
-  // total log-decay of the chunk = the last thread's inclusive sum
-  if (t == kQ - 1) scan_buf[4] = k.cum;
-  __syncthreads();
-  const float cum_end = scan_buf[4];
-  const float scale = k.beta * __expf(cum_end - k.cum);  // e^{cum_end - cum_s} beta_s
-
-  // stage both operands: row s of B scaled by e^{cum_end - cum_s} beta_s (A operand, MN-major
-  // along n), row s of X (B operand, MN-major along p)
-  float *row_scale = scan_buf + 8;  // kQ floats after the scan scratch
-  row_scale[t] = scale;
-  __syncthreads();
+  load_x(0);
+  // row weights: thread (r, hf) takes step r of heads hf, hf + 2, ...
   {
-    const int64_t rows_left = p.L - c * kQ;
-    auto valid = [&](int r) { return r < rows_left; };
+    const int64_t tg = c * kQ + r;
+    float beta[HH], sc[HH];
+#pragma unroll
+    for (int j = 0; j < HH; j++) {
+      const int hi = 2 * j + hf;
+      float la = 0.f;
+      beta[j] = 0.f;
+      if (hi < HG && tg < p.L) {
+        const int64_t h = hgrp * HG + hi;
+        const float A = -expf(p.A_log[h]);
+        const float v = to_f32(static_cast<const __nv_bfloat16 *>(p.dt)[(b * p.H + h) * p.L + tg]) +
+                        (p.dt_bias ? p.dt_bias[h] : 0.f);
+        const float dl = p.delta_softplus ? softplus<false>(v) : v;
+        la = dl * A;
+        beta[j] = p.euler ? dl : expm1f(la) / A;  // 0 past the sequence end: identity steps
+      }
+      sc[j] = la;
+    }
+    const int lane = t & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int j = 0; j < HH; j++) {
+        const float o = __shfl_up_sync(0xffffffffu, sc[j], off);
+        if (lane >= off) sc[j] += o;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int j = 0; j < HH; j++) scan_buf[(2 * j + hf) * 4 + wq] = sc[j];
+    }
+    __syncthreads();
+    if (t < HG) cend_s[t] = scan_buf[t * 4] + scan_buf[t * 4 + 1] + scan_buf[t * 4 + 2] + scan_buf[t * 4 + 3];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < HH; j++) {
+      const int hi = 2 * j + hf;
+      if (hi < HG) {
+        float base = 0.f;
+        for (int i = 0; i < wq; i++) base += scan_buf[hi * 4 + i];
+        scale_s[hi * kQ + r] = beta[j] * __expf(cend_s[hi] - (sc[j] + base));  // e^{cum_end - cum_s} beta_s
+      }
+    }
+    if (t < HG) p.cum_end[(b * p.H + hgrp * HG + t) * nC + c] = cend_s[t];
+  }
+  // this thread's vectors of the raw B tile (rows past the sequence end and n >= N read as zero)
+  uint4 braw[NV];
+  {
     const __nv_bfloat16 *Bsrc = static_cast<const __nv_bfloat16 *>(p.B) + (b * p.L + c * kQ) * p.N;
-    coop_tile<kQ, kNP / 8>(sA, Bsrc, p.N, (int)(p.N / 8),
-                           [](int r, int v) { return mnmaj_off(kNP, v * 8, r); }, valid,
-                           [&](int r, uint4 pk) {
-                             const float sc = row_scale[r];
-                             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&pk);
-                             uint4 o;
-                             uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+    const int vmax = (int)(p.N / 8);
 #pragma unroll
-                             for (int i = 0; i < 4; i++) {
-                               const float2 f = __bfloat1622float2(h2[i]);
-                               ow[i] = pack_bf16(f.x * sc, f.y * sc);
-                             }
-                             return o;
-                           });
-    const __nv_bfloat16 *Xsrc = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
-    coop_tile<kQ, P / 8>(sX, Xsrc, P, P / 8, [](int r, int v) { return mnmaj_off(P, v * 8, r); },
-                         valid, NoXform());
-  }
-  fence_async_smem();
-  __syncthreads();
-  tc_fence_after();
-  if (t == 0) {
-    constexpr uint32_t idesc = instr_desc(128, P, 1, 1);
-#pragma unroll
-    for (int ks = 0; ks < kQ / 16; ks++) {
-      const uint64_t da = smem_desc(sA + ks * 2 * (kNP / 8) * 128, (kNP / 8) * 128, 128);
-      const uint64_t db = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
-      mma_bf16(tbase, da, db, idesc, ks > 0);
+    for (int it = 0; it < NV; it++) {
+      const int idx = it * kThr + t;
+      const int row = ((idx >> 3) / VPR) * 8 + (idx & 7), v = (idx >> 3) % VPR;
+      braw[it] = (valid(row) && v < vmax) ? *reinterpret_cast<const uint4 *>(Bsrc + (int64_t)row * p.N + v * 8)
+                                          : make_uint4(0u, 0u, 0u, 0u);
     }
-    mma_commit(bar);
   }
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
-  tc_fence_after();
+  __syncthreads();  // the row weights of every head are in place
+
+  bool ok = true;
+  const uint32_t lane_addr = ssd_lane_addr(tbase);
+  for (int hi = 0; hi < HG; hi++) {
+    const int64_t bh = b * p.H + hgrp * HG + hi;
+    const unsigned char *sX = sX0 + (hi & 1) * P * kQ * 2;
+    // A operand of this head: row s of B times its weight, MN-major along n
+    {
+      const float *wts = scale_s + hi * kQ;
+#pragma unroll
+      for (int it = 0; it < NV; it++) {
+        const int idx = it * kThr + t;
+        const int row = ((idx >> 3) / VPR) * 8 + (idx & 7), v = (idx >> 3) % VPR;
+        const float sw = wts[row];
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&braw[it]);
+        uint4 o;
+        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          const float2 f = __bfloat1622float2(h2[i]);
+          ow[i] = pack_bf16(f.x * sw, f.y * sw);
+        }
+        *reinterpret_cast<uint4 *>(sA + mnmaj_off(kNP, v * 8, row)) = o;
+      }
+    }
+    cp_async_wait<0>();  // this thread's copies of this head's X landed
+    tc_fence_before();
+    fence_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      constexpr uint32_t idesc = instr_desc(128, P, 1, 1);
+#pragma unroll
+      for (int ks = 0; ks < kQ / 16; ks++) {
+        const uint64_t da = smem_desc(sA + ks * 2 * (kNP / 8) * 128, (kNP / 8) * 128, 128);
+        const uint64_t db = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+        mma_bf16(tbase, da, db, idesc, ks > 0);
+      }
+      mma_commit(bar);
+    }
+    // the other X buffer was read by the previous head's product, which has completed
+    if (hi + 1 < HG) load_x(hi + 1);
+    ok = __all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)(hi & 1))) && ok;
+    tc_fence_after();
+    // row n = r of S_c, columns of this half, straight from the accumulator to global memory
+    // (rows n >= N are padding)
+    {
+      float *dst = p.S + ((bh * nC + c) * p.N + r) * P + hf * (P / 2);
+#pragma unroll 1
+      for (int q = 0; q < P / 2; q += 32) {
+        float v[32];
+        tmem_ld32(lane_addr + hf * (P / 2) + q, v);
+        if (ok && r < p.N) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(dst + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+    }
+  }
   if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
-  // row n = t of S_c: TMEM -> registers -> shared (padded rows, over the consumed A tile) ->
-  // coalesced global stores
-  constexpr int SR = P + 4;  // padded row, floats
-  float *stage = reinterpret_cast<float *>(sA);
-  {
-    const uint32_t lane_addr = tmem_lane_addr(tbase);
-#pragma unroll
-    for (int q = 0; q < P; q += 32) {
-      float v[32];
-      tmem_ld32(lane_addr + q, v);
-#pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4 *>(stage + t * SR + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-    }
-  }
-  __syncthreads();
-  if (ok) {
-    float *dst = p.S + (bh * nC + c) * p.N * P;
-    for (int i = t; i < p.N * P / 4; i += 128) {
-      const int r = i / (P / 4), q = (i % (P / 4)) * 4;
-      *reinterpret_cast<float4 *>(dst + r * P + q) = *reinterpret_cast<const float4 *>(stage + r * SR + q);
-    }
-  }
-  if (t == 0) p.cum_end[bh * nC + c] = cum_end;
   tc_fence_before();
-  tmem_free_cta(tbase, (uint32_t)P);
+  tmem_free_cta(tbase, kCols);
 }
 
 // ---- kernel 2: carry over chunks ------------------------------------------------------------
@@ -320,31 +358,48 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
 }
 
 // ---- kernel 3: chunk outputs ------------------------------------------------------------------
-// One CTA per (batch, chunk, group of HG heads): C and B are shared by the heads, so they are
+// One CTA per (batch, chunk, group of HG <= 8 heads): C and B are shared by the heads, so they are
 // staged once and G = C B^T is formed once; each head then applies its own decays to G.
+//
+// The decay of score (t, s) is written e^{cum_t - cum_s} beta_s = 2^{ct_t - q_s} with
+// ct_t = cum_t log2 e and q_s = cum_s log2 e - log2 beta_s, both computed once per step and head
+// (beta_s = 0 gives q_s = +inf and a zero score). The skip term D x_t is the diagonal of the
+// product G' X, so it is added to G'[t][t] rather than re-reading x. Scores above the diagonal are
+// zero for every head: those blocks are cleared once and never rewritten. Thread t owns row
+// t mod 128 of every accumulator and half of its columns.
 template <int P, typename Tout>
-__global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int HG) {
+__global__ void __launch_bounds__(kThr, 1) ssd_out_kernel(const SsdParams p, int HG) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  float *cum_s = reinterpret_cast<float *>(smem);  // header: 2 kQ + 8 floats, 2 barriers, slot
-  float *beta_s = cum_s + kQ;
-  float *scan_buf = beta_s + kQ;
+  float *scan_buf = reinterpret_cast<float *>(smem);  // header: kHGMax x 4 warp sums, D per head
+  float *Dh_s = scan_buf + kHGMax * 4;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSsdHeader - 24);  // two barriers
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + kSsdHeader - 8);
-  unsigned char *sC = smem + kSsdHeader;           // C: M = t (128), K = n (128), K-major
-  unsigned char *sB = sC + kQ * kNP * 2;           // B: N = s, K = n, K-major; then each head's G'
-  unsigned char *sX = sB + kQ * kNP * 2;           // X: N = p (P), K = s (128), MN-major
-  unsigned char *sH = sX + P * kQ * 2;             // H_in: N = p (P), K = n (128), MN-major
-  float *stage = reinterpret_cast<float *>(sB);    // result rows, over G' and X once consumed
+  float *q_s = reinterpret_cast<float *>(smem + kSsdHeader);  // [head][step]
+  float *ct_s = q_s + kHGMax * kQ;
+  float *et_s = ct_s + kHGMax * kQ;
+  unsigned char *sC = smem + kSsdHeader + kCoefBytes;  // C: M = t (128), K = n (128), K-major
+  unsigned char *sB = sC + kQ * kNP * 2;  // B: N = s, K = n, K-major; then each head's G' (K = s)
+  unsigned char *sX = sB + kQ * kNP * 2;  // X: N = p (P), K = s (128), MN-major
+  unsigned char *sH = sX + P * kQ * 2;    // H_in: N = p (P), K = n (128), MN-major
 
   constexpr uint32_t kCols = (128 + 2 * P <= 256) ? 256u : 512u;  // G (128) + Y (P) + C H (P)
+  constexpr int HH = kHGMax / 2;  // heads per thread in the coefficient pass
   const int64_t nC = (p.L + kQ - 1) / kQ;
   const int64_t ngrp = p.H / HG;
   const int64_t c = blockIdx.x % nC, rest = blockIdx.x / nC;
   const int64_t hgrp = rest % ngrp, b = rest / ngrp;
-  const int t = threadIdx.x;
-  const int64_t tg = c * kQ + t;
+  const int t = threadIdx.x, r = t & 127, hf = t >> 7, wq = (t >> 5) & 3;
   const int64_t rows_left = p.L - c * kQ;
-  auto valid = [&](int r) { return r < rows_left; };
+  auto valid = [&](int row) { return row < rows_left; };
+  const int nks = (int)((p.N + 15) / 16);  // K slices of C H that are not all zero padding
+  auto load_xh = [&](int hi) {  // this head's X and H_in tiles, asynchronously
+    const int64_t bh = b * p.H + hgrp * HG + hi;
+    const auto mnmaj = [](int row, int v) { return mnmaj_off(P, v * 8, row); };
+    coop_tile_async<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid);
+    const int64_t nrows = p.N;
+    coop_tile_async<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int row) { return row < nrows; });
+    cp_async_commit();
+  };
 
   const uint32_t tbase = tmem_alloc_cta(slot, kCols);
   if (t == 0) {
@@ -352,11 +407,16 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
     mbar_init(bar + 1, 1);
   }
   {
+    // C and B first (one group), then the first head's X and H_in (a second group): every copy is
+    // in flight at once, and only the first group is waited for before C B^T
     const int64_t off = (b * p.L + c * kQ) * p.N;
-    const auto kmaj = [](int r, int v) { return kmaj_off(kQ, r, v * 8); };
-    coop_tile<kQ, kNP / 8>(sC, static_cast<const __nv_bfloat16 *>(p.C) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
-    coop_tile<kQ, kNP / 8>(sB, static_cast<const __nv_bfloat16 *>(p.B) + off, p.N, (int)(p.N / 8), kmaj, valid, NoXform());
+    const auto kmaj = [](int row, int v) { return kmaj_off(kQ, row, v * 8); };
+    coop_tile_async<kQ, kNP / 8>(sC, static_cast<const __nv_bfloat16 *>(p.C) + off, p.N, (int)(p.N / 8), kmaj, valid);
+    coop_tile_async<kQ, kNP / 8>(sB, static_cast<const __nv_bfloat16 *>(p.B) + off, p.N, (int)(p.N / 8), kmaj, valid);
+    cp_async_commit();
   }
+  load_xh(0);
+  cp_async_wait<1>();
   fence_async_smem();
   __syncthreads();
   tc_fence_after();
@@ -370,43 +430,97 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
     }
     mma_commit(bar);
   }
+
+  // while G is formed: the decay coefficients, thread (r, hf) taking step r of heads hf, hf + 2, ...
+  {
+    const int64_t tg = c * kQ + r;
+    float beta[HH], sc[HH];
+#pragma unroll
+    for (int j = 0; j < HH; j++) {
+      const int hi = 2 * j + hf;
+      float la = 0.f;
+      beta[j] = 0.f;
+      if (hi < HG && tg < p.L) {
+        const int64_t h = hgrp * HG + hi;
+        const float A = -expf(p.A_log[h]);
+        const float v = to_f32(static_cast<const __nv_bfloat16 *>(p.dt)[(b * p.H + h) * p.L + tg]) +
+                        (p.dt_bias ? p.dt_bias[h] : 0.f);
+        const float dl = p.delta_softplus ? softplus<false>(v) : v;
+        la = dl * A;
+        beta[j] = p.euler ? dl : expm1f(la) / A;  // 0 past the sequence end: identity steps
+      }
+      sc[j] = la;
+    }
+    // inclusive scan of log a over the chunk (the 4 warps of this thread's half)
+    const int lane = t & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int j = 0; j < HH; j++) {
+        const float o = __shfl_up_sync(0xffffffffu, sc[j], off);
+        if (lane >= off) sc[j] += o;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int j = 0; j < HH; j++) scan_buf[(2 * j + hf) * 4 + wq] = sc[j];
+    }
+    if (t < HG) Dh_s[t] = p.D ? p.D[hgrp * HG + t] : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < HH; j++) {
+      const int hi = 2 * j + hf;
+      if (hi < HG) {
+        float base = 0.f;
+        for (int i = 0; i < wq; i++) base += scan_buf[hi * 4 + i];
+        const float cum = sc[j] + base;
+        q_s[hi * kQ + r] = cum * kLog2e - lg2_approx(beta[j]);
+        ct_s[hi * kQ + r] = cum * kLog2e;
+        et_s[hi * kQ + r] = __expf(cum);
+      }
+    }
+  }
   bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0));
+  tc_fence_after();
+  // B is consumed: clear this thread's half of the score blocks above the diagonal, once
+#pragma unroll
+  for (int kb = 1; kb < 4; kb++)
+    if (kb > wq) {
+      *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, r, kb * 32 + hf * 16)) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, r, kb * 32 + hf * 16 + 8)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  __syncthreads();  // the coefficients of every head are in place
+
   uint32_t phase = 0;  // of bar + 1, one completion per head
-  const uint32_t lane_addr = tmem_lane_addr(tbase);
+  const uint32_t lane_addr = ssd_lane_addr(tbase);
   for (int hi = 0; hi < HG; hi++) {
     const int64_t h = hgrp * HG + hi, bh = b * p.H + h;
-    // this head's X and H_in tiles travel while the decays and G' are computed
+    // G'[t][s] = G[t][s] 2^{ct_t - q_s} for s <= t (+ D on the diagonal): the A operand of G' X;
+    // this thread: row r, the 16 columns hf*16.. of every block on or below the diagonal
     {
-      const auto mnmaj = [](int r, int v) { return mnmaj_off(P, v * 8, r); };
-      coop_tile_async<kQ, P / 8>(sX, static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P, P, P / 8, mnmaj, valid);
-      const int64_t nrows = p.N;
-      coop_tile_async<kNP, P / 8>(sH, p.Hin + (bh * nC + c) * p.N * P, P, P / 8, mnmaj, [&](int r) { return r < nrows; });
-      cp_async_commit();
-    }
-    const float A = -expf(p.A_log[h]);
-    const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
-    const StepCoefs k = chunk_coefs(p, bh, tg, A, bias, scan_buf);  // (synchronises the CTA)
-    cum_s[t] = k.cum;
-    beta_s[t] = k.beta;
-    __syncthreads();  // cum_s / beta_s of this head
-    tc_fence_after();
-    // G'[t][s] = G[t][s] e^{cum_t - cum_s} beta_s for s <= t -> the A operand of G' X
-    {
-      const float ct = k.cum;
+      const float ct = ct_s[hi * kQ + r], Dh = Dh_s[hi];
+      const float *qh = q_s + hi * kQ;
 #pragma unroll 1
-      for (int s0 = 0; s0 < kQ; s0 += 32) {
-        float g[32];
-        tmem_ld32(lane_addr + s0, g);
+      for (int kb = 0; kb < 4; kb++) {
+        if (kb > wq) break;  // warp-uniform: the blocks above the diagonal stay zero
+        const int s0 = kb * 32 + hf * 16;
+        float g[16];
+        tmem_ld2<8>(lane_addr + s0, g, lane_addr + s0 + 8, g + 8);
+        const bool diag = kb == wq;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
+        for (int e = 0; e < 16; e += 8) {
+          const float4 q0 = *reinterpret_cast<const float4 *>(qh + s0 + e);
+          const float4 q1 = *reinterpret_cast<const float4 *>(qh + s0 + e + 4);
+          const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
           float v[8];
 #pragma unroll
           for (int j = 0; j < 8; j++) {
             const int s = s0 + e + j;
-            v[j] = (s <= t) ? g[e + j] * __expf(ct - cum_s[s]) * beta_s[s] : 0.f;
+            const float sv = g[e + j] * ex2_approx(ct - qv[j]);
+            v[j] = (!diag || s < r) ? sv : (s == r ? sv + Dh : 0.f);
           }
-          uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-          *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, t, s0 + e)) = pk;
+          const uint4 pk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, r, s0 + e)) = pk;
         }
       }
     }
@@ -420,9 +534,11 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
       for (int ks = 0; ks < kQ / 16; ks++) {
         const uint64_t dg = smem_desc(sB + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
         const uint64_t dx = smem_desc(sX + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
+        mma_bf16(tY, dg, dx, instr_desc(128, P, 0, 1), ks > 0);
+      }
+      for (int ks = 0; ks < nks; ks++) {
         const uint64_t dc = smem_desc(sC + ks * 2 * (kQ / 8) * 128, (kQ / 8) * 128, 128);
         const uint64_t dh = smem_desc(sH + ks * 2 * (P / 8) * 128, (P / 8) * 128, 128);
-        mma_bf16(tY, dg, dx, instr_desc(128, P, 0, 1), ks > 0);
         mma_bf16(tCH, dc, dh, instr_desc(128, P, 0, 1), ks > 0);
       }
       mma_commit(bar + 1);
@@ -430,40 +546,25 @@ __global__ void __launch_bounds__(128, 1) ssd_out_kernel(const SsdParams p, int 
     ok = __all_sync(0xffffffffu, mbar_wait(bar + 1, phase)) && ok;
     phase ^= 1u;
     tc_fence_after();
-    // y row t = G'X + e^{cum_t} C H_in -> shared (padded) -> coalesced stores with + D x
-    constexpr int SR = P + 4;
+    // the products have read X, H_in and G': the next head's tiles travel during this epilogue
+    if (hi + 1 < HG) load_xh(hi + 1);
+    // y row r, this half's columns = G'X + e^{cum_t} C H_in, from the accumulators to global memory
     {
-      const float et = __expf(k.cum);
+      const float et = et_s[hi * kQ + r];
+      Tout *yrow = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ + r) * P + hf * (P / 2);
 #pragma unroll 1
-      for (int q = 0; q < P; q += 32) {
+      for (int q = 0; q < P / 2; q += 32) {
         float yv[32], cv[32];
-        tmem_ld32(lane_addr + 128 + q, yv);
-        tmem_ld32(lane_addr + 128 + P + q, cv);
+        tmem_ld32(lane_addr + 128 + hf * (P / 2) + q, yv);
+        tmem_ld32(lane_addr + 128 + P + hf * (P / 2) + q, cv);
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4 *>(stage + t * SR + q + j) =
-              make_float4(fmaf(et, cv[j], yv[j]), fmaf(et, cv[j + 1], yv[j + 1]),
-                          fmaf(et, cv[j + 2], yv[j + 2]), fmaf(et, cv[j + 3], yv[j + 3]));
+        for (int j = 0; j < 32; j++) yv[j] = fmaf(et, cv[j], yv[j]);
+        if (ok && r < rows_left) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) store8(yrow + q + j, yv + j);
+        }
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (ok) {
-      const float Dh = p.D ? p.D[h] : 0.f;
-      const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(p.x) + (bh * p.L + c * kQ) * P;
-      Tout *ys = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ) * P;
-      for (int i = t; i < kQ * P / 4; i += 128) {
-        const int r = i / (P / 4), q = (i % (P / 4)) * 4;
-        if (r >= rows_left) continue;
-        const float4 v = *reinterpret_cast<const float4 *>(stage + r * SR + q);
-        const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (int64_t)r * P + q);
-        const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
-        const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
-        const float o[4] = {fmaf(Dh, x01.x, v.x), fmaf(Dh, x01.y, v.y), fmaf(Dh, x23.x, v.z), fmaf(Dh, x23.y, v.w)};
-        VecStore<Tout, 4>::run(ys + (int64_t)r * P + q, o);
-      }
-    }
-    __syncthreads();  // the staged rows, G' and X are rewritten by the next head
   }
   if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
   tc_fence_before();
@@ -491,14 +592,12 @@ __global__ void __launch_bounds__(128) wait_selftest_kernel(int arrive, int poll
 
 // header + operand tiles, or header + the padded fp32 result rows staged over them
 size_t ssd_smem_state(int P) {
-  const size_t tiles = (size_t)kNP * kQ * 2 + (size_t)P * kQ * 2, stage = (size_t)kNP * (P + 4) * 4;
-  return kSsdHeader + (tiles > stage ? tiles : stage);
+  // header, the heads' row weights, the A operand, two X buffers
+  return kSsdHeader + (size_t)kHGMax * kQ * 4 + (size_t)kNP * kQ * 2 + (size_t)2 * P * kQ * 2;
 }
 size_t ssd_smem_out(int P) {
-  // C, B / G', X, H_in; the staged result rows overlay G' and X (kQ x (P + 4) floats)
-  const size_t tiles = (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2;
-  const size_t stage_end = (size_t)kQ * kNP * 2 + (size_t)kQ * (P + 4) * 4;
-  return kSsdHeader + (tiles > stage_end ? tiles : stage_end);
+  // header, the heads' decay coefficients, then C, B / G', X, H_in
+  return kSsdHeader + kCoefBytes + (size_t)2 * kQ * kNP * 2 + (size_t)P * kQ * 2 + (size_t)P * kNP * 2;
 }
 
 template <int P, typename Tout>
@@ -510,17 +609,17 @@ static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(ssd_state_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(ssd_out_kernel<P, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
   if (e != cudaSuccess) return e;
-  ssd_state_kernel<P><<<(unsigned)grid, 128, s1, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H * (p.N * P / 1024)), 256, 0, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  int HG = 1;  // heads per CTA: C, B and C B^T are shared by them
+  int HG = 1;  // heads per CTA: B (and C, C B^T) are shared by them
   for (int cand : {8, 4, 2})
     if (p.H % cand == 0) {
       HG = cand;
       break;
     }
-  ssd_out_kernel<P, Tout><<<(unsigned)(grid / HG), 128, s3, s>>>(p, HG);
+  ssd_state_kernel<P><<<(unsigned)(grid / HG), kThr, s1, s>>>(p, HG);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H * (p.N * P / 1024)), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ssd_out_kernel<P, Tout><<<(unsigned)(grid / HG), kThr, s3, s>>>(p, HG);
   return cudaGetLastError();
 }
 

@@ -3,8 +3,8 @@
 
 Tolerance, from the arithmetic: three bf16 roundings reach an output -- beta_s e^{cum_end-cum_s}
 B_s as an operand of the chunk-state product, the state entering a chunk, and the masked scores
-(C_t . B_s) e^{cum_t-cum_s} beta_s -- each a relative error of at most 2^-9 per term, with fp32
-accumulation. So |y - y_ref| <= 3 * 2^-9 * Y_abs where Y_abs bounds the sum of the terms' magnitudes:
+(C_t . B_s) e^{cum_t-cum_s} beta_s, whose diagonal also carries the skip weight D -- each a
+relative error of at most 2^-9 per term, with fp32 accumulation. So |y - y_ref| <= 3 * 2^-9 * Y_abs where Y_abs bounds the sum of the terms' magnitudes:
 the oracle run on |x|, |B|, |C|, |D| (|C_t . B_s| <= |C_t| . |B_s|; beta, the decays and the state
 recursion are non-negative maps of non-negative inputs). The tests allow 2^-6 * Y_abs, plus 2^-8 |y|
 for a bf16 output."""
