@@ -121,14 +121,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Eight consecutive outputs (16-byte aligned destination): one 16-byte store for bf16, two for fp32.
-__device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
+// One 16-byte chunk of outputs into shared memory: 8 values as bf16, or 4 as fp32.
+__device__ __forceinline__ void put16(unsigned char *dst, const float *v, __nv_bfloat16 *) {
   *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
                                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
-__device__ __forceinline__ void store8(float *dst, const float *v) {
+__device__ __forceinline__ void put16(unsigned char *dst, const float *v, float *) {
   *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-  *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
 // Threads per CTA of the chunk-state and output kernels: two threads per tensor-memory lane (warps
@@ -309,19 +308,30 @@ __global__ void __launch_bounds__(kThr, 2) ssd_state_kernel(const SsdParams p, i
     if (hi + 1 < HG) load_x(hi + 1);
     ok = __all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)(hi & 1))) && ok;
     tc_fence_after();
-    // row n = r of S_c, columns of this half, straight from the accumulator to global memory
-    // (rows n >= N are padding)
+    // S_c leaves through the consumed A tile, 64 columns at a time: thread (r, hf) parks its 32
+    // columns of row r as 16-byte chunks at slot (chunk ^ (r mod 16)) -- no bank conflicts -- and
+    // the CTA then writes whole rows (256 contiguous bytes) to global memory; rows n >= N are padding
     {
-      float *dst = p.S + ((bh * nC + c) * p.N + r) * P + hf * (P / 2);
+      float *stage = reinterpret_cast<float *>(sA);  // 128 rows x 64 floats
+      float *dst = p.S + (bh * nC + c) * p.N * P;
 #pragma unroll 1
-      for (int q = 0; q < P / 2; q += 32) {
+      for (int q0 = 0; q0 < P; q0 += 64) {
         float v[32];
-        tmem_ld32(lane_addr + hf * (P / 2) + q, v);
-        if (ok && r < p.N) {
+        tmem_ld32(lane_addr + q0 + hf * 32, v);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4 *>(dst + q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        for (int i = 0; i < 8; i++) {
+          const int slot = (hf * 8 + i) ^ (r & 15);
+          *reinterpret_cast<float4 *>(stage + r * 64 + slot * 4) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
+        __syncthreads();
+#pragma unroll
+        for (int it = 0; it < 128 * 16 / kThr; it++) {
+          const int idx = it * kThr + t, row = idx >> 4, j = idx & 15;
+          if (ok && row < p.N)
+            *reinterpret_cast<float4 *>(dst + (int64_t)row * P + q0 + j * 4) =
+                *reinterpret_cast<const float4 *>(stage + row * 64 + ((j ^ (row & 15)) * 4));
+        }
+        __syncthreads();  // the stage (the A tile) is rewritten next
       }
     }
   }
@@ -368,7 +378,7 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
 // zero for every head: those blocks are cleared once and never rewritten. Thread t owns row
 // t mod 128 of every accumulator and half of its columns.
 template <int P, typename Tout>
-__global__ void __launch_bounds__(kThr, 1) ssd_out_kernel(const SsdParams p, int HG) {
+__global__ void __launch_bounds__(kThr, 2) ssd_out_kernel(const SsdParams p, int HG) {
   extern __shared__ __align__(1024) unsigned char smem[];
   float *scan_buf = reinterpret_cast<float *>(smem);  // header: kHGMax x 4 warp sums, D per head
   float *Dh_s = scan_buf + kHGMax * 4;
@@ -548,22 +558,49 @@ __global__ void __launch_bounds__(kThr, 1) ssd_out_kernel(const SsdParams p, int
     tc_fence_after();
     // the products have read X, H_in and G': the next head's tiles travel during this epilogue
     if (hi + 1 < HG) load_xh(hi + 1);
-    // y row r, this half's columns = G'X + e^{cum_t} C H_in, from the accumulators to global memory
+    // y = G'X + e^{cum_t} C H_in leaves through the consumed G' tile, W columns at a time (staged
+    // rows of at most 256 bytes): thread (r, hf) parks its half of row r as 16-byte chunks at slot
+    // (chunk ^ (r mod CPR)) -- no bank conflicts -- and the CTA then writes whole rows to global
+    // memory. The zero blocks above the diagonal of G' are cleared again afterwards.
     {
+      constexpr int ES = (int)sizeof(Tout);
+      constexpr int W = P * ES <= 256 ? P : 256 / ES;  // columns per pass
+      constexpr int CPR = W * ES / 16;                 // 16-byte chunks per staged row
+      constexpr int EPC = 16 / ES;                     // elements per chunk
       const float et = et_s[hi * kQ + r];
-      Tout *yrow = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ + r) * P + hf * (P / 2);
+      Tout *yblk = static_cast<Tout *>(p.y) + (bh * p.L + c * kQ) * P;
 #pragma unroll 1
-      for (int q = 0; q < P / 2; q += 32) {
-        float yv[32], cv[32];
-        tmem_ld32(lane_addr + 128 + hf * (P / 2) + q, yv);
-        tmem_ld32(lane_addr + 128 + P + hf * (P / 2) + q, cv);
+      for (int q0 = 0; q0 < P; q0 += W) {
+#pragma unroll 1
+        for (int q = 0; q < W / 2; q += 32) {
+          const int col = q0 + hf * (W / 2) + q;
+          float yv[32], cv[32];
+          tmem_ld32(lane_addr + 128 + col, yv);
+          tmem_ld32(lane_addr + 128 + P + col, cv);
 #pragma unroll
-        for (int j = 0; j < 32; j++) yv[j] = fmaf(et, cv[j], yv[j]);
-        if (ok && r < rows_left) {
+          for (int j = 0; j < 32; j++) yv[j] = fmaf(et, cv[j], yv[j]);
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) store8(yrow + q + j, yv + j);
+          for (int i = 0; i < 32 / EPC; i++) {
+            const int slot = ((hf * (W / 2) + q) / EPC + i) ^ (r & (CPR - 1));
+            put16(sB + r * CPR * 16 + slot * 16, yv + i * EPC, static_cast<Tout *>(nullptr));
+          }
         }
+        __syncthreads();
+#pragma unroll
+        for (int it = 0; it < kQ * CPR / kThr; it++) {
+          const int idx = it * kThr + t, row = idx / CPR, j = idx % CPR;
+          if (ok && row < rows_left)
+            *reinterpret_cast<uint4 *>(yblk + (int64_t)row * P + q0 + j * EPC) =
+                *reinterpret_cast<const uint4 *>(sB + row * CPR * 16 + (j ^ (row & (CPR - 1))) * 16);
+        }
+        __syncthreads();  // the stage is read out
       }
+#pragma unroll
+      for (int kb = 1; kb < 4; kb++)
+        if (kb > wq) {
+          *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, r, kb * 32 + hf * 16)) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4 *>(sB + kmaj_off(kQ, r, kb * 32 + hf * 16 + 8)) = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
   }
   if (!ok && (t & 31) == 0) atomicExch(p.error, 1);
