@@ -187,6 +187,10 @@ typedef struct ssm_ssd_args {
   int32_t discretization;/* ssm_discretization */
   void *workspace;       /* device scratch of ssm_ssd_workspace_size() bytes, 256-byte aligned */
   size_t workspace_bytes;
+  void *const *timing_events; /* NULL, or 2 caller-created cudaEvent_t: [0] is recorded on
+                                 `stream` just before the output kernel (the last of the three
+                                 launches), [1] just after it; lets a caller time that kernel
+                                 alone. Recording does not synchronise. */
 } ssm_ssd_args;
 
 /* Scratch bytes ssm_ssd_fwd needs: the chunk states (fp32), the state entering every chunk

@@ -73,6 +73,7 @@ class SsdArgs(ctypes.Structure):
         ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
         ("delta_softplus", ctypes.c_int32), ("discretization", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("timing_events", ctypes.c_void_p),
     ]
 
 

@@ -469,6 +469,7 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream) {
   p.N = args->N;
   p.delta_softplus = args->delta_softplus ? 1 : 0;
   p.euler = args->discretization == SSM_EULER ? 1 : 0;
+  p.timing_events = args->timing_events;
   p.S = reinterpret_cast<float *>(w);
   w += rnd(sizeof(float) * chunks * np);
   p.Hin = reinterpret_cast<__nv_bfloat16 *>(w);

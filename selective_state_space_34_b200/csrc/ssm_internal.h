@@ -57,6 +57,7 @@ struct SsdParams {
   __nv_bfloat16 *Hin;          // workspace: state entering each chunk, same shape, bf16
   float *cum_end;              // workspace: log-decay of each chunk (Bt, H, n_chunks)
   int *error;                  // workspace: set to 1 if a tensor-core wait timed out
+  void *const *timing_events;  // optional: 2 cudaEvent_t around the output kernel
 };
 cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream);
 size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);

@@ -656,8 +656,14 @@ static cudaError_t launch_ssd_t(const SsdParams &p, cudaStream_t s) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ssd_pass_kernel<P><<<(unsigned)(p.Bt * p.H * (p.N * P / 1024)), 256, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p.timing_events && p.timing_events[0] &&
+      (e = cudaEventRecord(static_cast<cudaEvent_t>(p.timing_events[0]), s)) != cudaSuccess)
+    return e;
   ssd_out_kernel<P, Tout><<<(unsigned)(grid / HG), kThr, s3, s>>>(p, HG);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p.timing_events && p.timing_events[1])
+    e = cudaEventRecord(static_cast<cudaEvent_t>(p.timing_events[1]), s);
+  return e;
 }
 
 size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N) {

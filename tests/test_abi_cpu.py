@@ -52,8 +52,8 @@ def _header_fields(struct):
     ("ssm_bwd_args", "BwdArgs", 208 + 17 * 8 + 8),
     # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
     ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
-    # 10 pointers, 5 int64, 4 int32, workspace pointer and size
-    ("ssm_ssd_args", "SsdArgs", 10 * 8 + 5 * 8 + 4 * 4 + 8 + 8),
+    # 10 pointers, 5 int64, 4 int32, workspace pointer and size, timing events
+    ("ssm_ssd_args", "SsdArgs", 10 * 8 + 5 * 8 + 4 * 4 + 8 + 8 + 8),
 ])
 def test_struct_layout_matches_header_field_order(struct, cls, size):
     ct = [f[0] for f in getattr(_abi, cls)._fields_]
