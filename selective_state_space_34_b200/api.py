@@ -300,12 +300,14 @@ def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = 
 
 def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplus: bool = True,
                 out_dtype=None, discretization: str = "zoh", return_state: bool = False,
-                check: bool = False):
+                check: bool = False, timing_events=None):
     """Mamba-2 state-space duality forward. x: (Bt, H, L, P) bf16; dt: (Bt, H, L) bf16; B, C:
     (Bt, L, N) bf16 shared by the heads; A_log, D, dt_bias: (H,) fp32; h0: (Bt, H, N, P) fp32.
     P and N must be 64 or 128. Returns y (Bt, H, L, P), or (y, h_last) with return_state.
     check=True synchronises the stream afterwards and raises SSMError (code SSM_ERR_TIMEOUT) if a
-    bounded wait for the tensor cores ran out."""
+    bounded wait for the tensor cores ran out. ``timing_events``: optional pair of
+    torch.cuda.Event(enable_timing=True), recorded once already; the library records them just
+    before and just after the output kernel (the last of its three launches)."""
     for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
         _need_cuda(n, t)
     for n, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
@@ -338,6 +340,10 @@ def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplu
         ws = torch.empty(need + 256, dtype=torch.uint8, device=x.device)
         a.workspace = (ws.data_ptr() + 255) & ~255
         a.workspace_bytes = need
+    ev_arr = None
+    if timing_events is not None:
+        ev_arr = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in timing_events])
+        a.timing_events = ctypes.cast(ev_arr, ctypes.c_void_p)
     _abi.check("ssm_ssd_fwd", lib.ssm_ssd_fwd(ctypes.byref(a), _stream_handle(x.device)))
     if check:
         _abi.check("ssm_ssd_check", lib.ssm_ssd_check(ctypes.byref(a), _stream_handle(x.device)))

@@ -139,3 +139,25 @@ def test_ssd_deterministic_and_empty():
                              e(t["B"], (2, 0, 128)), e(t["C"], (2, 0, 128)), h0=h0, **kw)
     torch.cuda.synchronize()
     assert y0.numel() == 0 and torch.equal(hl, h0)
+
+
+def test_ssd_timing_events_bracket_the_output_kernel():
+    """The optional event pair is recorded around the output kernel alone: its interval is positive
+    and shorter than the whole three-launch call."""
+    a = wl.generate_ssd(2, 16, 1024, 64, 128, seed=5)
+    t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev[:2]:
+        e.record()  # the handles exist before they are passed down
+    torch.cuda.synchronize()
+    ev[2].record()
+    y = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
+                        timing_events=ev[:2])
+    ev[3].record()
+    torch.cuda.synchronize()
+    kernel_ms, call_ms = ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3])
+    assert 0.0 < kernel_ms < call_ms
+    y2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)  # recording changes nothing in the result
