@@ -12,12 +12,14 @@
 //
 // Three kernels: ssd_state_kernel (S_c, one tcgen05 product per chunk and head), ssd_pass_kernel
 // (the carry over chunks, fp32, CUDA cores), ssd_out_kernel (C B^T and C H_{c-1} on the tensor
-// cores, the masked decay applied to C B^T in registers, then the product with X). Operands are
-// bf16 in shared memory in the canonical no-swizzle layouts (8 x 16-byte core matrices);
-// accumulators are fp32 in tensor memory with M = 128, so accumulator row i is TMEM lane i and
-// thread i of the 128-thread CTA owns it. One elected thread issues the MMAs; completion is
-// signalled through an mbarrier whose wait is bounded (on a timeout the kernel records an error
-// and still frees its tensor memory).
+// cores, the masked decay applied to C B^T in registers, then the product with X). The state and
+// output kernels take a group of up to 8 heads per CTA, since B, C and C B^T do not depend on the
+// head. Operands are bf16 in shared memory in the canonical no-swizzle layouts (8 x 16-byte core
+// matrices); accumulators are fp32 in tensor memory with M = 128, so accumulator row i is TMEM
+// lane i. A CTA has 256 threads: threads i and i + 128 (warps w and w + 4 reach the same 32 lanes)
+// own row i and split its columns. One elected thread issues the MMAs; completion is signalled
+// through an mbarrier whose wait is bounded (on a timeout the kernel records an error and still
+// frees its tensor memory).
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
