@@ -68,6 +68,16 @@ def test_ssd_shapes(P, N, L):
     _run(2, 3, L, P, N)
 
 
+@pytest.mark.parametrize("Bt,H,L,P,N,out", [
+    (1, 8, 300, 128, 128, torch.float32),   # 8 heads per CTA; fp32 rows of 512 B leave in two passes
+    (2, 4, 200, 128, 64, torch.bfloat16),   # 4 heads per CTA
+    (1, 8, 130, 64, 64, torch.float32),     # 8 heads, N = 64 (half the C H_in slices), ragged tail
+    (1, 6, 257, 64, 128, torch.bfloat16),   # 2 heads per CTA
+])
+def test_ssd_head_groups(Bt, H, L, P, N, out):
+    _run(Bt, H, L, P, N, out_dtype=out, carry=True)
+
+
 @pytest.mark.parametrize("variant", ["euler", "no_softplus", "bf16_out", "no_D", "carried_state"])
 def test_ssd_variants(variant):
     _run(1, 2, 257, 64, 128, euler=variant == "euler", softplus=variant != "no_softplus",
