@@ -311,9 +311,14 @@ ssm_fwd_kernel(const FwdParams p) {
         if (p.chunk_states && live && t0 + sb * kSub < te) {
           const int64_t kk = (t0 + sb * kSub) / kSub;
           float *dst = p.chunk_states + ((b * p.Dn + d) * p.n_ck + kk) * N;
+          if (NS == 4 && N % 4 == 0 && g * NS < N && (reinterpret_cast<uintptr_t>(p.chunk_states) & 15) == 0) {
+            // 16-byte aligned: an aligned base, rows of N floats with N a multiple of 4, lane offset g * 4
+            *reinterpret_cast<float4 *>(dst + g * NS) = make_float4(h[0], h[NS > 1 ? 1 : 0], h[NS > 2 ? 2 : 0], h[NS > 3 ? 3 : 0]);
+          } else {
 #pragma unroll
-          for (int j = 0; j < NS; j++)
-            if (g * NS + j < N) dst[g * NS + j] = h[j];
+            for (int j = 0; j < NS; j++)
+              if (g * NS + j < N) dst[g * NS + j] = h[j];
+          }
         }
       }
       __syncwarp();  // ud / yp are rewritten by the next block

@@ -110,6 +110,27 @@ def test_misaligned_views_take_the_scalar_path():
     assert_close("out", to_np(out), ref, *TOL[("bf16", "f32")])
 
 
+@pytest.mark.parametrize("Dn,N", [(4800, 16), (20, 16), (20, 12), (20, 5)])  # 4800: 4 states per lane
+def test_saved_states_into_a_misaligned_buffer(Dn, N):
+    """A caller's saved-state buffer need only be 4-byte aligned: one starting a float in gives the
+    same bits as an aligned one (16-byte stores only where base, row and lane offsets allow them)."""
+    import ctypes
+    from selective_state_space_34_b200 import _abi, api
+    w = wl.shaped("mamba130m_fwd", Bt=2, Dn=Dn, N=N, L=72)
+    t = dev_arrays(wl.generate(w), "bf16")
+    kw = param_kw(t)
+    ref = ssm.ssm_scan_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], save_states=True, **kw)
+    flat = torch.full((ref["chunk_states"].numel() + 1,), float("nan"), device="cuda")
+    out = torch.empty_like(ref["out"])
+    args, _ = api._fwd_args(t["x"], t["dt"], t["A_log"], t["B"], t["C"], kw["D"], kw["z"], kw["dt_bias"],
+                            kw["conv_w"], kw["conv_b"], True, ref["out"].dtype)
+    args.out, args.chunk_states = out.data_ptr(), flat[1:].data_ptr()
+    _abi.check("ssm_scan_fwd", _abi.load().ssm_scan_fwd(ctypes.byref(args), torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert torch.equal(flat[1:].view_as(ref["chunk_states"]), ref["chunk_states"])
+    assert torch.equal(out, ref["out"])
+
+
 def test_empty_problems_leave_outputs_alone():
     x = torch.zeros(2, 4, 0, device="cuda")
     out = ssm.ssm_scan_fwd(x, x, torch.zeros(4, 16, device="cuda"), torch.zeros(2, 16, 0, device="cuda"),
