@@ -545,7 +545,7 @@ def main():
     picks = []
     for i in range(4):
         b, d = i % Bt, (i * 997) % max(1, Dn - 4)
-        picks.append((b, d, out[b, d:d + 4].float().cpu().numpy(),
+        picks.append((b, d, out[b, d:d + 4].cpu().float().numpy(),
                       grads["dx"][b, d:d + 4].cpu().numpy() if backward else None))
     fwd_ms = float(np.mean([ev_f0[i].elapsed_time(ev_f1[i]) for i in range(args.steps)]))
     kern = {"ssm_fwd_kernel": fwd_ms}
