@@ -230,6 +230,33 @@ ssm_bwd_kernel(const BwdParams P) {
     }
     const int tb = g * EPL;  // first owned step (stage-local)
 
+    // the stage's saved start state, requested now so that phase A hides the load: the state
+    // after the previous chunk of SSM_STATE_CHUNK = TS steps, h0 for the first, else zero; one
+    // 16-byte load where base, row and lane offset allow it
+    float2 hs2[NH];
+    {
+      float *hs = reinterpret_cast<float *>(hs2);
+      const float *src = t0 > 0 ? states + ((b * p.Dn + d) * p.n_ck + (t0 / TS - 1)) * N
+                                : (p.h0 ? p.h0 + (b * p.Dn + d) * N : nullptr);
+      bool vec4 = false;
+      if constexpr (NS == 4) {
+        vec4 = N % 4 == 0 && src && live && g * NS < N &&
+               (reinterpret_cast<uintptr_t>(t0 > 0 ? states : p.h0) & 15) == 0;
+        if (vec4) {
+          const float4 v = *reinterpret_cast<const float4 *>(src + g * NS);
+          hs2[0] = make_float2(v.x, v.y);
+          hs2[1] = make_float2(v.z, v.w);
+        }
+      }
+      if (!vec4) {
+#pragma unroll
+        for (int j = 0; j < 2 * NH; j++) {
+          const int n = g * NS + j;
+          hs[j] = (j < NS && live && n < N && src) ? src[n] : 0.f;
+        }
+      }
+    }
+
     // (A) per-element values of the owned steps: (Delta, u, dy, dSiLU/dc) -> e3, (dDelta/dv,
     //     dout/dz) -> pe
     {
@@ -285,16 +312,7 @@ ssm_bwd_kernel(const BwdParams P) {
       float2 h2[NH];
       float *h = reinterpret_cast<float *>(h2);
 #pragma unroll
-      for (int j = 0; j < 2 * NH; j++) {
-        const int n = g * NS + j;
-        h[j] = 0.f;
-        if (j < NS && live && n < N) {
-          if (t0 > 0)  // the saved state after the previous chunk of SSM_STATE_CHUNK = TS steps
-            h[j] = states[((b * p.Dn + d) * p.n_ck + (t0 / TS - 1)) * N + n];
-          else if (p.h0)
-            h[j] = p.h0[(b * p.Dn + d) * N + n];
-        }
-      }
+      for (int q = 0; q < NH; q++) h2[q] = hs2[q];
       float *my0 = y0 + c * S::YC + g * S::YG;
 #pragma unroll
       for (int tq = 0; tq < TS; tq += 4) {

@@ -129,6 +129,15 @@ def test_saved_states_into_a_misaligned_buffer(Dn, N):
     torch.cuda.synchronize()
     assert torch.equal(flat[1:].view_as(ref["chunk_states"]), ref["chunk_states"])
     assert torch.equal(out, ref["out"])
+    # the backward reads such a buffer as well (16-byte loads only where aligned): same gradients
+    dout = torch.randn(out.shape, device="cuda", generator=torch.Generator("cuda").manual_seed(2)).to(t["x"].dtype)
+    g_al = ssm.ssm_scan_bwd(dout, t["x"], t["dt"], t["A_log"], t["B"], t["C"],
+                            chunk_states=ref["chunk_states"], **kw)
+    g_mis = ssm.ssm_scan_bwd(dout, t["x"], t["dt"], t["A_log"], t["B"], t["C"],
+                             chunk_states=flat[1:].view_as(ref["chunk_states"]), **kw)
+    torch.cuda.synchronize()
+    for k in g_al:
+        assert torch.equal(g_al[k], g_mis[k]), k
 
 
 def test_empty_problems_leave_outputs_alone():
