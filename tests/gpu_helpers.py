@@ -13,7 +13,6 @@ import numpy as np
 import torch
 
 import oracle
-import selective_state_space_34_b200 as ssm
 
 TOL = {
     ("bf16", "f32"): (2e-3, 1e-4),
