@@ -4,7 +4,6 @@ than the stated tolerance."""
 import os
 import sys
 
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
