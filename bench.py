@@ -66,16 +66,17 @@ def job_throughput(units_per_rank, world, steps, max_ms):
 
 
 def ncu_traffic(kernel, source):
-    """DRAM bytes per launch of `kernel` from profiles/ncu_traffic.md, or None when the recorded
+    """DRAM bytes per launch of `kernel` (dram__bytes_read.sum + dram__bytes_write.sum from one ncu
+    capture, stored in profiles/ncu_traffic.json with the command that took it), or None when the
     capture was taken on a different version of the kernel's source file."""
     import hashlib
     try:
         sha = hashlib.sha256(open(os.path.join(ROOT, "selective_state_space_34_b200", "csrc", source),
                                   "rb").read()).hexdigest()[:16]
-        for ln in open(os.path.join(ROOT, "profiles", "ncu_traffic.md")):
-            f = [x.strip() for x in ln.strip().strip("|").split("|")]
-            if len(f) == 3 and f[0] == kernel and f[1] == sha:
-                return int(f[2])
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f)["kernels"].get(kernel)
+        if rec and rec.get("source_sha256_16") == sha:
+            return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
     return None
@@ -94,24 +95,33 @@ def load_peaks():
 
 # ---- algorithmic bytes (the minimum the method must move; intermediates never touch HBM) -------
 
-def fwd_bytes(Bt, Dn, N, L, s_in, s_out, states=False):
+def fwd_bytes(Bt, Dn, N, L, s_in, s_out, n_states=0):
+    """The forward's algorithmic bytes (x, dt, z, B, C and the parameters in, out out), plus the
+    n_states saved chunk states per channel when the step saves them for the backward."""
     elems = Bt * Dn * L
     b = elems * (3 * s_in + s_out)              # x, dt, z in; out
     b += Bt * N * L * 2 * s_in                  # B, C (shared by all channels)
     b += Dn * (N + 4 + 4) * 4                   # A_log, D, dt_bias, conv taps + bias
-    if states:
-        b += Bt * Dn * ((L + 15) // 16) * N * 4  # chunk states for the backward
+    b += Bt * Dn * n_states * N * 4             # chunk states for the backward
     return b
 
 
-def bwd_bytes(Bt, Dn, N, L, s_in, states=True):
+def bwd_bytes(Bt, Dn, N, L, s_in):
+    """The backward's algorithmic bytes: x, dt, z, dout, B, C and the parameters in; dx, ddt, dz,
+    dB, dC and the parameter gradients out. The saved states and the per-tile dB / dC partials
+    are this implementation's own traffic (see bwd_overhead_bytes), not the method's."""
     elems = Bt * Dn * L
     b = elems * (4 * s_in + 3 * 4)              # x, dt, z, dout in; dx, ddt, dz out (fp32)
     b += Bt * N * L * (2 * s_in + 2 * 4)        # B, C in; dB, dC out (fp32)
     b += Dn * (N + 8) * 4 * 2                   # parameters in, parameter grads out
-    if states:
-        b += Bt * Dn * ((L + 15) // 16) * N * 4
     return b
+
+
+def bwd_overhead_bytes(Bt, Dn, N, n_states):
+    """Traffic of the backward kernel beyond the algorithmic bytes that follows from the interface:
+    the saved chunk states it reads (n_states per channel). Its scratch traffic (partial sums)
+    shows in the measured `traffic` against `algorithmic_bytes`."""
+    return {"saved_states_read": Bt * Dn * n_states * N * 4}
 
 
 # ---- clocks during the timed region -------------------------------------------------------------
@@ -438,7 +448,8 @@ def main():
     backward = w.backward
 
     out = torch.empty((Bt, Dn, L), dtype=odt, device=dev)
-    states = torch.empty((Bt, Dn, ssm.ssm_num_state_chunks(L), N), dtype=torch.float32, device=dev)
+    n_ck = ssm.ssm_num_state_chunks(L)
+    states = torch.empty((Bt, Dn, n_ck, N), dtype=torch.float32, device=dev)
     grads = None
     ws = None
     need = 0
@@ -569,7 +580,7 @@ def main():
 
     peaks = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fb = fwd_bytes(Bt, Dn, N, L, s_in, s_out, states=False)
+    fb = fwd_bytes(Bt, Dn, N, L, s_in, s_out)
     fwd_roof = {"bound": "hbm", "achieved": fb / (fo_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": fb / (fo_ms * 1e-3) / 1e9 / hbm,
                 "traffic": ncu_traffic("ssm_fwd_kernel", "ssm_fwd.cu") if (s_out == 2 and s_in == 2) else None,
@@ -591,12 +602,13 @@ def main():
 
     if backward:
         bms = kern["ssm_bwd_kernel"]
-        bb = bwd_bytes(Bt, Dn, N, L, s_in, states=True)
+        bb = bwd_bytes(Bt, Dn, N, L, s_in)
         roof = {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": bb / (bms * 1e-3) / 1e9 / hbm,
                 "traffic": ncu_traffic("ssm_bwd_kernel", "ssm_bwd.cu") if s_in == 2 else None,
                 "algorithmic_bytes": bb, "kernel": "ssm_bwd_kernel", "ms": bms,
-                "peak_source": peaks.get("source")}
+                "peak_source": peaks.get("source"),
+                "overhead_bytes": bwd_overhead_bytes(Bt, Dn, N, n_ck)}
     else:
         roof = dict(fwd_roof)
     # a split forward is three launches (segment summaries, carry, segments); a split backward
@@ -605,24 +617,30 @@ def main():
     launches_per_step = (3 if split else 1) + ((6 if split else 3) if backward else 0)
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, compute, D2H results ----
-    # Every step copies its inputs from pinned host memory and reads its results back. The copies
-    # of step i+1 travel on their own stream into a second device input set while step i computes,
-    # and the results return on a third stream, so a step costs the slowest of the three.
+    # Every step copies its inputs from pinned host memory and reads all of its results back (the
+    # output and, with the backward, every gradient). Copies in and out run on their own streams,
+    # so a step costs the slowest of the three.
     names_in = [k for k in ("x", "dt", "z", "B", "C") + (("dout",) if backward else ()) if T[k] is not None]
     host = {k: torch.empty(T[k].shape, dtype=T[k].dtype, pin_memory=True) for k in names_in}
     for k in names_in:
         host[k].copy_(T[k].cpu())
     h2d = sum(host[k].numel() * host[k].element_size() for k in names_in)
-    res_names = ["dA_log", "dB", "dC", "dD", "ddt_bias", "dconv_w", "dconv_b"] if backward else []
+    res_names = (["dx", "ddt", "dz", "dA_log", "dB", "dC", "dD", "ddt_bias", "dconv_w", "dconv_b"]
+                 if backward else [])
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     host_res = {k: torch.empty(grads[k].shape, dtype=torch.float32, pin_memory=True) for k in res_names}
     d2h = host_out.numel() * host_out.element_size() + sum(v.numel() * 4 for v in host_res.values())
 
+    # two device sets of inputs and of results: while step i computes, step i+1's inputs arrive
+    # and step i-1's results leave
     T2 = {k: torch.empty_like(T[k]) for k in names_in}
+    out2 = torch.empty_like(out)
+    grads2 = {k: torch.empty_like(v) for k, v in grads.items()} if backward else None
     fa2 = _abi.FwdArgs.from_buffer_copy(fwd_args)
     for k in ("x", "dt", "z", "B", "C"):
         if k in T2:
             setattr(fa2, k, T2[k].data_ptr())
+    fa2.out = out2.data_ptr()
     ba2 = None
     if backward:
         ba2 = _abi.BwdArgs.from_buffer_copy(bw_args)
@@ -630,9 +648,11 @@ def main():
             if k in T2:
                 setattr(ba2.fwd, k, T2[k].data_ptr())
         ba2.dout = T2["dout"].data_ptr()
-    sets = [(T, fwd_args, bw_args if backward else None), (T2, fa2, ba2)]
+        for k, v in grads2.items():
+            setattr(ba2, k, v.data_ptr())
+    sets = [(T, fwd_args, bw_args if backward else None, out, grads), (T2, fa2, ba2, out2, grads2)]
     h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_ready, ev_free, ev_comp, ev_back = [E(), E()], [E(), E()], E(), E()
+    ev_ready, ev_done, ev_back = [E(), E()], [E(), E()], [E(), E()]
 
     def run_step(fa, ba):
         _abi.check("ssm_scan_fwd", lib.ssm_scan_fwd(ctypes.byref(fa), s.cuda_stream))
@@ -641,28 +661,28 @@ def main():
             _abi.check("ssm_scan_bwd", lib.ssm_scan_bwd(ctypes.byref(ba), s.cuda_stream))
 
     def e2e_run(n):
-        for ev in ev_free:
-            ev.record(s)
-        ev_back.record(s)
+        for j in range(2):
+            ev_done[j].record(s)
+            ev_back[j].record(s)
         for i in range(n):
-            Tk, fa, ba = sets[i % 2]
-            h2d_s.wait_event(ev_free[i % 2])          # step i-2 is done with this input set
+            Tk, fa, ba, ok, gk = sets[i % 2]
+            h2d_s.wait_event(ev_done[i % 2])          # step i-2 is done with this input set
             with torch.cuda.stream(h2d_s):
                 for k in names_in:
                     Tk[k].copy_(host[k], non_blocking=True)
             ev_ready[i % 2].record(h2d_s)
             s.wait_event(ev_ready[i % 2])
-            s.wait_event(ev_back)                     # step i-1's results have been read out
+            s.wait_event(ev_back[i % 2])              # step i-2's results have been read out
             run_step(fa, ba)
-            ev_free[i % 2].record(s)
-            ev_comp.record(s)
-            d2h_s.wait_event(ev_comp)
+            ev_done[i % 2].record(s)
+            d2h_s.wait_event(ev_done[i % 2])
             with torch.cuda.stream(d2h_s):
-                host_out.copy_(out, non_blocking=True)
+                host_out.copy_(ok, non_blocking=True)
                 for k in res_names:
-                    host_res[k].copy_(grads[k], non_blocking=True)
-            ev_back.record(d2h_s)
-        s.wait_event(ev_back)
+                    host_res[k].copy_(gk[k], non_blocking=True)
+            ev_back[i % 2].record(d2h_s)
+        for j in range(2):
+            s.wait_event(ev_back[j])
 
     e2e_run(3)
     torch.cuda.synchronize()
@@ -676,7 +696,8 @@ def main():
     e2e = {"value": job_throughput(es, world, args.e2e_steps, e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": e_ms / args.e2e_steps,
-           "overlap": "inputs of step i+1 copied while step i computes; results read back on a third stream"}
+           "overlap": "two device sets of inputs and results: step i+1's inputs copied in and step "
+                      "i-1's results (out and every gradient) copied out while step i computes"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -701,7 +722,7 @@ def main():
                        "in_dtype": w.in_dtype, "out_dtype": args.out_dtype,
                        "step": "fwd(save states)+bwd" if backward else "fwd",
                        "l2": "inputs larger than L2 (per-step working set %.2f GB)"
-                             % ((fwd_bytes(Bt, Dn, N, L, s_in, s_out, backward)
+                             % ((fwd_bytes(Bt, Dn, N, L, s_in, s_out, n_ck if backward else 0)
                                  + (bwd_bytes(Bt, Dn, N, L, s_in) if backward else 0)) / 1e9),
                        "parallelism": "replica per GPU" if world > 1 else "single GPU",
                        "n_segments": args.n_segments},

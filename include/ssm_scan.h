@@ -28,8 +28,11 @@
  *
  * Conventions for every entry point:
  *  - Pointers named "device" are CUDA device (or managed) memory on the current device. The
- *    caller owns every buffer; the library allocates nothing on the device and keeps no global
- *    mutable state, so calls from several host threads on different streams are safe.
+ *    caller owns every buffer; the entry points allocate no device memory. Library state is
+ *    limited to a per-thread last-CUDA-error word (ssm_last_cuda_error) and, for
+ *    ssm_scan_bwd_noalloc only, one built-in scratch array per device with a per-device address
+ *    cache behind a mutex. Calls from several host threads on different streams are safe, except
+ *    that ssm_scan_bwd_noalloc calls must not overlap on one device (they share that array).
  *  - Layouts are dense, row-major, innermost axis last: activations (Bt, Dn, L) with L
  *    contiguous; B and C (Bt, N, L) with L contiguous; per-channel parameters fp32.
  *    conv_w is [Dn, K] (each channel's taps contiguous, tap 0 = the current token), i.e. the
@@ -266,10 +269,22 @@ typedef struct ssm_bwd_args {
 size_t ssm_bwd_workspace_size(const ssm_bwd_args *args);
 
 /*
+ * Workspace bytes from the forward arguments alone: for_bwd = 0 gives ssm_fwd_workspace_size(args);
+ * for_bwd != 0 gives ssm_bwd_workspace_size() of a backward whose fwd block is *args and which is
+ * handed saved states exactly when args->chunk_states is not NULL (the forward that saved them).
+ * The caller allocates the answer (256-byte aligned) and passes it as `workspace`. 0 when nothing
+ * is needed or the arguments are invalid.
+ */
+size_t ssm_workspace_size(const ssm_fwd_args *args, int32_t for_bwd);
+
+/*
  * Backward (vector-Jacobian product) of ssm_scan_fwd against `dout`: the reverse-time adjoint
  * recurrence lambda_t = C_t * dy_t + A_bar_{t+1} * lambda_{t+1} over the states recomputed from
- * chunk_states, with all parameter gradients. Deterministic: cross-channel and cross-batch sums
- * are reduced in a fixed order. Errors as ssm_scan_fwd, plus SSM_ERR_WORKSPACE.
+ * chunk_states, with all parameter gradients. Always deterministic -- there is no switch for it,
+ * and no faster non-deterministic variant: every cross-channel and cross-batch sum (dB, dC and the
+ * per-channel parameter gradients) is reduced in a fixed order without atomics, so the same
+ * inputs on the same device give bit-identical gradients on every run. Errors as ssm_scan_fwd,
+ * plus SSM_ERR_WORKSPACE.
  */
 ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream);
 
@@ -317,7 +332,9 @@ ssm_status ssm_scan_step(const ssm_step_args *args, void *stream);
  * requirement small). The first call on a device looks up the array's device address (a runtime
  * API call): make it before any stream capture on that device. All calls on a device share the
  * array, so calls that overlap on the GPU race; order them (one stream, or events). The call
- * allocates nothing (no cudaMalloc / cudaFree). Errors: as ssm_scan_bwd.
+ * allocates nothing (no cudaMalloc / cudaFree). Errors: as ssm_scan_bwd; SSM_ERR_CUDA also when
+ * the current device or the array's address cannot be read (ssm_last_cuda_error() says why), and
+ * SSM_ERR_UNSUPPORTED on a device index of 64 or more.
  */
 ssm_status ssm_scan_bwd_noalloc(const ssm_bwd_args *args, void *stream);
 

@@ -83,6 +83,7 @@ SIGNATURES = [
     ("ssm_scan_fwd", ctypes.c_int, [ctypes.POINTER(FwdArgs), ctypes.c_void_p]),
     ("ssm_fwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(FwdArgs)]),
     ("ssm_bwd_workspace_size", ctypes.c_size_t, [ctypes.POINTER(BwdArgs)]),
+    ("ssm_workspace_size", ctypes.c_size_t, [ctypes.POINTER(FwdArgs), ctypes.c_int32]),
     ("ssm_scan_bwd", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_bwd_noalloc", ctypes.c_int, [ctypes.POINTER(BwdArgs), ctypes.c_void_p]),
     ("ssm_scan_step", ctypes.c_int, [ctypes.POINTER(StepArgs), ctypes.c_void_p]),

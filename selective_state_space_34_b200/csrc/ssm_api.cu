@@ -29,6 +29,14 @@ ssm_status cuda_status(cudaError_t e) {
   return SSM_ERR_CUDA;
 }
 
+}  // namespace
+
+namespace ssm {
+int record_cuda_error_code(cudaError_t e) { return (int)cuda_status(e); }
+}  // namespace ssm
+
+namespace {
+
 size_t dtype_size(int32_t dt) { return dt == SSM_BF16 ? 2 : 4; }
 bool dtype_ok(int32_t dt) { return dt == SSM_F32 || dt == SSM_BF16; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -272,6 +280,16 @@ ssm_status ssm_scan_step(const ssm_step_args *a, void *stream) {
   p.euler = a->discretization == SSM_EULER ? 1 : 0;
   return cuda_status(ssm::launch_step(p, a->in_dtype == SSM_BF16, a->out_dtype == SSM_BF16,
                                       static_cast<cudaStream_t>(stream)));
+}
+
+size_t ssm_workspace_size(const ssm_fwd_args *args, int32_t for_bwd) {
+  if (!args) return 0;
+  if (!for_bwd) return ssm_fwd_workspace_size(args);
+  ssm_bwd_args b;
+  memset(&b, 0, sizeof(b));
+  b.fwd = *args;
+  b.chunk_states = args->chunk_states;
+  return ssm_bwd_workspace_size(&b);
 }
 
 size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {

@@ -114,6 +114,10 @@ struct BwdParams {
                                // before it, added into the previous segment's dx afterwards
 };
 
+// Maps a CUDA error to the C ABI's status and records it for ssm_last_cuda_error() on this host
+// thread (SSM_OK for cudaSuccess). The status type is the ABI's, passed as int here.
+int record_cuda_error_code(cudaError_t e);
+
 LaneLayout choose_layout(int64_t N, int64_t channels);
 int channels_per_cta(const LaneLayout &lay);
 

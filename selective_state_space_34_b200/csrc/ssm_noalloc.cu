@@ -43,14 +43,16 @@ ssm_status ssm_scan_bwd_noalloc(const ssm_bwd_args *args, void *stream) {
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSM_ERR_CUDA;
+  if (e != cudaSuccess) return (ssm_status)ssm::record_cuda_error_code(e);
+  if (dev < 0 || dev >= kMaxDevices) return SSM_ERR_UNSUPPORTED;  // beyond the address cache
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     if (!g_scratch_ptr[dev]) {
       void *p = nullptr;
       e = cudaGetSymbolAddress(&p, g_bwd_scratch);
-      if (e != cudaSuccess || p == nullptr) return SSM_ERR_CUDA;
+      if (e == cudaSuccess && p == nullptr) e = cudaErrorInvalidSymbol;
+      if (e != cudaSuccess) return (ssm_status)ssm::record_cuda_error_code(e);
       g_scratch_ptr[dev] = p;
     }
     scratch = g_scratch_ptr[dev];

@@ -145,6 +145,21 @@ def test_bwd_validation_codes(lib):
     assert lib.ssm_bwd_workspace_size(ctypes.byref(bw)) < full
 
 
+def test_workspace_size_from_forward_arguments(lib):
+    """ssm_workspace_size(fwd args, for_bwd): the forward's own size, or the backward's for a
+    backward with that fwd block, handed saved states exactly when fwd.chunk_states is set."""
+    for kw in (dict(), dict(n_segments=4, L=1000), dict(n_segments=-1, L=4096), dict(L=0)):
+        a = _args(**kw)
+        assert lib.ssm_workspace_size(ctypes.byref(a), 0) == lib.ssm_fwd_workspace_size(ctypes.byref(a))
+        for states in (0, 0xA000):
+            a.chunk_states = states
+            bw = _abi.BwdArgs()
+            bw.fwd = a
+            bw.chunk_states = states
+            assert lib.ssm_workspace_size(ctypes.byref(a), 1) == lib.ssm_bwd_workspace_size(ctypes.byref(bw))
+    assert lib.ssm_workspace_size(None, 0) == 0 and lib.ssm_workspace_size(None, 1) == 0
+
+
 def test_state_carry_validation_codes(lib):
     assert _fwd(lib, _args(discretization=2)) == 5
     assert _fwd(lib, _args(discretization=1, x=0x1001)) == 3   # Euler passes the flag check
