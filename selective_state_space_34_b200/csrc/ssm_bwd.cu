@@ -32,6 +32,19 @@
 
 namespace ssm {
 
+// 1: the dB / dC channel sum of the 4-lane, 4-state layout runs as a warp butterfly (below).
+#ifndef SSM_BWD_BFLY
+#define SSM_BWD_BFLY 1
+#endif
+// Resident CTAs per SM the backward is compiled for (its register budget: 65536 / (128 x this)).
+#ifndef SSM_BWD_MIN_CTAS
+#define SSM_BWD_MIN_CTAS 4
+#endif
+// 1: the adjoint recomputes A_bar on the bf16 path instead of reading it back from TMEM.
+#ifndef SSM_BWD_AREC
+#define SSM_BWD_AREC 0
+#endif
+
 template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr int CH = kThreads / G;
   static constexpr int NP = G * NS;
@@ -49,7 +62,16 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr int RBC = CHH * NP + 16;       // half-tile of channels (+16 words: banks)
   static constexpr int RBT = 2 * RBC + 4;         // one step
   static constexpr int RBW = RH * RBT;            // one quantity (dB or dC)
-  static constexpr uint32_t NCOLS = 32 * NS;      // TMEM: h and A_bar of TS steps x NS states
+  // With 4 lanes of 4 states per channel the channel sum runs as a warp butterfly (BFLY): each
+  // lane ends each step with the 8-channel sum of one (quantity, state), parked in a row of
+  // 4 warps x 32 lanes (+2 words: the per-stage cross-warp sum then reads without bank conflicts)
+  static constexpr bool BFLY = (G == 4 && NS == 4 && SSM_BWD_BFLY);
+  static constexpr int WPT = 4 * 32 + 2;
+  // AREC (bf16 path): TMEM keeps only h of the stage's steps and the adjoint recomputes A_bar
+  // from Delta (bitwise the same value: the same product and the same ex2); otherwise TMEM keeps
+  // h and A_bar (A_bar - 1 on the precise path). At least 32 columns per allocation.
+  static constexpr bool AREC = sizeof(Tin) == 2 && SSM_BWD_AREC;
+  static constexpr uint32_t NCOLS = (AREC ? (16 * NS < 32 ? 32 : 16 * NS) : 32 * NS);
   static constexpr size_t x_off = 0;
   static constexpr size_t dt_off = x_off + sizeof(Tin) * 2 * CH * XS;
   static constexpr size_t z_off = dt_off + sizeof(Tin) * 2 * CH * TS;
@@ -62,7 +84,7 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr size_t y1_off = y0_off + sizeof(float) * CH * YC;
   static constexpr size_t dcs_off = y1_off + (SHFL ? 0 : sizeof(float) * CH * YC);
   static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
-  static constexpr size_t slot_off = rb_off + sizeof(float) * 2 * RBW;
+  static constexpr size_t slot_off = rb_off + (BFLY ? sizeof(float) * TS * WPT : sizeof(float) * 2 * RBW);
   static constexpr size_t bytes = slot_off + 16;
   __host__ __device__ static constexpr int rb_index(int which, int tt, int c, int n) {
     return which * RBW + tt * RBT + (c / CHH) * RBC + (c % CHH) * NP + n;
@@ -86,7 +108,7 @@ template <int NS> __device__ __forceinline__ void store_states(float *dst, const
 // SEG: split-L pass 3 (a grid of segments x batch x channel tiles); without it the segment is
 // the whole sequence and its bounds are compile-time constants of the one-pass kernel.
 template <int G, int NS, typename Tin, bool EULER, bool SEG>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, SSM_BWD_MIN_CTAS)
 ssm_bwd_kernel(const BwdParams P) {
   using S = BwdSmem<G, NS, Tin>;
   constexpr int CH = S::CH, NP = S::NP, TS = S::TS, EPL = TS / G, RH = S::RH;
@@ -376,7 +398,7 @@ ssm_bwd_kernel(const BwdParams P) {
         *reinterpret_cast<float4 *>(my0 + tq) = make_float4(yq[0], yq[1], yq[2], yq[3]);
         __syncwarp();  // the TMEM stores are warp-collective
         tmem_st<GV>(th + tq * NS, hv);
-        tmem_st<GV>(ta + tq * NS, av);
+        if constexpr (!S::AREC) tmem_st<GV>(ta + tq * NS, av);
       }
     }
     tmem_wait_st();
@@ -398,8 +420,10 @@ ssm_bwd_kernel(const BwdParams P) {
     }
     __syncwarp();  // y0 is reused for the du partials
 
-    // (C) the adjoint backwards through the stage, one 4-step TMEM group per quarter; each
-    //     quarter's dB / dC partials are summed over the CTA's channels right after it
+    // (C) the adjoint backwards through the stage, one 4-step TMEM group per quarter. The dB / dC
+    //     partials are summed over the CTA's channels: with the butterfly, per step inside each
+    //     warp and once per stage across the 4 warps; otherwise through shared memory after
+    //     every quarter
     float duo[EPL], ddo[EPL];  // lane sums of du / dDelta of the owned steps (shuffle path)
 #pragma unroll
     for (int j = 0; j < EPL; j++) {
@@ -410,7 +434,10 @@ ssm_bwd_kernel(const BwdParams P) {
     for (int hf = TS / RH - 1; hf >= 0; hf--) {
       const int tq = hf * RH;
       float hv[GV], av[GV];
-      tmem_ld2<GV>(th + tq * NS, hv, ta + tq * NS, av);
+      if constexpr (S::AREC)
+        tmem_ld1<GV>(th + tq * NS, hv);
+      else
+        tmem_ld2<GV>(th + tq * NS, hv, ta + tq * NS, av);
       float duq[4], ddq[4];
 #pragma unroll
       for (int tt = 3; tt >= 0; tt--) {
@@ -428,7 +455,13 @@ ssm_bwd_kernel(const BwdParams P) {
           const float2 dl2 = make_float2(e.x, e.x), u2 = make_float2(e.y, e.y), dy2 = make_float2(e.z, e.z);
 #pragma unroll
           for (int q = 0; q < NH; q++) {
-            const float2 a2 = make_float2(av[tt * NS + 2 * q], av[tt * NS + 2 * q + 1]);
+            float2 a2;
+            if constexpr (S::AREC) {
+              const float2 x = __fmul2_rn(dl2, Ac2[q]);  // as in the recompute: same bits
+              a2 = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            } else {
+              a2 = make_float2(av[tt * NS + 2 * q], av[tt * NS + 2 * q + 1]);
+            }
             const float2 hs = make_float2(hv[tt * NS + 2 * q], hv[tt * NS + 2 * q + 1]);
             lam2[q] = __ffma2_rn(aN2[q], lam2[q], __fmul2_rn(Cv[q], dy2));         // lambda_t
             aN2[q] = a2;
@@ -454,10 +487,11 @@ ssm_bwd_kernel(const BwdParams P) {
           const float *Ct = reinterpret_cast<const float *>(Cv);
 #pragma unroll
           for (int j = 0; j < NS; j++) {
-            const float em1 = PRECISE ? av[tt * NS + j] : av[tt * NS + j] - 1.f;
+            const float aj = S::AREC ? ex2_approx(e.x * Acoef[j]) : av[tt * NS + j];
+            const float em1 = PRECISE ? aj : aj - 1.f;
             const float hs = hv[tt * NS + j];
             lam[j] = fmaf(aN[j], lam[j], Ct[j] * e.z);
-            aN[j] = PRECISE ? 1.f + av[tt * NS + j] : av[tt * NS + j];
+            aN[j] = PRECISE ? 1.f + aj : aj;
             const float em1n = EULER ? -e.x : em1 * nIA[j];
             const float nlb = lam[j] * (em1n * Bt[j]);
             ndu += nlb;
@@ -469,8 +503,29 @@ ssm_bwd_kernel(const BwdParams P) {
             dAl[j] = fmaf(e.y, nlb, fmaf(e.x, dterm, dAl[j]));
           }
         }
-        store_states<NS>(rb + S::rb_index(0, tt, c, g * NS), nB);
-        store_states<NS>(rb + S::rb_index(1, tt, c, g * NS), dCv);
+        if constexpr (S::BFLY) {
+          // reduce-scatter over the warp's 8 channels (lane bits 2, 3, 4): at each level a lane
+          // keeps half of its values, sends the other half to its partner and adds what it gets.
+          // Lane l ends with quantity l>>4 (0: -dB, 1: dC) of state g*4 + 2*bit3 + bit2.
+          const int lane = tid & 31;
+          const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+          float s4[4], s2[2];
+#pragma unroll
+          for (int k = 0; k < 4; k++) {
+            const float send = b4 ? nB[k] : dCv[k], keep = b4 ? dCv[k] : nB[k];
+            s4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+          }
+#pragma unroll
+          for (int k = 0; k < 2; k++) {
+            const float send = b3 ? s4[k] : s4[k + 2], keep = b3 ? s4[k + 2] : s4[k];
+            s2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+          }
+          const float send = b2 ? s2[0] : s2[1], keep = b2 ? s2[1] : s2[0];
+          rb[tl * S::WPT + (tid >> 5) * 32 + lane] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        } else {
+          store_states<NS>(rb + S::rb_index(0, tt, c, g * NS), nB);
+          store_states<NS>(rb + S::rb_index(1, tt, c, g * NS), dCv);
+        }
         if (S::SHFL) {
           // sum over the channel's G lanes; the step's owner keeps it
           float su = -ndu, sd = dd;
@@ -492,63 +547,90 @@ ssm_bwd_kernel(const BwdParams P) {
         *reinterpret_cast<float4 *>(y0 + c * S::YC + g * S::YG + tq) = make_float4(duq[0], duq[1], duq[2], duq[3]);
         *reinterpret_cast<float4 *>(y1 + c * S::YC + g * S::YG + tq) = make_float4(ddq[0], ddq[1], ddq[2], ddq[3]);
       }
-      __syncthreads();  // the quarter's dB / dC partials of every channel are in place
-      {
-        // every thread runs the same number of rounds, so the shuffles below see whole warps
-        // (threads without a column still take part in them)
-        constexpr int NQ = NP / 4;
-        constexpr int NGRP = 2 * RH * NQ;
-        // two threads per column: fewer shuffles than a wider split, and half the CTA's warps
-        // stay free (measured fastest on B200)
-        constexpr int SPLIT = NGRP >= kThreads ? 1 : 2;
-        constexpr int CPS = CH / SPLIT;
-        constexpr int ROUNDS = (NGRP * SPLIT + kThreads - 1) / kThreads;
-        const int part = tid % SPLIT;
-#pragma unroll
-        for (int r = 0; r < ROUNDS; r++) {
-          const int gi = (r * kThreads + tid) / SPLIT;
-          const bool ok = gi < NGRP;
-          const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
-          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
-          if (ok) {
-            if (SPLIT > 1) {
-              // this thread's channels lie in one half: walk them with a fixed stride
-              const float *src = rb + S::rb_index(which, tt, part * CPS, 4 * q);
-#pragma unroll 8
-              for (int ci = 0; ci < CPS; ci++) {
-                const float4 v = *reinterpret_cast<const float4 *>(src + ci * NP);
-                a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
-                a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
-              }
-            } else {
-#pragma unroll 4
-              for (int ci = 0; ci < CPS; ci++) {
-                const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, ci, 4 * q));
-                a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
-                a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
+      if constexpr (!S::BFLY) {
+        __syncthreads();  // the quarter's dB / dC partials of every channel are in place
+        {
+          // every thread runs the same number of rounds, so the shuffles below see whole warps
+          // (threads without a column still take part in them)
+          constexpr int NQ = NP / 4;
+          constexpr int NGRP = 2 * RH * NQ;
+          // two threads per column: fewer shuffles than a wider split, and half the CTA's warps
+          // stay free (measured fastest on B200)
+          constexpr int SPLIT = NGRP >= kThreads ? 1 : 2;
+          constexpr int CPS = CH / SPLIT;
+          constexpr int ROUNDS = (NGRP * SPLIT + kThreads - 1) / kThreads;
+          const int part = tid % SPLIT;
+  #pragma unroll
+          for (int r = 0; r < ROUNDS; r++) {
+            const int gi = (r * kThreads + tid) / SPLIT;
+            const bool ok = gi < NGRP;
+            const int which = gi / (RH * NQ), rem = gi % (RH * NQ), q = rem / RH, tt = rem % RH;
+            float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+            if (ok) {
+              if (SPLIT > 1) {
+                // this thread's channels lie in one half: walk them with a fixed stride
+                const float *src = rb + S::rb_index(which, tt, part * CPS, 4 * q);
+  #pragma unroll 8
+                for (int ci = 0; ci < CPS; ci++) {
+                  const float4 v = *reinterpret_cast<const float4 *>(src + ci * NP);
+                  a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
+                  a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
+                }
+              } else {
+  #pragma unroll 4
+                for (int ci = 0; ci < CPS; ci++) {
+                  const float4 v = *reinterpret_cast<const float4 *>(rb + S::rb_index(which, tt, ci, 4 * q));
+                  a01 = __fadd2_rn(a01, make_float2(v.x, v.y));
+                  a23 = __fadd2_rn(a23, make_float2(v.z, v.w));
+                }
               }
             }
-          }
-          float4 acc = make_float4(a01.x, a01.y, a23.x, a23.y);
-#pragma unroll
-          for (int off = 1; off < SPLIT; off <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-          }
-          const int64_t t = t0 + tq + tt;
-          if (ok && part == 0 && t < te) {
-            float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
-            const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
-            const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-            for (int k = 0; k < 4; k++)
-              if (4 * q + k < N) dst[(int64_t)(4 * q + k) * L] = sg * vals[k];
+            float4 acc = make_float4(a01.x, a01.y, a23.x, a23.y);
+  #pragma unroll
+            for (int off = 1; off < SPLIT; off <<= 1) {
+              acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+              acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+              acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+              acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+            }
+            const int64_t t = t0 + tq + tt;
+            if (ok && part == 0 && t < te) {
+              float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N) * L + t;
+              const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
+              const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+  #pragma unroll
+              for (int k = 0; k < 4; k++)
+                if (4 * q + k < N) dst[(int64_t)(4 * q + k) * L] = sg * vals[k];
+            }
           }
         }
+        __syncthreads();  // rb is rewritten by the next quarter
       }
-      __syncthreads();  // rb is rewritten by the next quarter
+    }
+    if constexpr (S::BFLY) {
+      // the stage's per-warp 8-channel sums -> this tile's dB / dC partials: thread (slot l, 4-step
+      // group tq) adds the 4 warps in order and writes 4 consecutive steps of one (quantity, state)
+      __syncthreads();
+      const int l = tid >> 2, tq = tid & 3;
+      const int which = l >> 4, n = (l & 3) * 4 + ((l >> 3) & 1) * 2 + ((l >> 2) & 1);
+      float acc[4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float *src = rb + (4 * tq + i) * S::WPT + l;
+        acc[i] = ((src[0] + src[32]) + src[64]) + src[96];
+      }
+      const int64_t t = t0 + 4 * tq;
+      if (n < N && t < te) {
+        const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
+        float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N + n) * L + t;
+        if (vec && t + 3 < te) {
+          *reinterpret_cast<float4 *>(dst) = make_float4(sg * acc[0], sg * acc[1], sg * acc[2], sg * acc[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            if (t + i < te) dst[i] = sg * acc[i];
+        }
+      }
     }
 
     __syncwarp();  // the du / dDelta partial rows (shared-memory path) are complete

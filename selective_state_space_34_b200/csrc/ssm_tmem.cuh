@@ -134,6 +134,30 @@ template <> __device__ __forceinline__ void tmem_ld2<16>(uint32_t a, float *va, 
     vb[i] = __uint_as_float(y[i]);
   }
 }
+// Load 16 consecutive columns of this thread's lane and wait for them.
+__device__ __forceinline__ void tmem_ld16(uint32_t a, float *va) {
+  uint32_t x[16];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+               "%10, %11, %12, %13, %14, %15}, [%16];"
+               : SSM_O(x, 0), SSM_O(x, 1), SSM_O(x, 2), SSM_O(x, 3), SSM_O(x, 4), SSM_O(x, 5),
+                 SSM_O(x, 6), SSM_O(x, 7), SSM_O(x, 8), SSM_O(x, 9), SSM_O(x, 10), SSM_O(x, 11),
+                 SSM_O(x, 12), SSM_O(x, 13), SSM_O(x, 14), SSM_O(x, 15) : "r"(a) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : SSM_W(x, 0), SSM_W(x, 1), SSM_W(x, 2), SSM_W(x, 3), SSM_W(x, 4), SSM_W(x, 5),
+                 SSM_W(x, 6), SSM_W(x, 7), SSM_W(x, 8), SSM_W(x, 9), SSM_W(x, 10), SSM_W(x, 11),
+                 SSM_W(x, 12), SSM_W(x, 13), SSM_W(x, 14), SSM_W(x, 15) :: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; i++) va[i] = __uint_as_float(x[i]);
+}
+// Same for 4 or 8 columns (the 1- and 2-state lane layouts).
+template <int NV> __device__ __forceinline__ void tmem_ld1(uint32_t a, float *va) {
+  if constexpr (NV == 16) {
+    tmem_ld16(a, va);
+  } else {
+    float dummy[NV];
+    tmem_ld2<NV>(a, va, a, dummy);
+  }
+}
 #undef SSM_O
 #undef SSM_W
 
