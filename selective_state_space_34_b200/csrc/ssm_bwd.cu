@@ -18,13 +18,14 @@
 //
 // Decomposition mirrors the forward: a CTA owns CH = 128/G channels of one batch element, lanes
 // hold NS states each, and the sequence is walked backwards in stages of 16 steps (one saved-state
-// chunk each): recompute the stage forward from its saved start state, keeping h_t and a_t of every
-// step in the thread's lane of tensor memory (TMEM, otherwise idle here) instead of registers, then
-// run the adjoint backwards through it one 4-step group at a time. Moving that trajectory out of
-// the register file is what lets four CTAs share an SM. dB and dC are summed over the CTA's
-// channels in shared memory after every 4 steps and written as per-tile partials; a second kernel
-// adds the tiles (and the per-batch partials of the per-channel parameter gradients) in a fixed
-// order, so the result is deterministic.
+// chunk each): recompute the stage forward from its saved start state, keeping h_t of every step
+// (and a_t on the precise path; the fast path recomputes it) in the thread's lane of tensor memory
+// (TMEM, otherwise idle here) instead of registers, then run the adjoint backwards through it one
+// 4-step group at a time. Moving that trajectory out of the register file is what lets four CTAs
+// share an SM. dB and dC are summed over the CTA's channels (a warp butterfly per step and one
+// cross-warp sum per stage, or a shared-memory sum after every 4 steps for the other lane layouts)
+// and written as per-tile partials; a second kernel adds the tiles (and the per-batch partials of
+// the per-channel parameter gradients) in a fixed order, so the result is deterministic.
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
@@ -40,9 +41,11 @@ namespace ssm {
 #ifndef SSM_BWD_MIN_CTAS
 #define SSM_BWD_MIN_CTAS 4
 #endif
-// 1: the adjoint recomputes A_bar on the bf16 path instead of reading it back from TMEM.
+// 1: the adjoint recomputes A_bar on the bf16 path instead of reading it back from TMEM (one
+// more exp per element-state on a pipe the backward keeps ~15% busy, 16 fewer live registers;
+// measured 2.63 -> 2.46 ms on 4x4096x16x4096, bit-identical gradients).
 #ifndef SSM_BWD_AREC
-#define SSM_BWD_AREC 0
+#define SSM_BWD_AREC 1
 #endif
 
 template <int G, int NS, typename Tin> struct BwdSmem {
@@ -56,7 +59,10 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr int YC = G * YG + 4;
   // with 4 lanes per channel the du / dDelta lane sums go through shuffles (no shared rows)
   static constexpr bool SHFL = (G == 4);
-  static constexpr int DCS = TS + 8;              // dc row: this stage, then the next stage's 3
+  // dc row: this stage, then the next stage's 3. With 4 lanes per channel each lane stores its 4
+  // values and reads its 8-value window as 16-byte vectors; a stride of 48 floats (16 mod 32)
+  // keeps those accesses free of bank conflicts
+  static constexpr int DCS = (G == 4) ? 48 : TS + 8;
   static constexpr int RH = 4;                    // steps per cross-channel reduction
   static constexpr int CHH = CH / 2;
   static constexpr int RBC = CHH * NP + 16;       // half-tile of channels (+16 words: banks)
@@ -328,8 +334,8 @@ ssm_bwd_kernel(const BwdParams P) {
     }
     __syncwarp();
 
-    // (B) recompute the stage forward from its saved start state; h and A_bar of every step go
-    //     to TMEM, the readout partials to y0
+    // (B) recompute the stage forward from its saved start state; h (and A_bar unless the
+    //     adjoint recomputes it) of every step go to TMEM, the readout partials to y0
     {
       float2 h2[NH];
       float *h = reinterpret_cast<float *>(h2);
@@ -466,8 +472,10 @@ ssm_bwd_kernel(const BwdParams P) {
             lam2[q] = __ffma2_rn(aN2[q], lam2[q], __fmul2_rn(Cv[q], dy2));         // lambda_t
             aN2[q] = a2;
             // kb = -dB_bar/dB: (A_bar - 1)(-1/A) for the exact ZOH, -Delta for Euler
+            // (A_bar - 1)(-1/A) as one fused multiply-add: A_bar - 1 is exact in fp32, so this is
+            // the same single rounding as the product
             const float2 em1n = EULER ? make_float2(-e.x, -e.x)
-                                      : __fmul2_rn(__fadd2_rn(a2, make_float2(-1.f, -1.f)), nIA2[q]);
+                                      : __ffma2_rn(a2, nIA2[q], make_float2(-nIA2[q].x, -nIA2[q].y));
             const float2 k = __fmul2_rn(lam2[q], em1n);
             const float2 nlb = __fmul2_rn(k, Bv[q]);                                // -lambda B_bar
             ndu2 = __fadd2_rn(ndu2, nlb);
@@ -675,12 +683,15 @@ ssm_bwd_kernel(const BwdParams P) {
         accDtb += dtv[j];
         dcv[j] = du * e.w;
         if (has_conv) {
-          dcs[c * S::DCS + tb + j] = dcv[j];
+          if (EPL != 4) dcs[c * S::DCS + tb + j] = dcv[j];
           accCb += dcv[j];
 #pragma unroll
           for (int k = 0; k < 4; k++) accW[k] = fmaf(dcv[j], xw[j + 4 - k], accW[k]);
         }
       }
+      if (EPL == 4 && has_conv)
+        *reinterpret_cast<float4 *>(dcs + c * S::DCS + tb) = make_float4(dcv[0], dcv[EPL > 1 ? 1 : 0],
+                                                                         dcv[EPL > 2 ? 2 : 0], dcv[EPL > 3 ? 3 : 0]);
       if (live) {
         const int64_t roff = (b * p.Dn + d) * L;
         if (has_z && P.dz) store_run<float, EPL>(P.dz + roff, t0 + tb, te, dzv, vec);
@@ -695,13 +706,27 @@ ssm_bwd_kernel(const BwdParams P) {
       __syncwarp();
       {
         float dxv[EPL];
+        if constexpr (EPL == 4) {
+          // dc of the owned steps and the 4 after them (the next lane's, or the halo)
+          const float4 lo = *reinterpret_cast<const float4 *>(dcs + c * S::DCS + tb);
+          const float4 hi = *reinterpret_cast<const float4 *>(dcs + c * S::DCS + tb + 4);
+          const float dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-        for (int j = 0; j < EPL; j++) {
-          const int t = tb + j;
-          float acc = 0.f;
+          for (int j = 0; j < EPL; j++) {
+            float acc = 0.f;
 #pragma unroll
-          for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
-          dxv[j] = acc;
+            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dw[j + k], acc);
+            dxv[j] = acc;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < EPL; j++) {
+            const int t = tb + j;
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; k++) acc = fmaf(w4[k], dcs[c * S::DCS + t + k], acc);
+            dxv[j] = acc;
+          }
         }
         if (live && P.dx) store_run<float, EPL>(P.dx + (b * p.Dn + d) * L, t0 + tb, te, dxv, vec);
       }
