@@ -406,6 +406,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--n-segments", type=int, default=0,
                     help="split-L for the forward: 0 one pass, k up to k segments, -1 automatic")
+    ap.add_argument("--scan-form", default="lanes", choices=["lanes", "chunked"],
+                    help="layout of a one-pass forward scan: states over lanes, or chunked in time")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -472,7 +474,8 @@ def main():
 
     # argument structs built once; each step is then plain C-ABI calls on the current stream
     fwd_args, _ = api._fwd_args(T["x"], T["dt"], T["A_log"], T["B"], T["C"], kw["D"], kw["z"],
-                                kw["dt_bias"], kw["conv_w"], kw["conv_b"], True, odt)
+                                kw["dt_bias"], kw["conv_w"], kw["conv_b"], True, odt,
+                                scan_form=args.scan_form)
     fwd_args.out = out.data_ptr()
     fwd_args.chunk_states = states.data_ptr() if backward else None
     ws_f = None
@@ -725,7 +728,7 @@ def main():
                              % ((fwd_bytes(Bt, Dn, N, L, s_in, s_out, n_ck if backward else 0)
                                  + (bwd_bytes(Bt, Dn, N, L, s_in) if backward else 0)) / 1e9),
                        "parallelism": "replica per GPU" if world > 1 else "single GPU",
-                       "n_segments": args.n_segments},
+                       "n_segments": args.n_segments, "scan_form": args.scan_form},
             "roofline": roof,
             "alu_roofline": alu_roof("ssm_bwd_kernel" if backward else "ssm_fwd_kernel",
                                      kern["ssm_bwd_kernel"] if backward else fo_ms),

@@ -78,6 +78,16 @@ typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
  * "Selective Mamba", step). A_bar = exp(Delta * A) in both. */
 typedef enum ssm_discretization { SSM_ZOH = 0, SSM_EULER = 1 } ssm_discretization;
 
+/* How the forward's one-pass scan is laid out on the GPU (both compute the same outputs; fp32
+ * rounding differs). SSM_SCAN_LANES: a channel's states are spread over lanes that each walk the
+ * whole sequence in time order. SSM_SCAN_CHUNKED: lanes own consecutive time steps; each 64-step
+ * chunk of a channel is scanned in parallel -- every lane runs its 8 steps from a zero state, an
+ * associative warp-shuffle scan of the (product of A_bar, end state) pairs gives every lane the
+ * state entering its steps ("State-Space Models & Long-Context Sequence Architectures (Mamba)",
+ * Lab 3; "state-space models", "One recurrence, one convolution"), and the chunk's end state is
+ * carried into the next chunk. Split-L calls (ssm_fwd_args.n_segments) use the lane layout. */
+typedef enum ssm_scan_form { SSM_SCAN_LANES = 0, SSM_SCAN_CHUNKED = 1 } ssm_scan_form;
+
 /* Time steps between saved states (chunk_states) and of the backward's recompute blocks. */
 #define SSM_STATE_CHUNK 16
 
@@ -142,13 +152,15 @@ typedef struct ssm_fwd_args {
   void *workspace;       /* device scratch of at least ssm_fwd_workspace_size() bytes, 256-byte
                             aligned, when the call splits L; may be NULL otherwise */
   size_t workspace_bytes;
+  int32_t scan_form;     /* ssm_scan_form of a one-pass call (0 = SSM_SCAN_LANES) */
 } ssm_fwd_args;
 
 /*
  * Forward selective scan with the causal depthwise conv1d + SiLU fused in front and the SiLU(z)
  * gate fused behind: computes every output listed in ssm_fwd_args on `stream`.
  * Errors: SSM_ERR_NULL (x, dt, A_log, B, C or out NULL), SSM_ERR_SHAPE (also n_segments < -1),
- * SSM_ERR_ALIGN, SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED (N > 64, K outside 1..4), SSM_ERR_WORKSPACE
+ * SSM_ERR_ALIGN, SSM_ERR_DTYPE, SSM_ERR_UNSUPPORTED (N > 64, K outside 1..4, an unknown
+ * discretization or scan_form), SSM_ERR_WORKSPACE
  * (a split-L call whose workspace is NULL, too small or not 256-byte aligned), SSM_ERR_CUDA.
  */
 ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream);

@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 
 SSM_F32, SSM_BF16 = 0, 1
 SSM_ZOH, SSM_EULER = 0, 1
+SSM_SCAN_LANES, SSM_SCAN_CHUNKED = 0, 1
 SSM_STATE_CHUNK = 16
 SSM_NOALLOC_SCRATCH_BYTES = 64 << 20
 SSM_ERR_TIMEOUT = 8
@@ -33,7 +34,7 @@ class FwdArgs(ctypes.Structure):
         ("h0", ctypes.c_void_p), ("conv_hist", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
         ("conv_hist_out", ctypes.c_void_p), ("discretization", ctypes.c_int32),
         ("n_segments", ctypes.c_int32), ("workspace", ctypes.c_void_p),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("workspace_bytes", ctypes.c_size_t), ("scan_form", ctypes.c_int32),
     ]
 
 

@@ -49,8 +49,11 @@ def ssm_num_state_chunks(L: int) -> int:
 _DISC = {"zoh": _abi.SSM_ZOH, "euler": _abi.SSM_EULER}
 
 
+_SCAN = {"lanes": _abi.SSM_SCAN_LANES, "chunked": _abi.SSM_SCAN_CHUNKED}
+
+
 def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
-              discretization="zoh", h0=None, conv_hist=None):
+              discretization="zoh", h0=None, conv_hist=None, scan_form="lanes"):
     for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
         _need_cuda(n, t)
     if x.dtype not in _DT:
@@ -92,6 +95,9 @@ def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
     if discretization not in _DISC:
         raise ValueError("discretization must be 'zoh' or 'euler'")
     a.discretization = _DISC[discretization]
+    if scan_form not in _SCAN:
+        raise ValueError("scan_form must be 'lanes' or 'chunked'")
+    a.scan_form = _SCAN[scan_form]
     if h0 is not None:
         _opt("h0", h0, torch.float32)
         if tuple(h0.shape) != (Bt, Dn, N):
@@ -109,16 +115,17 @@ def ssm_scan_fwd(x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=None, 
                  delta_softplus: bool = True, out_dtype=None, save_states: bool = False,
                  return_u: bool = False, out: Optional[torch.Tensor] = None,
                  discretization: str = "zoh", h0=None, conv_hist=None, return_state: bool = False,
-                 n_segments: int = 0):
+                 n_segments: int = 0, scan_form: str = "lanes"):
     """Fused forward. Returns ``out`` or a dict with ``out`` and, when asked, ``chunk_states``
     ((Bt, Dn, ceil(L/16), N) fp32, for ssm_scan_bwd), ``u`` (the scan input), and ``h_last`` /
     ``conv_hist`` (the state to carry into the next chunk). ``h0`` / ``conv_hist`` carry the state
     in from a previous chunk; ``discretization`` is "zoh" (exact) or "euler" (Delta * B).
     ``n_segments`` splits the sequence across CTAs (0/1: one pass; k >= 2: up to k segments;
     -1: the library decides from the device and the shape); the scratch it needs is allocated
-    here."""
+    here. ``scan_form`` lays a one-pass scan out as "lanes" (a channel's states over lanes, each
+    walking the sequence) or "chunked" (lanes over time steps, a warp-shuffle scan per chunk)."""
     a, od = _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
-                      discretization, h0, conv_hist)
+                      discretization, h0, conv_hist, scan_form)
     Bt, Dn, L = x.shape
     N = A_log.shape[1]
     if out is None:
@@ -187,14 +194,19 @@ def ssm_scan_bwd(dout, x, dt, A_log, B, C, D=None, z=None, dt_bias=None, conv_w=
                  conv_b=None, delta_softplus: bool = True, chunk_states=None,
                  workspace: Optional[torch.Tensor] = None, grads: Optional[Dict] = None,
                  timing_events=None, discretization: str = "zoh", h0=None, conv_hist=None,
-                 dh_last=None, state_grads: bool = False, n_segments: int = 0):
+                 dh_last=None, state_grads: bool = False, n_segments: int = 0,
+                 scan_form: str = "lanes"):
     """Backward. Returns a dict of fp32 gradients: dx, ddt, dA_log, dB, dC, and dD / ddt_bias /
     dz / dconv_w / dconv_b where the corresponding input exists. ``workspace`` (uint8, at least
     ssm_bwd_workspace_size bytes) may be passed to avoid an allocation per call.
     ``timing_events``: optional pair of recorded-once torch.cuda.Event(enable_timing=True); the
-    library records them just before and just after its main backward kernel."""
+    library records them just before and just after its main backward kernel. ``scan_form``
+    selects the forward layout used to recompute the chunk states when none are passed."""
     bw = _bwd_struct(dout, x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus,
                      chunk_states, discretization, h0, conv_hist, dh_last)
+    if scan_form not in _SCAN:
+        raise ValueError("scan_form must be 'lanes' or 'chunked'")
+    bw.fwd.scan_form = _SCAN[scan_form]
     Bt, Dn, L = x.shape
     N = A_log.shape[1]
     dev = x.device

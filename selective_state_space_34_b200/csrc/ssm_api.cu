@@ -53,6 +53,7 @@ ssm_status check_fwd(const ssm_fwd_args *a, bool need_out, bool *empty) {
   if (!a) return SSM_ERR_NULL;
   if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SSM_ERR_DTYPE;
   if (a->discretization != SSM_ZOH && a->discretization != SSM_EULER) return SSM_ERR_UNSUPPORTED;
+  if (a->scan_form != SSM_SCAN_LANES && a->scan_form != SSM_SCAN_CHUNKED) return SSM_ERR_UNSUPPORTED;
   if (a->Bt < 0 || a->Dn < 0 || a->N < 0 || a->L < 0) return SSM_ERR_SHAPE;
   if (a->Dn == 0 || a->N == 0) return SSM_ERR_SHAPE;  // empty internal axes are rejected
   if (a->conv_w && a->K <= 0) return SSM_ERR_SHAPE;
@@ -134,6 +135,7 @@ ssm::FwdParams make_fwd_params(const ssm_fwd_args *a, int vec) {
   p.delta_softplus = a->delta_softplus ? 1 : 0;
   p.vec = vec;
   p.euler = a->discretization == SSM_EULER ? 1 : 0;
+  p.chunked = a->scan_form == SSM_SCAN_CHUNKED ? 1 : 0;
   p.h0 = a->h0;
   p.conv_hist = a->conv_w ? a->conv_hist : nullptr;
   p.h_last = a->h_last;

@@ -487,6 +487,7 @@ SegPlan plan_segments(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int requeste
 }
 
 cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream) {
+  if (p.n_seg <= 1 && p.chunked) return launch_fwd_tp(p, in_bf16, out_bf16, stream);
   if (p.n_seg <= 1) {
     FwdParams q = p;
     q.n_seg = 1;

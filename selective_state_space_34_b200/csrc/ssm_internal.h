@@ -32,6 +32,7 @@ struct FwdParams {
   int delta_softplus;
   int vec;  // 1: rows are 16-byte aligned, stage with cp.async and store with vector stores
   int euler;  // input discretisation: 0 exact ZOH, 1 Delta * B
+  int chunked;  // one-pass scan layout: 0 states over lanes (ssm_fwd.cu), 1 chunked in time (ssm_fwd_tp.cu)
   const float *h0;        // (Bt, Dn, N) or null
   const void *conv_hist;  // (Bt, Dn, K-1) in-dtype or null
   float *h_last;          // (Bt, Dn, N) or null
@@ -122,6 +123,8 @@ LaneLayout choose_layout(int64_t N, int64_t channels);
 int channels_per_cta(const LaneLayout &lay);
 
 cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
+// The time-parallel forward (ssm_fwd_tp.cu): one pass, the same outputs as launch_fwd.
+cudaError_t launch_fwd_tp(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
 size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg);
 cudaError_t launch_step(const StepParams &p, int in_bf16, int out_bf16, cudaStream_t stream);

@@ -46,10 +46,10 @@ def _header_fields(struct):
 
 
 @pytest.mark.parametrize("struct,cls,size", [
-    # 18 pointers, 4 int64, 6 int32, one size
-    ("ssm_fwd_args", "FwdArgs", 18 * 8 + 4 * 8 + 6 * 4 + 8),
+    # 18 pointers, 4 int64, 7 int32, one size (+4 bytes of tail padding)
+    ("ssm_fwd_args", "FwdArgs", 18 * 8 + 4 * 8 + 7 * 4 + 8 + 4),
     # the forward block, 17 pointers and one size
-    ("ssm_bwd_args", "BwdArgs", 208 + 17 * 8 + 8),
+    ("ssm_bwd_args", "BwdArgs", 216 + 17 * 8 + 8),
     # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
     ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
     # 10 pointers, 5 int64, 4 int32, workspace pointer and size, timing events
@@ -107,6 +107,8 @@ def test_fwd_validation_codes(lib):
     assert _fwd(lib, _args(in_dtype=1, x=0x1001)) == 3
     assert _fwd(lib, _args(A_log=0x3002)) == 3
     assert _fwd(lib, _args(out_dtype=1, out=0x6001)) == 3
+    assert _fwd(lib, _args(scan_form=2)) == 5   # unknown scan layout
+    assert _fwd(lib, _args(discretization=2)) == 5
 
 
 def test_empty_problems_are_noops(lib):

@@ -60,13 +60,13 @@ def _to_host(t):
 
 # ---- forward ------------------------------------------------------------------------------------
 
-def _full_forward(name, out_dtype, n_segments, per=64):
+def _full_forward(name, out_dtype, n_segments, per=64, scan_form="lanes"):
     w = wl.WORKLOADS[name]
     a = wl.generate(w)
     t = dev_arrays(a, w.in_dtype)
     tdt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
     out = ssm.ssm_scan_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], out_dtype=tdt,
-                           n_segments=n_segments, **param_kw(t, w.conv, w.gate))
+                           n_segments=n_segments, scan_form=scan_form, **param_kw(t, w.conv, w.gate))
     torch.cuda.synchronize()
     got = _to_host(out)
     del out, t
@@ -105,6 +105,12 @@ def test_mamba1p4b_every_element(out_dtype):
 def test_long_context_every_element(n_segments):
     # 1 x 5120 x 16 x 65536: one pass, and the automatic split (8 segments on B200)
     _full_forward("long_fwd", "bf16", n_segments, per=32)
+
+
+@pytest.mark.parametrize("name,per", [("mamba1p4b_fwd", 64), ("long_fwd", 32)])
+def test_chunked_layout_every_element(name, per):
+    # the chunked (time-parallel) scan layout, one pass, bf16 out
+    _full_forward(name, "bf16", 0, per=per, scan_form="chunked")
 
 
 # ---- forward + backward step --------------------------------------------------------------------
