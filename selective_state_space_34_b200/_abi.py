@@ -12,7 +12,7 @@ SSM_F32, SSM_BF16 = 0, 1
 SSM_ZOH, SSM_EULER = 0, 1
 SSM_SCAN_LANES, SSM_SCAN_CHUNKED = 0, 1
 SSM_STATE_CHUNK = 16
-SSM_NOALLOC_SCRATCH_BYTES = 64 << 20
+SSM_NOALLOC_SCRATCH_BYTES = 72 << 20
 SSM_ERR_TIMEOUT = 8
 
 STATUS = {

@@ -294,15 +294,25 @@ size_t ssm_workspace_size(const ssm_fwd_args *args, int32_t for_bwd) {
   return ssm_bwd_workspace_size(&b);
 }
 
-size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) {
+size_t ssm_bwd_workspace_size(const ssm_bwd_args *args) { return ssm::bwd_workspace_for(args, 1); }
+
+ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
+  return ssm::scan_bwd_clustered(args, stream, 1);
+}
+
+}  // extern "C"
+
+namespace ssm {
+
+size_t bwd_workspace_for(const ssm_bwd_args *args, int max_cluster) {
   if (!args) return 0;
   const ssm_fwd_args *a = &args->fwd;
   if (a->Bt <= 0 || a->L <= 0 || a->Dn <= 0 || a->N <= 0 || a->n_segments < -1) return 0;
-  return ssm::bwd_workspace_bytes(a->Bt, a->Dn, a->N, a->L, args->chunk_states == nullptr,
-                                  fwd_plan(a).n_seg);
+  return bwd_workspace_bytes(a->Bt, a->Dn, a->N, a->L, args->chunk_states == nullptr,
+                             fwd_plan(a).n_seg, max_cluster);
 }
 
-ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
+ssm_status scan_bwd_clustered(const ssm_bwd_args *args, void *stream, int max_cluster) {
   SSM_RANGE("ssm_scan_bwd");
   if (!args) return SSM_ERR_NULL;
   bool empty = false;
@@ -339,7 +349,7 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
                          args->dh_last, args->dh0, args->dconv_hist};
   for (const void *p : g32)
     if (p && !aligned(p, 4)) return SSM_ERR_ALIGN;
-  const size_t need = ssm_bwd_workspace_size(args);
+  const size_t need = bwd_workspace_for(args, max_cluster);
   if (need > 0 && (!args->workspace || args->workspace_bytes < need || !aligned(args->workspace, 256)))
     return SSM_ERR_WORKSPACE;
 
@@ -382,14 +392,16 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   const ssm::LaneLayout lay = ssm::choose_layout(a->N, a->Bt * a->Dn * p.n_seg);
   const int64_t ch = ssm::channels_per_cta(lay);
   p.n_dtiles = (a->Dn + ch - 1) / ch;
+  p.cluster = ssm::bwd_cluster(lay, p.n_dtiles, max_cluster);
+  p.n_ptiles = p.n_dtiles / p.cluster;
   const int64_t BD = a->Bt * a->Dn, PD = BD * p.n_seg;
   p.p_dA_log = reinterpret_cast<float *>(take(sizeof(float) * PD * a->N));
   p.p_dD = reinterpret_cast<float *>(take(sizeof(float) * PD));
   p.p_ddt_bias = reinterpret_cast<float *>(take(sizeof(float) * PD));
   p.p_dconv_w = reinterpret_cast<float *>(take(sizeof(float) * PD * 4));
   p.p_dconv_b = reinterpret_cast<float *>(take(sizeof(float) * PD));
-  p.p_dB = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
-  p.p_dC = reinterpret_cast<float *>(take(sizeof(float) * p.n_dtiles * a->Bt * a->N * a->L));
+  p.p_dB = reinterpret_cast<float *>(take(sizeof(float) * p.n_ptiles * a->Bt * a->N * a->L));
+  p.p_dC = reinterpret_cast<float *>(take(sizeof(float) * p.n_ptiles * a->Bt * a->N * a->L));
   if (!args->chunk_states)
     p.f.chunk_states = reinterpret_cast<float *>(take(sizeof(float) * BD * p.f.n_ck * a->N));
   if (p.n_seg > 1) {
@@ -401,7 +413,7 @@ ssm_status ssm_scan_bwd(const ssm_bwd_args *args, void *stream) {
   return cuda_status(ssm::launch_bwd(p, a->in_dtype == SSM_BF16, static_cast<cudaStream_t>(stream)));
 }
 
-}  // extern "C"
+}  // namespace ssm
 
 namespace {
 ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {

@@ -90,12 +90,35 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   static constexpr size_t y1_off = y0_off + sizeof(float) * CH * YC;
   static constexpr size_t dcs_off = y1_off + (SHFL ? 0 : sizeof(float) * CH * YC);
   static constexpr size_t rb_off = dcs_off + sizeof(float) * CH * DCS;
-  static constexpr size_t slot_off = rb_off + (BFLY ? sizeof(float) * TS * WPT : sizeof(float) * 2 * RBW);
+  // cluster exchange: every thread's 4-step sums of the stage, two rows (one per stage parity)
+  static constexpr size_t cx_off = rb_off + (BFLY ? sizeof(float) * TS * WPT : sizeof(float) * 2 * RBW);
+  static constexpr size_t slot_off = cx_off + (BFLY ? sizeof(float4) * 2 * kThreads : 0);
   static constexpr size_t bytes = slot_off + 16;
   __host__ __device__ static constexpr int rb_index(int which, int tt, int c, int n) {
     return which * RBW + tt * RBT + (c / CHH) * RBC + (c % CHH) * NP + n;
   }
 };
+
+// Thread-block cluster helpers: a full barrier of the cluster's CTAs (release / acquire, so shared
+// memory written before it is visible to the other CTAs after it), this CTA's rank, and a 16-byte
+// load from the same offset of another CTA's shared memory.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(const float4 *local, uint32_t rank) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(ra) : "memory");
+  return v;
+}
 
 template <int NS> __device__ __forceinline__ void store_states(float *dst, const float *v) {
   if (NS % 4 == 0) {
@@ -620,17 +643,47 @@ ssm_bwd_kernel(const BwdParams P) {
       // group tq) adds the 4 warps in order and writes 4 consecutive steps of one (quantity, state)
       __syncthreads();
       const int l = tid >> 2, tq = tid & 3;
-      const int which = l >> 4, n = (l & 3) * 4 + ((l >> 3) & 1) * 2 + ((l >> 2) & 1);
       float acc[4];
 #pragma unroll
       for (int i = 0; i < 4; i++) {
         const float *src = rb + (4 * tq + i) * S::WPT + l;
         acc[i] = ((src[0] + src[32]) + src[64]) + src[96];
       }
-      const int64_t t = t0 + 4 * tq;
-      if (n < N && t < te) {
-        const float sg = which ? 1.f : -1.f;  // dB partials were kept negated
-        float *dst = (which ? P.p_dC : P.p_dB) + ((tile * p.Bt + b) * N + n) * L + t;
+      // with a cluster, the CTAs of the cluster (consecutive channel tiles of this batch element)
+      // first add their sums in rank order: every thread parks its 4 values, and thread i of
+      // rank r then adds item r * 128 / CL + i of every rank through distributed shared memory
+      int item = tid, ptile = (int)tile;
+      bool mine = true;
+      if (P.cluster > 1) {
+        float4 *cx = reinterpret_cast<float4 *>(smem + S::cx_off) + (st & 1) * kThreads;
+        cx[tid] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        cluster_sync();  // every rank's sums of this stage are in place
+        const uint32_t rank = cluster_rank();
+        const int per = kThreads / P.cluster;
+        mine = tid < per;
+        item = (int)rank * per + tid;
+        ptile = (int)(tile / P.cluster);
+        if (mine) {
+          float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int r = 0; r < P.cluster; r++) {
+            const float4 v = ld_cluster_f4(cx + item, (uint32_t)r);
+            tot.x += v.x;
+            tot.y += v.y;
+            tot.z += v.z;
+            tot.w += v.w;
+          }
+          acc[0] = tot.x;
+          acc[1] = tot.y;
+          acc[2] = tot.z;
+          acc[3] = tot.w;
+        }
+      }
+      const int li = item >> 2, qi = item & 3;
+      const int wi = li >> 4, ni = (li & 3) * 4 + ((li >> 3) & 1) * 2 + ((li >> 2) & 1);
+      const int64_t t = t0 + 4 * qi;
+      if (mine && ni < N && t < te) {
+        const float sg = wi ? 1.f : -1.f;  // dB partials were kept negated
+        float *dst = (wi ? P.p_dC : P.p_dB) + (((int64_t)ptile * p.Bt + b) * N + ni) * L + t;
         if (vec && t + 3 < te) {
           *reinterpret_cast<float4 *>(dst) = make_float4(sg * acc[0], sg * acc[1], sg * acc[2], sg * acc[3]);
         } else {
@@ -776,6 +829,7 @@ ssm_bwd_kernel(const BwdParams P) {
     P.p_dconv_b[sbd] = accCb;
     for (int k = 0; k < 4; k++) P.p_dconv_w[sbd * 4 + k] = accW[k];
   }
+  if (S::BFLY && P.cluster > 1) cluster_sync();  // no rank leaves while another may still read its rows
   tmem_free_cta(tbase, S::NCOLS);
 }
 
@@ -972,11 +1026,20 @@ __global__ void seg_dx_fixup_kernel(const BwdParams P) {
   for (int j = 0; j < p.K - 1; j++) P.dx[bd * p.L + ts - 1 - j] += P.seg_dxh[(seg * BD + bd) * 4 + j];
 }
 
-size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg) {
+int bwd_cluster(const LaneLayout &lay, int64_t n_dtiles, int max_cluster) {
+  if (lay.G != 4 || lay.NS != 4) return 1;
+  for (int cl = 8; cl > 1; cl >>= 1)
+    if (cl <= max_cluster && n_dtiles % cl == 0) return cl;
+  return 1;
+}
+
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg,
+                           int max_cluster) {
   auto rnd = [](size_t x) { return (x + 255) & ~size_t(255); };
   const LaneLayout lay = choose_layout(N, Bt * Dn * n_seg);
   const int64_t ch = channels_per_cta(lay);
-  const int64_t n_tiles = (Dn + ch - 1) / ch;
+  const int64_t n_dtiles = (Dn + ch - 1) / ch;
+  const int64_t n_tiles = n_dtiles / bwd_cluster(lay, n_dtiles, max_cluster);  // partial tiles
   const int64_t BD = Bt * Dn, PD = BD * n_seg;  // parameter partials: one row per (segment, b, d)
   size_t s = 0;
   s += rnd(sizeof(float) * PD * N);
@@ -1017,6 +1080,25 @@ static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int64_t grid = P.n_dtiles * P.f.Bt * P.n_seg;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (P.cluster > 1) {
+    // consecutive blocks are consecutive channel tiles of one (segment, batch element), and the
+    // tile count is a multiple of the cluster size, so a cluster never straddles two of them
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, P);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   kern<<<(unsigned)grid, kThreads, smem, stream>>>(P);
   return cudaGetLastError();
 }
@@ -1082,10 +1164,10 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
       const int64_t blocks = (per_tile / 4 + 255) / 256;
       reduce_tiles_vec_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
           reinterpret_cast<const float4 *>(P.p_dB), reinterpret_cast<const float4 *>(P.p_dC),
-          reinterpret_cast<float4 *>(P.dB), reinterpret_cast<float4 *>(P.dC), P.n_dtiles, per_tile / 4);
+          reinterpret_cast<float4 *>(P.dB), reinterpret_cast<float4 *>(P.dC), P.n_ptiles, per_tile / 4);
     } else {
       const int64_t blocks = (per_tile + 255) / 256;
-      reduce_tiles_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P.p_dB, P.p_dC, P.dB, P.dC, P.n_dtiles, per_tile);
+      reduce_tiles_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P.p_dB, P.p_dC, P.dB, P.dC, P.n_ptiles, per_tile);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

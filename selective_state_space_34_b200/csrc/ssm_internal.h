@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/ssm_scan.h"
+
 namespace ssm {
 
 constexpr int kThreads = 128;  // threads per CTA for the scan kernels
@@ -96,9 +98,12 @@ struct BwdParams {
   float *p_ddt_bias; // (Bt, Dn)
   float *p_dconv_w;  // (Bt, Dn, 4)
   float *p_dconv_b;  // (Bt, Dn)
-  // per-channel-tile partial sums of dB / dC: (n_dtiles, Bt, N, L) each
+  // per-tile partial sums of dB / dC: (n_ptiles, Bt, N, L) each; a tile is one channel tile, or
+  // the `cluster` consecutive channel tiles of a thread-block cluster whose CTAs add their sums
   float *p_dB, *p_dC;
   int64_t n_dtiles;
+  int64_t n_ptiles;
+  int cluster;
   float *dA_log, *dD, *ddt_bias, *dconv_w, *dconv_b;
   void *const *timing_events;  // optional: 2 cudaEvent_t around the main backward kernel
   const float *dh_last;        // (Bt, Dn, N) or null
@@ -126,7 +131,19 @@ cudaError_t launch_fwd(const FwdParams &p, int in_bf16, int out_bf16, cudaStream
 // The time-parallel forward (ssm_fwd_tp.cu): one pass, the same outputs as launch_fwd.
 cudaError_t launch_fwd_tp(const FwdParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, int in_bf16, cudaStream_t stream);
-size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg);
+// Backward scratch for a cluster size of at most max_cluster (see bwd_cluster).
+size_t bwd_workspace_bytes(int64_t Bt, int64_t Dn, int64_t N, int64_t L, int need_states, int n_seg,
+                           int max_cluster);
+// CTAs per thread-block cluster of the backward, at most max_cluster: the CTAs of a cluster (4 or 8
+// consecutive channel tiles) add their dB / dC stage sums through distributed shared memory before
+// writing them, which divides the per-tile partials (scratch and traffic) by the cluster size at
+// the price of one cluster barrier per stage (measured 6% slower on 4x4096x16x4096). 1 when the
+// layout (4 lanes x 4 states) or the tile count does not allow max_cluster.
+int bwd_cluster(const LaneLayout &lay, int64_t n_dtiles, int max_cluster);
+// ssm_scan_bwd with clusters of up to max_cluster CTAs (ssm_scan_bwd itself uses 1), and the
+// scratch it needs (ssm_bwd_workspace_size for max_cluster = 1).
+ssm_status scan_bwd_clustered(const ssm_bwd_args *args, void *stream, int max_cluster);
+size_t bwd_workspace_for(const ssm_bwd_args *args, int max_cluster);
 cudaError_t launch_step(const StepParams &p, int in_bf16, int out_bf16, cudaStream_t stream);
 cudaError_t launch_conv1d_silu(const void *x, void *u, const float *w, const float *b, int64_t Bt,
                                int64_t Dn, int64_t L, int K, int in_bf16, int out_bf16, int vec,

@@ -20,7 +20,6 @@
 // them) race on the array and give wrong gradients. Order them on one stream or with events.
 #include <mutex>
 
-#include "../../include/ssm_scan.h"
 #include "ssm_internal.h"
 
 namespace {
@@ -37,9 +36,17 @@ extern "C" {
 
 ssm_status ssm_scan_bwd_noalloc(const ssm_bwd_args *args, void *stream) {
   if (!args) return SSM_ERR_NULL;
-  // Reject problems whose scratch does not fit before touching the device.
-  const size_t need = ssm_bwd_workspace_size(args);
-  if (need > (size_t)SSM_NOALLOC_SCRATCH_BYTES) return SSM_ERR_WORKSPACE;
+  // The smallest thread-block cluster whose scratch fits the array: clusters of 4 or 8 CTAs add
+  // their dB / dC partial sums on chip, dividing that (largest) part of the scratch by 4 or 8 for
+  // a slightly slower kernel. Problems that fit with none of them are rejected before anything
+  // touches the device.
+  int cluster = 0;
+  for (int c : {1, 4, 8})
+    if (ssm::bwd_workspace_for(args, c) <= (size_t)SSM_NOALLOC_SCRATCH_BYTES) {
+      cluster = c;
+      break;
+    }
+  if (!cluster) return SSM_ERR_WORKSPACE;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -60,7 +67,7 @@ ssm_status ssm_scan_bwd_noalloc(const ssm_bwd_args *args, void *stream) {
   ssm_bwd_args a = *args;
   a.workspace = scratch;
   a.workspace_bytes = (size_t)SSM_NOALLOC_SCRATCH_BYTES;
-  return ssm_scan_bwd(&a, stream);
+  return ssm::scan_bwd_clustered(&a, stream, cluster);
 }
 
 }  // extern "C"

@@ -125,6 +125,22 @@ def test_fwd_guards(monkeypatch, dtype, N, L, nseg):
     _same(a, b)
 
 
+@pytest.mark.parametrize("dtype,N,L", [("bf16", 16, 333), ("f32", 64, 100), ("bf16", 5, 77), ("f32", 16, 64)])
+def test_chunked_fwd_guards(monkeypatch, dtype, N, L):
+    """The chunked (time-parallel) forward: every output, saved state and carried state."""
+    t = _setup(2, 70, N, L, dtype)
+    od = torch.bfloat16 if dtype == "bf16" else torch.float32
+
+    def run(g):
+        i = _inputs(g, t)
+        return ssm.ssm_scan_fwd(i["x"], i["dt"], i["A_log"], i["B"], i["C"], out_dtype=od,
+                                save_states=True, return_u=True, return_state=True, h0=i["h0"],
+                                conv_hist=i["conv_hist"], scan_form="chunked", **param_kw(i))
+
+    a, b = _guarded(monkeypatch, run)
+    _same(a, b)
+
+
 @pytest.mark.parametrize("dtype,N,L,nseg,saved", [("bf16", 16, 333, 0, False), ("bf16", 16, 333, 3, False),
                                                   ("f32", 64, 100, 0, True), ("bf16", 16, 130, 2, True)])
 def test_bwd_guards(monkeypatch, dtype, N, L, nseg, saved):
