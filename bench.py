@@ -324,8 +324,9 @@ def reference_arm(args, w):
 # ---- the state-space-duality leg (Mamba-2 heads, tensor cores) ---------------------------------
 
 def ssd_bench(args, cfg, name):
-    """The Mamba-2 state-space-duality layer (three launches per step) through the C ABI, with the
-    output kernel (the dominant launch) timed on its own by the library's timing events."""
+    """The Mamba-2 state-space-duality layer through the C ABI: the fused form (one launch per step,
+    timed on its own by the library's timing events) or the three-pass form (three launches, the
+    output kernel -- the dominant one -- timed on its own)."""
     import ctypes
     import torch
     from selective_state_space_34_b200 import _abi
@@ -347,6 +348,8 @@ def ssd_bench(args, cfg, name):
     sa.B, sa.C, sa.D, sa.y = T["B"].data_ptr(), T["C"].data_ptr(), T["D"].data_ptr(), y.data_ptr()
     sa.Bt, sa.H, sa.L, sa.P, sa.N = Bt, H, L, P, N
     sa.in_dtype, sa.out_dtype, sa.delta_softplus, sa.discretization = _abi.SSM_BF16, _abi.SSM_BF16, 1, _abi.SSM_ZOH
+    fused = args.ssd_form == "fused" or (args.ssd_form == "auto" and P == 64)
+    sa.form = _abi.SSM_SSD_FUSED if fused else _abi.SSM_SSD_THREE_PASS
     lib = _abi.load()
     need = int(lib.ssm_ssd_workspace_size(ctypes.byref(sa)))
     ws = torch.empty(need + 256, dtype=torch.uint8, device=dev)
@@ -397,6 +400,13 @@ def ssd_bench(args, cfg, name):
     # C H_in (K = N) per head
     hg = 8 if H % 8 == 0 else (4 if H % 4 == 0 else (2 if H % 2 == 0 else 1))
     oflops = 2 * Bt * nC * ((H // hg) * 128 * 128 * 128 + H * (128 * P * 128 + 128 * P * N))
+    if fused:
+        # the one launch is the layer: its bytes are the layer's; tensor work per (batch, head,
+        # chunk) as issued: C B^T (K = N), G'X and the state product (K = Q), C H (K = N)
+        kname, ksrc, ob = "ssd_fused_kernel", "ssm_ssd_fused.cu", ab
+        oflops = 2 * Bt * H * nC * (128 * 128 * N + 2 * 128 * P * 128 + 128 * P * N)
+    else:
+        kname, ksrc = "ssd_out_kernel", "ssm_ssd.cu"
     peaks = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -407,16 +417,17 @@ def ssd_bench(args, cfg, name):
                     "p90": float(np.percentile(per_step, 90)), "of": "rank 0, CUDA events around each timed step"},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": name, "Bt": Bt, "H": H, "P": P, "N": N, "L": L, "chunk": 128,
-                   "step": "ssd forward (3 launches)", "l2": "inputs larger than L2"},
+                   "step": "ssd forward (1 launch, fused)" if fused else "ssd forward (3 launches)",
+                   "form": "fused" if fused else "three_pass", "l2": "inputs larger than L2"},
         "roofline": {"bound": "hbm", "achieved": ob / (out_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                     "frac": ob / (out_ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic("ssd_out_kernel", "ssm_ssd.cu"),
-                     "algorithmic_bytes": ob, "kernel": "ssd_out_kernel", "ms": out_ms,
+                     "frac": ob / (out_ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic(kname, ksrc),
+                     "algorithmic_bytes": ob, "kernel": kname, "ms": out_ms,
                      "peak_source": peaks.get("source")},
         "tensor": {"achieved": oflops / (out_ms * 1e-3) / 1e12, "peak": bf16, "unit": "TFLOP/s",
-                   "frac": oflops / (out_ms * 1e-3) / 1e12 / bf16, "kernel": "ssd_out_kernel", "flops": oflops},
+                   "frac": oflops / (out_ms * 1e-3) / 1e12 / bf16, "kernel": kname, "flops": oflops},
         "layer": {"ms": ms, "hbm_gbs": ab / (ms * 1e-3) / 1e9, "hbm_frac": ab / (ms * 1e-3) / 1e9 / hbm,
                   "algorithmic_bytes": ab},
-        "gpu_launches": 3 * args.steps, "clocks": clk,
+        "gpu_launches": (1 if fused else 3) * args.steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -441,6 +452,8 @@ def main():
                     help="split-L for the forward: 0 one pass, k up to k segments, -1 automatic")
     ap.add_argument("--scan-form", default="lanes", choices=["lanes", "chunked"],
                     help="layout of a one-pass forward scan: states over lanes, or chunked in time")
+    ap.add_argument("--ssd-form", default="auto", choices=["auto", "fused", "three_pass"],
+                    help="state-space-duality workloads: one fused launch, or three passes")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 

@@ -183,6 +183,16 @@ ssm_status ssm_scan_fwd(const ssm_fwd_args *args, void *stream);
  * shared by all heads of a batch element (one group). Supported: bf16 inputs, P (head dim) 64 or
  * 128, N (state) 64 or 128 (SSM_ERR_UNSUPPORTED otherwise).
  */
+/* How ssm_ssd_fwd schedules the chunks.
+ *   SSM_SSD_AUTO       the fused form where it applies (P = 64), else the three-pass form.
+ *   SSM_SSD_THREE_PASS three launches: every chunk's state product in parallel, the carry of the
+ *                      states over the chunks (fp32, through the workspace), every chunk's output
+ *                      in parallel.
+ *   SSM_SSD_FUSED      one launch: one CTA per (batch, head) walks the chunks in order with the
+ *                      state in tensor memory, tiles loaded by TMA; P = 64 only
+ *                      (SSM_ERR_UNSUPPORTED otherwise). */
+typedef enum ssm_ssd_form { SSM_SSD_AUTO = 0, SSM_SSD_THREE_PASS = 1, SSM_SSD_FUSED = 2 } ssm_ssd_form;
+
 typedef struct ssm_ssd_args {
   const void *x;         /* device (Bt, H, L, P) bf16, 16-byte aligned */
   const void *dt;        /* device (Bt, H, L) bf16 */
@@ -202,10 +212,11 @@ typedef struct ssm_ssd_args {
   int32_t discretization;/* ssm_discretization */
   void *workspace;       /* device scratch of ssm_ssd_workspace_size() bytes, 256-byte aligned */
   size_t workspace_bytes;
-  void *const *timing_events; /* NULL, or 2 caller-created cudaEvent_t: [0] is recorded on
-                                 `stream` just before the output kernel (the last of the three
-                                 launches), [1] just after it; lets a caller time that kernel
-                                 alone. Recording does not synchronise. */
+  void *const *timing_events; /* NULL, or 2 caller-created cudaEvent_t recorded on `stream`: with
+                                 the fused form [0] just before its one launch and [1] just after;
+                                 with the three-pass form around the output kernel (the last of the
+                                 three launches). Recording does not synchronise. */
+  int32_t form;          /* ssm_ssd_form: how the chunks are scheduled */
 } ssm_ssd_args;
 
 /* Scratch bytes ssm_ssd_fwd needs: the chunk states (fp32), the state entering every chunk
@@ -213,7 +224,8 @@ typedef struct ssm_ssd_args {
 size_t ssm_ssd_workspace_size(const ssm_ssd_args *args);
 
 /* Errors: SSM_ERR_NULL, SSM_ERR_SHAPE (negative sizes, H/P/N = 0), SSM_ERR_ALIGN,
- * SSM_ERR_DTYPE (codes), SSM_ERR_UNSUPPORTED (in_dtype not bf16, P not 64/128, N not 64/128),
+ * SSM_ERR_DTYPE (codes), SSM_ERR_UNSUPPORTED (in_dtype not bf16, P not 64/128, N not 64/128, an
+ * unknown form, SSM_SSD_FUSED with P != 64),
  * SSM_ERR_WORKSPACE, SSM_ERR_CUDA. Bt = 0 or L = 0: nothing to do (h_last = h0 or 0). */
 ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream);
 

@@ -11,6 +11,7 @@ LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 SSM_F32, SSM_BF16 = 0, 1
 SSM_ZOH, SSM_EULER = 0, 1
 SSM_SCAN_LANES, SSM_SCAN_CHUNKED = 0, 1
+SSM_SSD_AUTO, SSM_SSD_THREE_PASS, SSM_SSD_FUSED = 0, 1, 2
 SSM_STATE_CHUNK = 16
 SSM_NOALLOC_SCRATCH_BYTES = 72 << 20
 SSM_ERR_TIMEOUT = 8
@@ -74,7 +75,7 @@ class SsdArgs(ctypes.Structure):
         ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
         ("delta_softplus", ctypes.c_int32), ("discretization", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-        ("timing_events", ctypes.c_void_p),
+        ("timing_events", ctypes.c_void_p), ("form", ctypes.c_int32),
     ]
 
 

@@ -50,6 +50,7 @@ _DISC = {"zoh": _abi.SSM_ZOH, "euler": _abi.SSM_EULER}
 
 
 _SCAN = {"lanes": _abi.SSM_SCAN_LANES, "chunked": _abi.SSM_SCAN_CHUNKED}
+_SSD_FORM = {"auto": _abi.SSM_SSD_AUTO, "three_pass": _abi.SSM_SSD_THREE_PASS, "fused": _abi.SSM_SSD_FUSED}
 
 
 def _fwd_args(x, dt, A_log, B, C, D, z, dt_bias, conv_w, conv_b, delta_softplus, out_dtype,
@@ -312,14 +313,16 @@ def ssm_conv1d_silu(x, w, b=None, out_dtype=None, out: Optional[torch.Tensor] = 
 
 def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplus: bool = True,
                 out_dtype=None, discretization: str = "zoh", return_state: bool = False,
-                check: bool = False, timing_events=None):
+                check: bool = False, timing_events=None, form: str = "auto"):
     """Mamba-2 state-space duality forward. x: (Bt, H, L, P) bf16; dt: (Bt, H, L) bf16; B, C:
     (Bt, L, N) bf16 shared by the heads; A_log, D, dt_bias: (H,) fp32; h0: (Bt, H, N, P) fp32.
     P and N must be 64 or 128. Returns y (Bt, H, L, P), or (y, h_last) with return_state.
+    ``form``: "fused" (one launch, the state kept on chip; P = 64), "three_pass" (chunk states,
+    their carry and the outputs as three launches) or "auto" (fused where it applies).
     check=True synchronises the stream afterwards and raises SSMError (code SSM_ERR_TIMEOUT) if a
     bounded wait for the tensor cores ran out. ``timing_events``: optional pair of
     torch.cuda.Event(enable_timing=True), recorded once already; the library records them just
-    before and just after the output kernel (the last of its three launches)."""
+    before and just after the fused kernel, or the output kernel of the three-pass form."""
     for n, t in (("x", x), ("dt", dt), ("A_log", A_log), ("B", B), ("C", C)):
         _need_cuda(n, t)
     for n, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
@@ -345,6 +348,9 @@ def ssm_ssd_fwd(x, dt, A_log, B, C, D=None, dt_bias=None, h0=None, delta_softplu
     if discretization not in _DISC:
         raise ValueError("discretization must be 'zoh' or 'euler'")
     a.discretization = _DISC[discretization]
+    if form not in _SSD_FORM:
+        raise ValueError("form must be 'auto', 'fused' or 'three_pass'")
+    a.form = _SSD_FORM[form]
     lib = _abi.load()
     need = int(lib.ssm_ssd_workspace_size(ctypes.byref(a)))
     ws = None

@@ -424,6 +424,9 @@ ssm_status check_ssd(const ssm_ssd_args *a, bool *empty) {
   if (a->H == 0 || a->P == 0 || a->N == 0) return SSM_ERR_SHAPE;
   if (a->in_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if ((a->P != 64 && a->P != 128) || (a->N != 64 && a->N != 128)) return SSM_ERR_UNSUPPORTED;
+  if (a->form != SSM_SSD_AUTO && a->form != SSM_SSD_THREE_PASS && a->form != SSM_SSD_FUSED)
+    return SSM_ERR_UNSUPPORTED;
+  if (a->form == SSM_SSD_FUSED && a->P != 64) return SSM_ERR_UNSUPPORTED;
   int64_t bh, rows, elems;
   if (!mul_ok(a->Bt, a->H, &bh) || !mul_ok(bh, a->L, &rows) || !mul_ok(rows, a->P, &elems) ||
       elems > (INT64_C(1) << 50) || (bh > 0 && (a->L + 127) / 128 > (INT64_C(1) << 31) / bh))
@@ -502,6 +505,7 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream) {
   p.delta_softplus = args->delta_softplus ? 1 : 0;
   p.euler = args->discretization == SSM_EULER ? 1 : 0;
   p.timing_events = args->timing_events;
+  p.form = args->form;
   p.S = reinterpret_cast<float *>(w);
   w += rnd(sizeof(float) * chunks * np);
   p.Hin = reinterpret_cast<__nv_bfloat16 *>(w);

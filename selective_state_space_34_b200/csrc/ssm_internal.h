@@ -60,9 +60,13 @@ struct SsdParams {
   __nv_bfloat16 *Hin;          // workspace: state entering each chunk, same shape, bf16
   float *cum_end;              // workspace: log-decay of each chunk (Bt, H, n_chunks)
   int *error;                  // workspace: set to 1 if a tensor-core wait timed out
-  void *const *timing_events;  // optional: 2 cudaEvent_t around the output kernel
+  void *const *timing_events;  // optional: 2 cudaEvent_t around the output (or the fused) kernel
+  int form;                    // ssm_ssd_form
 };
 cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream);
+// The fused one-launch form (ssm_ssd_fused.cu): P = 64, N = 64 or 128.
+bool ssd_fused_supported(const SsdParams &p);
+cudaError_t launch_ssd_fused(const SsdParams &p, int out_bf16, cudaStream_t stream);
 size_t ssd_workspace_bytes(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);
 // Byte offset of the SSD error word inside the workspace (its last 256-byte block).
 size_t ssd_error_offset(int64_t Bt, int64_t H, int64_t L, int64_t P, int64_t N);

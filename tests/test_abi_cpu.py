@@ -52,8 +52,9 @@ def _header_fields(struct):
     ("ssm_bwd_args", "BwdArgs", 216 + 17 * 8 + 8),
     # 13 pointers, 3 int64, 5 int32 (+4 bytes of tail padding)
     ("ssm_step_args", "StepArgs", 13 * 8 + 3 * 8 + 5 * 4 + 4),
-    # 10 pointers, 5 int64, 4 int32, workspace pointer and size, timing events
-    ("ssm_ssd_args", "SsdArgs", 10 * 8 + 5 * 8 + 4 * 4 + 8 + 8 + 8),
+    # 10 pointers, 5 int64, 4 int32, workspace pointer and size, timing events, the form (+4 bytes
+    # of tail padding)
+    ("ssm_ssd_args", "SsdArgs", 10 * 8 + 5 * 8 + 4 * 4 + 8 + 8 + 8 + 8),
 ])
 def test_struct_layout_matches_header_field_order(struct, cls, size):
     ct = [f[0] for f in getattr(_abi, cls)._fields_]
@@ -235,6 +236,8 @@ def test_ssd_validation_codes(lib):
     assert f(_ssd(P=32)) == 5 and f(_ssd(N=16)) == 5
     assert f(_ssd(H=0)) == 2 and f(_ssd(L=-1)) == 2
     assert f(_ssd(discretization=2)) == 5
+    assert f(_ssd(form=3)) == 5 and f(_ssd(form=-1)) == 5
+    assert f(_ssd(form=2, P=128)) == 5          # the fused form takes P = 64 only
     assert f(_ssd(x=0x10008)) == 3             # 16-byte alignment of the tile loads
     assert f(_ssd(dt=0x20001)) == 3
     assert f(_ssd(h0=0x70004)) == 3 and f(_ssd(h_last=0x70008)) == 3

@@ -190,9 +190,10 @@ def test_step_guards(monkeypatch, dtype):
     _same(a, b)
 
 
+@pytest.mark.parametrize("form", ["auto", "three_pass"])
 @pytest.mark.parametrize("H,L,P,N,od", [(3, 200, 64, 64, torch.bfloat16), (2, 130, 128, 128, torch.float32),
-                                        (8, 385, 64, 128, torch.bfloat16)])
-def test_ssd_guards(monkeypatch, H, L, P, N, od):
+                                        (8, 385, 64, 128, torch.bfloat16), (2, 77, 64, 128, torch.float32)])
+def test_ssd_guards(monkeypatch, H, L, P, N, od, form):
     Bt = 2
     a = wl.generate_ssd(Bt, H, L, P, N, seed=9)
     t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
@@ -203,7 +204,7 @@ def test_ssd_guards(monkeypatch, H, L, P, N, od):
         i = _inputs(g, dict(t, h0=h0))
         return ssm.ssm_ssd_fwd(i["x"], i["dt"], i["A_log"], i["B"], i["C"], D=i["D"],
                                dt_bias=i["dt_bias"], h0=i["h0"], out_dtype=od, return_state=True,
-                               check=True)
+                               check=True, form=form)
 
     a, b = _guarded(monkeypatch, run)
     _same(a, b)

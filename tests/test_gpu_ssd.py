@@ -1,5 +1,7 @@
 """Parity of the Mamba-2 state-space-duality forward on the tensor cores ("state-space models",
-"Mamba-2 and state-space duality") against the float64 recurrence of the oracle.
+"Mamba-2 and state-space duality") against the float64 recurrence of the oracle, in both forms: the
+fused one-launch kernel (form "auto" picks it for P = 64) and the three-pass one ("three_pass";
+"auto" picks it for P = 128).
 
 Bound, from the arithmetic. bf16 keeps 8 significant bits, so one round-to-nearest changes a value
 by at most 2^-8 of itself. Every output is a sum of terms (C_t . B_s) (decay) beta_s x_s (plus D x_t
@@ -7,8 +9,9 @@ and the carried state's terms); the inputs x, B, C are bf16 already, and a term 
 roundings on its way:
   * a term from the same chunk: the masked, decayed score (C_t . B_s) 2^{ct_t - q_s} (with D on its
     diagonal) rounded to bf16 as the operand of G'X -- one rounding;
-  * a term from an earlier chunk: the scaled B operand e^{cum_end - cum_s} beta_s B_s of the
-    chunk-state product, and the state entering the chunk (bf16 operand of C H_in) -- two.
+  * a term from an earlier chunk: the scaled operand of the chunk-state product (e^{cum_end - cum_s}
+    beta_s B_s in the three-pass form, the same weight times x_s in the fused form), and the state
+    entering the chunk (bf16 operand of C H_in) -- two.
 So the bf16 part is at most ((1 + 2^-8)^2 - 1) Y_abs, with Y_abs the oracle run on |x|, |B|, |C|,
 |D| (|h0|): an upper bound on the sum of the terms' magnitudes (|C_t . B_s| <= |C_t| . |B_s|; beta,
 the decays and the state recursion are non-negative maps of non-negative inputs). The fp32 part:
@@ -22,7 +25,7 @@ the decays and the state recursion are non-negative maps of non-negative inputs)
     base 2 move an exponent by at most about M 2^-24 (log2 e for base 2); a factor 2^e with e off by
     de changes by ln2 de of itself. 16 M 2^-24 Y_abs covers it.
 Total: |y - y_ref| <= (2^-7 + 2^-16 + 2^-12 + 16 M 2^-24) Y_abs, plus 2^-8 |y_ref| for a bf16 output.
-The final state h_last is carried in fp32 and meets only the scaled-B rounding:
+The final state h_last is carried in fp32 and meets only the scaled-operand rounding:
 |h - h_ref| <= (2^-8 + 2^-12 + 16 M 2^-24) H_abs."""
 import numpy as np
 import pytest
@@ -30,7 +33,7 @@ import torch
 
 import oracle
 import selective_state_space_34_b200 as ssm
-from selective_state_space_34_b200 import workloads as wl
+from selective_state_space_34_b200 import _abi, workloads as wl
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +57,7 @@ def bound_coefs(a, softplus=True):
 
 
 def _run(Bt, H, L, P, N, out_dtype=torch.float32, euler=False, softplus=True, carry=False, D=True,
-         seed=7):
+         seed=7, form="auto"):
     a = wl.generate_ssd(Bt, H, L, P, N, seed=seed)
     if not softplus:
         # without softplus dt + dt_bias is Delta itself: a step size, so non-negative
@@ -69,7 +72,7 @@ def _run(Bt, H, L, P, N, out_dtype=torch.float32, euler=False, softplus=True, ca
         h0 = torch.from_numpy(h0_np).to(dev)
     r = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"] if D else None,
                         dt_bias=t["dt_bias"], h0=h0, delta_softplus=softplus, out_dtype=out_dtype,
-                        discretization="euler" if euler else "zoh", return_state=carry)
+                        discretization="euler" if euler else "zoh", return_state=carry, form=form)
     torch.cuda.synchronize()
     y = (r[0] if carry else r).float().cpu().numpy()
     kw = dict(dt_bias=a["dt_bias"], delta_softplus=softplus, euler=euler)
@@ -98,10 +101,14 @@ def _run(Bt, H, L, P, N, out_dtype=torch.float32, euler=False, softplus=True, ca
     return y, yref
 
 
+FORMS = ["auto", "three_pass"]
+
+
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("P,N", [(64, 128), (64, 64), (128, 128), (128, 64)])
-@pytest.mark.parametrize("L", [128, 300, 1])
-def test_ssd_shapes(P, N, L):
-    _run(2, 3, L, P, N)
+@pytest.mark.parametrize("L", [128, 300, 1, 129, 8])
+def test_ssd_shapes(P, N, L, form):
+    _run(2, 3, L, P, N, form=form)
 
 
 @pytest.mark.parametrize("Bt,H,L,P,N,out", [
@@ -110,20 +117,32 @@ def test_ssd_shapes(P, N, L):
     (1, 8, 130, 64, 64, torch.float32),     # 8 heads, N = 64 (half the C H_in slices), ragged tail
     (1, 6, 257, 64, 128, torch.bfloat16),   # 2 heads per CTA
 ])
-def test_ssd_head_groups(Bt, H, L, P, N, out):
-    _run(Bt, H, L, P, N, out_dtype=out, carry=True)
+@pytest.mark.parametrize("form", FORMS)
+def test_ssd_head_groups(Bt, H, L, P, N, out, form):
+    _run(Bt, H, L, P, N, out_dtype=out, carry=True, form=form)
 
 
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("variant", ["euler", "no_softplus", "bf16_out", "no_D", "carried_state"])
-def test_ssd_variants(variant):
+def test_ssd_variants(variant, form):
     _run(1, 2, 257, 64, 128, euler=variant == "euler", softplus=variant != "no_softplus",
          out_dtype=torch.bfloat16 if variant == "bf16_out" else torch.float32,
-         D=variant != "no_D", carry=variant == "carried_state")
+         D=variant != "no_D", carry=variant == "carried_state", form=form)
 
 
-def test_ssd_longer_sequence():
+@pytest.mark.parametrize("form", FORMS)
+def test_ssd_longer_sequence(form):
     """16 chunks: the carried state crosses many chunk boundaries."""
-    _run(1, 4, 2048, 64, 128)
+    _run(1, 4, 2048, 64, 128, form=form)
+
+
+def test_ssd_fused_form_needs_head_dim_64():
+    a = wl.generate_ssd(1, 2, 64, 128, 64, seed=2)
+    t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
+         for k, v in a.items()}
+    with pytest.raises(_abi.SSMError) as e:
+        ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], form="fused")
+    assert e.value.code == 5  # SSM_ERR_UNSUPPORTED
 
 
 def test_ssd_matches_selective_scan_for_one_channel_semantics():
@@ -146,7 +165,8 @@ def test_ssd_matches_selective_scan_for_one_channel_semantics():
 
 
 @pytest.mark.slow
-def test_full_ssd_layer_sampled_heads():
+@pytest.mark.parametrize("form", FORMS)
+def test_full_ssd_layer_sampled_heads(form):
     """The benchmarked SSD layer at full size (4 x 64 heads x 64 x 4096, N = 128, bf16 out), on
     sampled (batch, head) pairs over the whole sequence, within the derived bound."""
     cfg = wl.SSD_WORKLOADS["ssd_fwd"]
@@ -154,7 +174,8 @@ def test_full_ssd_layer_sampled_heads():
     a = wl.generate_ssd(Bt, H, L, P, N, seed=cfg["seed"])
     t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
          for k, v in a.items()}
-    y = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"])
+    y = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
+                        form=form)
     torch.cuda.synchronize()
     y = y.float().cpu().numpy()
     for (b, h) in wl.sample_channels(Bt, H, 8):
@@ -169,11 +190,12 @@ def test_full_ssd_layer_sampled_heads():
         assert np.all(np.abs(got - ref) <= tol), "head (%d, %d): worst excess %g" % (b, h, (np.abs(got - ref) - tol).max())
 
 
-def test_ssd_deterministic_and_empty():
+@pytest.mark.parametrize("form", FORMS)
+def test_ssd_deterministic_and_empty(form):
     a = wl.generate_ssd(2, 8, 300, 64, 128, seed=11)
     t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
          for k, v in a.items()}
-    kw = dict(D=t["D"], dt_bias=t["dt_bias"], return_state=True)
+    kw = dict(D=t["D"], dt_bias=t["dt_bias"], return_state=True, form=form)
     y1, h1 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], **kw)
     y2, h2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], **kw)
     torch.cuda.synchronize()
@@ -187,9 +209,10 @@ def test_ssd_deterministic_and_empty():
     assert y0.numel() == 0 and torch.equal(hl, h0)
 
 
-def test_ssd_timing_events_bracket_the_output_kernel():
-    """The optional event pair is recorded around the output kernel alone: its interval is positive
-    and shorter than the whole three-launch call."""
+@pytest.mark.parametrize("form", FORMS)
+def test_ssd_timing_events_bracket_the_output_kernel(form):
+    """The optional event pair is recorded around the fused kernel, or the output kernel of the
+    three-pass form: its interval is positive and shorter than the whole call."""
     a = wl.generate_ssd(2, 16, 1024, 64, 128, seed=5)
     t = {k: torch.from_numpy(v).to("cuda", torch.bfloat16 if k in ("x", "dt", "B", "C") else torch.float32)
          for k, v in a.items()}
@@ -199,11 +222,12 @@ def test_ssd_timing_events_bracket_the_output_kernel():
     torch.cuda.synchronize()
     ev[2].record()
     y = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
-                        timing_events=ev[:2])
+                        timing_events=ev[:2], form=form)
     ev[3].record()
     torch.cuda.synchronize()
     kernel_ms, call_ms = ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3])
     assert 0.0 < kernel_ms < call_ms
-    y2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"])
+    y2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], D=t["D"], dt_bias=t["dt_bias"],
+                         form=form)
     torch.cuda.synchronize()
     assert torch.equal(y, y2)  # recording changes nothing in the result
