@@ -11,19 +11,25 @@
 //   y        = G' X + diag(e^{cum_t}) C H_{c-1}            (Q x P)
 //   H_c      = e^{cum_end} H_{c-1} + B^T diag(w) X          (N x P)
 //
-// Roles (320 threads): warp 0 loads the tiles with TMA (cp.async.bulk.tensor, completion counted
-// on mbarriers), warp 1 issues the tcgen05 products from one thread, warps 2..9 do everything
-// else -- two threads per accumulator row (warps w and w + 4 reach the same 32 TMEM lanes), each
-// taking half of the row's columns. Per chunk c the compute warps (1) form the decay coefficients,
-// (2) copy H_{c-1} out of tensor memory as the bf16 operand of C H_{c-1}, scale H in place by
-// e^{cum_end}, and write diag(w) X, (3) finish chunk c-1's output from its two accumulators, and
-// (4) turn G into G'. The MMA warp issues G for chunk c as soon as C and B have landed, the
-// C H_{c-1} and state products after step (2), and G' X after step (4), so the tensor core works
-// on one chunk while the compute warps are on the other. G is double-buffered in tensor memory, and
-// C, B and X in shared memory, so the next chunk's tiles load while this one is computed; the
-// scaled X, the bf16 state and G' are single buffers whose reuse is ordered by the barriers below. Every wait is bounded; a wait that runs out records the error
-// word and an abort flag, after which every role runs its loop to the end without issuing work,
-// waits for its own copies and products in flight, and the CTA frees its tensor memory.
+// Roles (576 threads): warp 0 loads the tiles with TMA (cp.async.bulk.tensor, completion counted
+// on mbarriers), warp 1 issues the tcgen05 products from one thread, warps 2..17 do everything
+// else -- four threads per accumulator row (warps w, w + 4, w + 8, w + 12 reach the same 32 TMEM
+// lanes), each taking a quarter of the row's columns. Per chunk c the compute warps (1) form the
+// decay coefficients, (2) copy H_{c-1} out of tensor memory as the bf16 operand of C H_{c-1},
+// scale H in place by e^{cum_end}, and write diag(w) X, (3) finish chunk c-1's output from its two
+// accumulators, and (4) turn G into G'. The MMA warp issues C H_{c-1} and the state product of
+// chunk c after step (2), then G of chunk c+1, then G' X of chunk c after step (4), so the tensor
+// core works on one chunk while the compute warps are on the other and the next chunk's G is
+// ready before the compute warps need it. G is double-buffered in tensor memory, C, B and X in
+// shared memory; the scaled X, the bf16 state and G' are single buffers whose reuse is ordered by
+// the barriers below. Every wait is bounded; a wait that runs out records the error word and an
+// abort flag, after which every role runs its loop to the end without issuing work, waits for its
+// own copies and products in flight, and the CTA frees its tensor memory.
+//
+// Scores below the diagonal blocks: with cum_ref the running sum at the last step of the column's
+// 32-step block, e^{cum_t - cum_s} beta_s = e^{cum_t - cum_ref} (beta_s e^{cum_ref - cum_s}); both
+// factors are at most 1 (the second at most beta_s), so a score there costs one exp per row and
+// block instead of one per score. The diagonal blocks keep one exp per score.
 //
 // Tile layouts in shared memory (bf16, no-swizzle canonical, 8 rows x 16 bytes per core matrix):
 //   C, B  [n/8][t][n%8]   -- C is the K-major A operand (M = t, K = n) of G and of C H, B the K-major
@@ -46,8 +52,8 @@ namespace {
 
 constexpr int kQ = 128;          // chunk length
 constexpr int kP = 64;           // head dimension this kernel takes
-constexpr int kFThreads = 320;   // producer warp, MMA warp, 8 compute warps
-constexpr int kCompute = 256;
+constexpr int kFThreads = 576;   // producer warp, MMA warp, 16 compute warps
+constexpr int kCompute = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRowBytes = kQ * 16;  // one 8-column group of a Q-row tile
 
@@ -58,8 +64,9 @@ constexpr int kOffX = kOffC + 2 * kCBStride;   // 2 x 16 KB
 constexpr int kOffXW = kOffX + 2 * 16384;      // 16 KB
 constexpr int kOffSH = kOffXW + 16384;         // 16 KB
 constexpr int kOffGP = kOffSH + 16384;         // 32 KB
-constexpr int kOffQ = kOffGP + 32768;          // q_s of the chunk, 128 floats
-constexpr int kOffTot = kOffQ + kQ * 4;        // scan totals: 2 halves x 4 warps
+constexpr int kOffQ = kOffGP + 32768;          // the chunk's q_s and v_s (score factors)
+constexpr int kOffRef = kOffQ + 2 * kQ * 4;    // the chunk's block references (4 floats)
+constexpr int kOffTot = kOffRef + 16;          // scan totals: 4 column quarters x 4 warps
 constexpr int kOffBar = kOffTot + 64;          // mbarriers
 constexpr int kNumBars = 17;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // TMEM slot, abort flag
@@ -138,24 +145,39 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *
   atomicExch(err, 1);
 }
 
-__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-__device__ __forceinline__ void store_row32(float *dst, const float *v) {
+// NK consecutive K-slices of one product: the descriptors of slice ks are the first slice's with
+// the start address moved on by ks steps (the address field counts 16-byte units, and every tile
+// lies below 256 KB, so the step is a plain add).
+template <int NK>
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, uint64_t da, uint32_t da_step, uint64_t db,
+                                          uint32_t db_step, uint32_t idesc, bool accumulate) {
 #pragma unroll
-  for (int i = 0; i < 8; i++)
-    reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  for (int ks = 0; ks < NK; ks++)
+    mma_bf16(d_tmem, da + (uint64_t)(ks * da_step), db + (uint64_t)(ks * db_step), idesc, accumulate || ks > 0);
 }
-__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const float *v) {
+
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+__device__ __forceinline__ void store_row16(float *dst, const float *v) {
 #pragma unroll
   for (int i = 0; i < 4; i++)
+    reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ void store_row16(__nv_bfloat16 *dst, const float *v) {
+#pragma unroll
+  for (int i = 0; i < 2; i++)
     reinterpret_cast<uint4 *>(dst)[i] =
         make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
                    pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
 }
 
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+}
+
 }  // namespace
 
-template <typename Tout>
+template <int NN, typename Tout>
 __global__ void __launch_bounds__(kFThreads, 1)
 ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC) {
@@ -163,6 +185,7 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
   unsigned char *sXW = smem + kOffXW;
   unsigned char *sSH = smem + kOffSH, *sGP = smem + kOffGP;
   float *qs = reinterpret_cast<float *>(smem + kOffQ);
+  float *vs = qs + kQ, *rref = reinterpret_cast<float *>(smem + kOffRef);
   float *tot = reinterpret_cast<float *>(smem + kOffTot);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
@@ -170,7 +193,7 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
-  const int N = (int)p.N;  // 64 or 128
+  constexpr int N = NN;  // 64 or 128
   const int64_t L = p.L, nC = (L + kQ - 1) / kQ;
 
   if (threadIdx.x == 0) {
@@ -184,13 +207,14 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       mbar_init(bars + FULL_X + i, 1);
       mbar_init(bars + XEMPTY + i, 1);
       mbar_init(bars + GFULL + i, 1);
-      mbar_init(bars + GFREE + i, 8);
+      mbar_init(bars + GFREE + i, 16);
+
     }
-    mbar_init(bars + HX_READY, 8);
+    mbar_init(bars + HX_READY, 16);
     mbar_init(bars + S_DONE, 1);
-    mbar_init(bars + GP_READY, 8);
+    mbar_init(bars + GP_READY, 16);
     mbar_init(bars + Y_FULL, 1);
-    mbar_init(bars + Y_FREE, 8);
+    mbar_init(bars + Y_FREE, 16);
   }
   // zero what no load or score ever writes: the B rows n >= N (read by the state product as
   // M rows) and the score blocks above the diagonal of G'
@@ -215,20 +239,14 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
   const uint32_t tG0 = tbase, tY1 = tbase + 256, tY2 = tbase + 320, tH = tbase + 384;
 
   if (warp == 0) {
-    // ---- producer: X of chunk c once its buffer is free, then C and B once S_c-1 consumed them
+    // ---- producer: C and B of chunk c once the state product of chunk c-2 released their buffer,
+    //      then X once G' X of chunk c-2 released its buffer
     if (lane == 0 && !*abort_flag) {
       const uint32_t bytesX = (kP / 8) * kRowBytes;
       const uint32_t bytesCB = 2u * (uint32_t)(N / 8) * kRowBytes;
-      uint32_t nX[2] = {0u, 0u}, nCB[2] = {0u, 0u};
+      uint32_t nX0 = 0u, nX1 = 0u, nCB0 = 0u, nCB1 = 0u;  // copies issued per buffer
       for (int64_t c = 0; c < nC; c++) {
         const int xb = (int)(c & 1);
-        if (c < 2 || fwait(bars + XEMPTY + xb, (uint32_t)(((c >> 1) - 1) & 1), abort_flag, p.error)) {
-          unsigned char *dst = smem + kOffX + xb * 16384;
-          mbar_expect_tx(bars + FULL_X + xb, bytesX);
-          for (int j = 0; j < kP / 8; j++)
-            tma_load_3d(dst + j * kRowBytes, &tmX, j * 8, (int)(c * kQ), (int)bh, bars + FULL_X + xb);
-          nX[xb]++;
-        }
         if (c < 2 || fwait(bars + CBEMPTY + xb, (uint32_t)(((c >> 1) - 1) & 1), abort_flag, p.error)) {
           unsigned char *sC = smem + kOffC + xb * kCBStride, *sB = sC + 32768;
           mbar_expect_tx(bars + FULL_CB + xb, bytesCB);
@@ -236,14 +254,21 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
             tma_load_3d(sC + j * kRowBytes, &tmC, j * 8, (int)(c * kQ), (int)b, bars + FULL_CB + xb);
             tma_load_3d(sB + j * kRowBytes, &tmB, j * 8, (int)(c * kQ), (int)b, bars + FULL_CB + xb);
           }
-          nCB[xb]++;
+          (xb ? nCB1 : nCB0)++;
+        }
+        if (c < 2 || fwait(bars + XEMPTY + xb, (uint32_t)(((c >> 1) - 1) & 1), abort_flag, p.error)) {
+          unsigned char *dst = smem + kOffX + xb * 16384;
+          mbar_expect_tx(bars + FULL_X + xb, bytesX);
+          for (int j = 0; j < kP / 8; j++)
+            tma_load_3d(dst + j * kRowBytes, &tmX, j * 8, (int)(c * kQ), (int)bh, bars + FULL_X + xb);
+          (xb ? nX1 : nX0)++;
         }
       }
       // every issued copy lands before the CTA may exit
-      for (int i = 0; i < 2; i++) {
-        if (nCB[i]) drain_wait(bars + FULL_CB + i, (nCB[i] - 1) & 1, p.error);
-        if (nX[i]) drain_wait(bars + FULL_X + i, (nX[i] - 1) & 1, p.error);
-      }
+      if (nCB0) drain_wait(bars + FULL_CB, (nCB0 - 1) & 1, p.error);
+      if (nCB1) drain_wait(bars + FULL_CB + 1, (nCB1 - 1) & 1, p.error);
+      if (nX0) drain_wait(bars + FULL_X, (nX0 - 1) & 1, p.error);
+      if (nX1) drain_wait(bars + FULL_X + 1, (nX1 - 1) & 1, p.error);
     }
   } else if (warp == 1) {
     // ---- tensor-core issue, one thread
@@ -253,58 +278,77 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       constexpr uint32_t idS = instr_desc(128, kP, 1, 1);
       uint64_t *last_bar = nullptr;  // the barrier of the latest commit, and its phase
       uint32_t last_phase = 0;
-      for (int64_t c = 0; c < nC; c++) {
-        const int gb = (int)(c & 1);
-        const uint32_t tG = tG0 + gb * 128;
-        const unsigned char *sC = smem + kOffC + gb * kCBStride, *sB = sC + 32768;
-        // G = C B^T
-        if (fwait(bars + FULL_CB + gb, (uint32_t)((c >> 1) & 1), abort_flag, p.error) &&
-            (c < 2 || fwait(bars + GFREE + gb, (uint32_t)(((c >> 1) - 1) & 1), abort_flag, p.error))) {
+      // every operand descriptor, built once: C / B of either buffer as K-major operands (G, C H),
+      // B as the MN-major A operand of the state product, X of either buffer, diag(w) X, the bf16
+      // state and G'. Steps per K-slice of 16, in 16-byte units: 2 K-groups of a K-major tile
+      // (2 x 2048 bytes), 2 of an MN-major one (2 x 128 bytes).
+      constexpr uint32_t kKStep = 2 * kRowBytes / 16, kMStep = 256 / 16;
+      const uint64_t dCk0 = smem_desc(smem + kOffC, kRowBytes, 128);
+      const uint64_t dCk1 = smem_desc(smem + kOffC + kCBStride, kRowBytes, 128);
+      const uint64_t dBk0 = smem_desc(smem + kOffC + 32768, kRowBytes, 128);
+      const uint64_t dBk1 = smem_desc(smem + kOffC + kCBStride + 32768, kRowBytes, 128);
+      const uint64_t dBm0 = smem_desc(smem + kOffC + 32768, 128, kRowBytes);
+      const uint64_t dBm1 = smem_desc(smem + kOffC + kCBStride + 32768, 128, kRowBytes);
+      const uint64_t dX0 = smem_desc(smem + kOffX, 128, kRowBytes);
+      const uint64_t dX1 = smem_desc(smem + kOffX + 16384, 128, kRowBytes);
+      const uint64_t dXW = smem_desc(sXW, 128, kRowBytes), dSH = smem_desc(sSH, 128, (uint32_t)N * 16);
+      const uint64_t dGP = smem_desc(sGP, kRowBytes, 128);
+      // G = C B^T of chunk cc into G buffer cc & 1, once its C and B landed and the compute warps
+      // read out that buffer's previous G
+      auto issue_g = [&](int64_t cc) {
+        const int gb = (int)(cc & 1);
+        if (fwait(bars + FULL_CB + gb, (uint32_t)((cc >> 1) & 1), abort_flag, p.error) &&
+            (cc < 2 || fwait(bars + GFREE + gb, (uint32_t)(((cc >> 1) - 1) & 1), abort_flag, p.error))) {
           tc_fence_after();
-          for (int ks = 0; ks < N / 16; ks++)
-            mma_bf16(tG, smem_desc(sC + ks * 2 * kRowBytes, kRowBytes, 128),
-                     smem_desc(sB + ks * 2 * kRowBytes, kRowBytes, 128), idG, ks > 0);
+          mma_chain<N / 16>(tG0 + gb * 128, gb ? dCk1 : dCk0, kKStep, gb ? dBk1 : dBk0, kKStep, idG, false);
           mma_commit(bars + GFULL + gb);
           last_bar = bars + GFULL + gb;
-          last_phase = (uint32_t)((c >> 1) & 1);
+          last_phase = (uint32_t)((cc >> 1) & 1);
         }
+      };
+      issue_g(0);
+      for (int64_t c = 0; c < nC; c++) {
+        const int cb = (int)(c & 1);
         // C H_{c-1} into the second output accumulator; H += B^T diag(w) X
         if (fwait(bars + HX_READY, (uint32_t)(c & 1), abort_flag, p.error) &&
             (c < 1 || fwait(bars + Y_FREE, (uint32_t)((c - 1) & 1), abort_flag, p.error))) {
           tc_fence_after();
-          for (int ks = 0; ks < N / 16; ks++)
-            mma_bf16(tY2, smem_desc(sC + ks * 2 * kRowBytes, kRowBytes, 128),
-                     smem_desc(sSH + ks * 256, 128, (uint32_t)N * 16), idY, ks > 0);
-          for (int ks = 0; ks < kQ / 16; ks++)
-            mma_bf16(tH, smem_desc(sB + ks * 256, 128, kRowBytes),
-                     smem_desc(sXW + ks * 256, 128, kRowBytes), idS, true);
+          mma_chain<N / 16>(tY2, cb ? dCk1 : dCk0, kKStep, dSH, kMStep, idY, false);
+          mma_chain<kQ / 16>(tH, cb ? dBm1 : dBm0, kMStep, dXW, kMStep, idS, true);
           mma_commit(bars + S_DONE);
-          mma_commit(bars + CBEMPTY + gb);
-          last_bar = bars + CBEMPTY + gb;
+          mma_commit(bars + CBEMPTY + cb);
+          last_bar = bars + CBEMPTY + cb;
           last_phase = (uint32_t)((c >> 1) & 1);
+        }
+        // the next chunk's C B^T now if its tiles and its G buffer are ready (so that its scores
+        // do not wait for the tensor core), else right after G' X
+        bool g_next = c + 1 < nC;
+        if (g_next && poll_once(bars + FULL_CB + ((c + 1) & 1), (uint32_t)(((c + 1) >> 1) & 1)) &&
+            (c + 1 < 2 || poll_once(bars + GFREE + ((c + 1) & 1), (uint32_t)((((c + 1) >> 1) - 1) & 1)))) {
+          issue_g(c + 1);
+          g_next = false;
         }
         // G' X into the first output accumulator
-        const int xb = (int)(c & 1);
         if (fwait(bars + GP_READY, (uint32_t)(c & 1), abort_flag, p.error) &&
-            fwait(bars + FULL_X + xb, (uint32_t)((c >> 1) & 1), abort_flag, p.error)) {
+            fwait(bars + FULL_X + cb, (uint32_t)((c >> 1) & 1), abort_flag, p.error)) {
           tc_fence_after();
-          const unsigned char *sX = smem + kOffX + xb * 16384;
-          for (int ks = 0; ks < kQ / 16; ks++)
-            mma_bf16(tY1, smem_desc(sGP + ks * 2 * kRowBytes, kRowBytes, 128),
-                     smem_desc(sX + ks * 256, 128, kRowBytes), idY, ks > 0);
+          mma_chain<kQ / 16>(tY1, dGP, kKStep, cb ? dX1 : dX0, kMStep, idY, false);
           mma_commit(bars + Y_FULL);
-          mma_commit(bars + XEMPTY + xb);
-          last_bar = bars + XEMPTY + xb;
+          mma_commit(bars + XEMPTY + cb);
+          last_bar = bars + XEMPTY + cb;
           last_phase = (uint32_t)((c >> 1) & 1);
         }
+        if (g_next) issue_g(c + 1);
       }
       // no product in flight when the CTA frees its tensor memory
       if (last_bar) drain_wait(last_bar, last_phase, p.error);
     }
   } else {
-    // ---- compute warps: thread (row r, half hf); row r is step t (outputs, scores, X) or state n
-    const int hf = (warp - 2) >> 2, q = warp & 3, r = q * 32 + lane;
+    // ---- compute warps: thread (row r, column quarter cq); row r is step t (outputs, scores, X) or
+    //      state n, the quarter picks 16 of the P columns and 8 of every 32-column score block
+    const int cq = (warp - 2) >> 2, q = warp & 3, r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const int p0 = cq * 16;  // this thread's columns of X, H and y
     const float A = -expf(p.A_log[h]);
     const float dtb = p.dt_bias ? p.dt_bias[h] : 0.f, Dh = p.D ? p.D[h] : 0.f;
     const __nv_bfloat16 *dtrow = static_cast<const __nv_bfloat16 *>(p.dt) + bh * L;
@@ -313,18 +357,17 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
 
     // the entering state (h0 or zero) into tensor memory
     if (has_h) {
-      float hv[32];
-      const float *src = p.h0 ? p.h0 + (bh * N + r) * kP + hf * 32 : nullptr;
+      float hv[16];
+      const float *src = p.h0 ? p.h0 + (bh * N + r) * kP + p0 : nullptr;
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
+      for (int i = 0; i < 4; i++) {
         const float4 v = src ? reinterpret_cast<const float4 *>(src)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         hv[4 * i] = v.x;
         hv[4 * i + 1] = v.y;
         hv[4 * i + 2] = v.z;
         hv[4 * i + 3] = v.w;
       }
-      tmem_st<16>(tH + lane_off + hf * 32, hv);
-      tmem_st<16>(tH + lane_off + hf * 32 + 16, hv + 16);
+      tmem_st<16>(tH + lane_off + p0, hv);
       tmem_wait_st();
     }
 
@@ -333,13 +376,12 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        float y1[32], y2[32];
-        tmem_ld32(tY1 + lane_off + hf * 32, y1);
-        tmem_ld32(tY2 + lane_off + hf * 32, y2);
+        float y1[16], y2[16];
+        tmem_ld2<16>(tY1 + lane_off + p0, y1, tY2 + lane_off + p0, y2);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y1[i] = fmaf(et, y2[i], y1[i]);
+        for (int i = 0; i < 16; i++) y1[i] = fmaf(et, y2[i], y1[i]);
         const int64_t t = cc * kQ + r;
-        if (t < L) store_row32(yh + t * kP + hf * 32, y1);
+        if (t < L) store_row16(yh + t * kP + p0, y1);
       }
       tc_fence_before();
       __syncwarp();
@@ -350,13 +392,12 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
     float et_prev = 0.f;
     for (int64_t c = 0; c < nC; c++) {
       // (1) decay coefficients of step r: Delta, log a = Delta A, beta; the running sum of log a
-      //     over the chunk by a warp scan plus the earlier warps' totals (each half on its own)
+      //     over the chunk by a warp scan plus the earlier warps' totals (each quarter on its own)
       const int64_t tg = c * kQ + r;
-      const bool valid = tg < L;
       const float v = dt_next + dtb;
       dt_next = (tg + kQ < L) ? to_f32(dtrow[tg + kQ]) : 0.f;  // the next chunk's, early
       float la = 0.f, beta = 0.f;
-      if (valid) {
+      if (tg < L) {
         const float dl = p.delta_softplus ? softplus<false>(v) : v;
         la = dl * A;
         beta = p.euler ? dl : expm1f(la) / A;  // padded steps: a = 1, beta = 0 (identity)
@@ -367,12 +408,12 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
         const float o = __shfl_up_sync(0xffffffffu, cum, off);
         if (lane >= off) cum += o;
       }
-      if (lane == 31) tot[hf * 4 + q] = cum;
+      if (lane == 31) tot[cq * 4 + q] = cum;
       compute_bar();
       float cend = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        const float s = tot[hf * 4 + i];
+        const float s = tot[cq * 4 + i];
         if (i < q) cum += s;
         cend += s;
       }
@@ -380,8 +421,18 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       const float et = __expf(cum);
       const float wgt = beta * __expf(cend - cum);  // row weight of the state product
       const float a = __expf(cend);                 // decay of the whole chunk
-      if (hf == 0) qs[r] = ct - lg2_approx(beta);   // beta = 0: +inf, a zero score
-      compute_bar();                                // every q_s in place
+      // score factors: q_s for the diagonal blocks, and for the blocks below the diagonal
+      // v_s = beta_s e^{cum_ref - cum_s}, with cum_ref the running sum at the last step of s's
+      // 32-step block (the last lane of this warp), so that a score there is
+      // G[t,s] e^{cum_t - cum_ref} v_s with both factors at most 1 (and v_s at most beta_s)
+      const float qv_r = ct - lg2_approx(beta);      // beta = 0: +inf, a zero score
+      const float cref = __shfl_sync(0xffffffffu, ct, 31);
+      if (cq == 0) {
+        qs[r] = qv_r;
+        vs[r] = ex2_approx(cref - qv_r);
+        if (lane == 31) rref[q] = ct;
+      }
+      compute_bar();                                // every q_s, v_s and block reference in place
 
       // (2) H_{c-1} -> bf16 operand, H *= a; X -> diag(w) X
       const int xb = (int)(c & 1);
@@ -391,32 +442,26 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       if (ok) {
         tc_fence_after();
         if (has_h) {
-          float hv[32];
-          tmem_ld32(tH + lane_off + hf * 32, hv);
+          float hv[16];
+          tmem_ld2<8>(tH + lane_off + p0, hv, tH + lane_off + p0 + 8, hv + 8);
 #pragma unroll
-          for (int j = 0; j < 4; j++)
-            *reinterpret_cast<uint4 *>(sSH + ((hf * 4 + j) * N + r) * 16) =
+          for (int j = 0; j < 2; j++)
+            *reinterpret_cast<uint4 *>(sSH + ((cq * 2 + j) * N + r) * 16) =
                 make_uint4(pack_bf16(hv[8 * j], hv[8 * j + 1]), pack_bf16(hv[8 * j + 2], hv[8 * j + 3]),
                            pack_bf16(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16(hv[8 * j + 6], hv[8 * j + 7]));
 #pragma unroll
-          for (int i = 0; i < 32; i++) hv[i] *= a;
-          tmem_st<16>(tH + lane_off + hf * 32, hv);
-          tmem_st<16>(tH + lane_off + hf * 32 + 16, hv + 16);
+          for (int i = 0; i < 16; i++) hv[i] *= a;
+          tmem_st<16>(tH + lane_off + p0, hv);
           tmem_wait_st();
         }
         const unsigned char *sX = smem + kOffX + xb * 16384;
 #pragma unroll
-        for (int j = hf * 4; j < hf * 4 + 4; j++) {
+        for (int j = cq * 2; j < cq * 2 + 2; j++) {
           const uint4 raw = *reinterpret_cast<const uint4 *>(sX + j * kRowBytes + r * 16);
-          const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-          uint4 o;
-          uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const float2 f = __bfloat1622float2(x2[i]);
-            ow[i] = pack_bf16(f.x * wgt, f.y * wgt);
-          }
-          *reinterpret_cast<uint4 *>(sXW + j * kRowBytes + r * 16) = o;
+          const float2 f0 = bf2_to_f2(raw.x), f1 = bf2_to_f2(raw.y), f2 = bf2_to_f2(raw.z), f3 = bf2_to_f2(raw.w);
+          *reinterpret_cast<uint4 *>(sXW + j * kRowBytes + r * 16) =
+              make_uint4(pack_bf16(f0.x * wgt, f0.y * wgt), pack_bf16(f1.x * wgt, f1.y * wgt),
+                         pack_bf16(f2.x * wgt, f2.y * wgt), pack_bf16(f3.x * wgt, f3.y * wgt));
         }
       }
       tc_fence_before();
@@ -428,34 +473,44 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
       if (c > 0) epilogue(c - 1, et_prev);
 
       // (4) G' = masked, decayed scores (+ D on the diagonal): row t = r, in every 32-column block
-      //     on or below the diagonal the 16 columns of this half
+      //     on or below the diagonal the 8 columns of this quarter. All four blocks' columns are
+      //     read in one go (the ones above the diagonal are not used).
       ok = fwait(bars + GFULL + xb, (uint32_t)((c >> 1) & 1), abort_flag, p.error);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        const uint32_t tg_addr = tG0 + xb * 128 + lane_off;
-#pragma unroll 1
-        for (int kb = 0; kb <= q; kb++) {
-          const int s0 = kb * 32 + hf * 16;
-          float g[16];
-          tmem_ld2<8>(tg_addr + s0, g, tg_addr + s0 + 8, g + 8);
-          const bool diag = kb == q;
+        const uint32_t tg_addr = tG0 + xb * 128 + lane_off + cq * 8;
+        float g[32];
+        tmem_ld2<8>(tg_addr, g, tg_addr + 32, g + 8);
+        tmem_ld2<8>(tg_addr + 64, g + 16, tg_addr + 96, g + 24);
 #pragma unroll
-          for (int e = 0; e < 16; e += 8) {
-            const float4 q0 = *reinterpret_cast<const float4 *>(qs + s0 + e);
-            const float4 q1 = *reinterpret_cast<const float4 *>(qs + s0 + e + 4);
-            const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-            float o[8];
+        for (int kb = 0; kb < 4; kb++) {
+          if (kb > q) break;  // warp-uniform: the blocks above the diagonal stay zero
+          const int s0 = kb * 32 + cq * 8;
+          float o[8];
+          if (kb < q) {
+            // below the diagonal: G[t,s] e^{cum_t - cum_ref} v_s
+            const float u = ex2_approx(ct - rref[kb]);
+            const float4 v0 = *reinterpret_cast<const float4 *>(vs + s0);
+            const float4 v1 = *reinterpret_cast<const float4 *>(vs + s0 + 4);
+            const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int j = 0; j < 8; j++) o[j] = g[kb * 8 + j] * u * vv[j];
+          } else {
+            // the diagonal block: one exp per score, s <= t, D on the diagonal
+            const float4 q0 = *reinterpret_cast<const float4 *>(qs + s0);
+            const float4 q1 = *reinterpret_cast<const float4 *>(qs + s0 + 4);
+            const float qq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
             for (int j = 0; j < 8; j++) {
-              const int s = s0 + e + j;
-              const float sv = g[e + j] * ex2_approx(ct - qv[j]);
-              o[j] = (!diag || s < r) ? sv : (s == r ? sv + Dh : 0.f);
+              const int s = s0 + j;
+              const float sv = g[kb * 8 + j] * ex2_approx(ct - qq[j]);
+              o[j] = s < r ? sv : (s == r ? sv + Dh : 0.f);
             }
-            *reinterpret_cast<uint4 *>(sGP + ((s0 + e) >> 3) * kRowBytes + r * 16) =
-                make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
-                           pack_bf16(o[6], o[7]));
           }
+          *reinterpret_cast<uint4 *>(sGP + (s0 >> 3) * kRowBytes + r * 16) =
+              make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                         pack_bf16(o[6], o[7]));
         }
       }
       tc_fence_before();
@@ -470,11 +525,11 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
     epilogue(nC - 1, et_prev);
     // the state after the last step (the last state product is done: it precedes G' X)
     if (p.h_last && has_h && __all_sync(0xffffffffu, *abort_flag == 0)) {
-      float hv[32];
-      tmem_ld32(tH + lane_off + hf * 32, hv);
-      float *dst = p.h_last + (bh * N + r) * kP + hf * 32;
+      float hv[16];
+      tmem_ld2<8>(tH + lane_off + p0, hv, tH + lane_off + p0 + 8, hv + 8);
+      float *dst = p.h_last + (bh * N + r) * kP + p0;
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+      for (int i = 0; i < 4; i++)
         reinterpret_cast<float4 *>(dst)[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
     }
   }
@@ -524,7 +579,8 @@ cudaError_t launch_ssd_fused(const SsdParams &p, int out_bf16, cudaStream_t s) {
       !encode_rows_map(&mB, p.B, (uint64_t)p.N, (uint64_t)p.L, (uint64_t)p.Bt) ||
       !encode_rows_map(&mC, p.C, (uint64_t)p.N, (uint64_t)p.L, (uint64_t)p.Bt))
     return cudaErrorNotSupported;  // the driver declined a tensor map; nothing was launched
-  auto kern = out_bf16 ? ssd_fused_kernel<__nv_bfloat16> : ssd_fused_kernel<float>;
+  auto kern = p.N == 64 ? (out_bf16 ? ssd_fused_kernel<64, __nv_bfloat16> : ssd_fused_kernel<64, float>)
+                        : (out_bf16 ? ssd_fused_kernel<128, __nv_bfloat16> : ssd_fused_kernel<128, float>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
   if (e != cudaSuccess) return e;
   if (p.timing_events && p.timing_events[0] &&
