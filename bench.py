@@ -436,6 +436,116 @@ def ssd_bench(args, cfg, name):
     return 0
 
 
+def decode_bench(args, w):
+    """Token-by-token decode through the C ABI (ssm_scan_step, one launch per token): T tokens of
+    Bt sequences, each token's x, dt, z, B, C its own resident arrays, the state and conv history
+    carried in place. Timed as replays of one CUDA graph holding the T launches (the way a decode
+    loop runs them), and as T plain launches from the host."""
+    import ctypes
+    import torch
+    from selective_state_space_34_b200 import _abi
+    from selective_state_space_34_b200 import workloads as wl
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    Bt, Dn, N, T, K = w.Bt, w.Dn, w.N, w.L, w.K
+    a = wl.generate(w, seed=w.seed + rank)
+    bf = torch.bfloat16
+    # token-major copies: token t's x / dt / z are (Bt, Dn), its B / C (Bt, N)
+    tok = {k: torch.from_numpy(np.ascontiguousarray(np.moveaxis(a[k], -1, 0))).to(dev, bf) for k in ("x", "dt", "z", "B", "C")}
+    par = {k: torch.from_numpy(a[k]).to(dev, torch.float32) for k in ("A_log", "D", "dt_bias", "conv_w", "conv_b")}
+    h = torch.zeros((Bt, Dn, N), dtype=torch.float32, device=dev)
+    hist = torch.zeros((Bt, Dn, K - 1), dtype=bf, device=dev)
+    out = torch.empty((T, Bt, Dn), dtype=bf, device=dev)
+    lib = _abi.load()
+    steps = []
+    for t in range(T):
+        sa = _abi.StepArgs()
+        sa.x, sa.dt, sa.z = tok["x"][t].data_ptr(), tok["dt"][t].data_ptr(), tok["z"][t].data_ptr()
+        sa.B, sa.C = tok["B"][t].data_ptr(), tok["C"][t].data_ptr()
+        sa.A_log, sa.D, sa.dt_bias = par["A_log"].data_ptr(), par["D"].data_ptr(), par["dt_bias"].data_ptr()
+        sa.conv_w, sa.conv_b = par["conv_w"].data_ptr(), par["conv_b"].data_ptr()
+        sa.h, sa.conv_hist, sa.out = h.data_ptr(), hist.data_ptr(), out[t].data_ptr()
+        sa.Bt, sa.Dn, sa.N, sa.K = Bt, Dn, N, K
+        sa.in_dtype, sa.out_dtype, sa.delta_softplus, sa.discretization = _abi.SSM_BF16, _abi.SSM_BF16, 1, _abi.SSM_ZOH
+        steps.append(sa)
+    s = torch.cuda.Stream(dev)
+
+    def run_tokens():
+        for sa in steps:
+            _abi.check("ssm_scan_step", lib.ssm_scan_step(ctypes.byref(sa), s.cuda_stream))
+
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            run_tokens()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run_tokens()
+    torch.cuda.synchronize()
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    e0, e1 = E(), E()
+    e0.record(s)
+    with torch.cuda.stream(s):
+        for _ in range(args.steps):
+            g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps  # per replay of T tokens
+    # the same T tokens as plain launches from the host
+    f0, f1 = E(), E()
+    f0.record(s)
+    with torch.cuda.stream(s):
+        run_tokens()
+    f1.record(s)
+    torch.cuda.synchronize()
+    eager_ms = f0.elapsed_time(f1)
+    us_tok = ms * 1e3 / T
+    # algorithmic bytes of one token step: per (sequence, channel) the state read and written
+    # (N fp32 each way), the conv history read and written ((K-1) bf16 each way), x, dt, z in and
+    # the output (bf16); per sequence B and C (bf16); the parameters once
+    bytes_step = (Bt * Dn * (N * 4 * 2 + (K - 1) * 2 * 2 + 3 * 2 + 2) + Bt * N * 2 * 2
+                  + Dn * (N + 3 + K) * 4)
+    peaks = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = bytes_step / (us_tok * 1e-6) / 1e9
+    line = {
+        "metric": "decode tokens/s (sequences x tokens per second), 1xB200", "value": Bt * T * world / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "Bt": Bt, "Dn": Dn, "N": N, "K": K, "tokens_per_step": T,
+                   "step": "%d decode steps (one launch each) replayed as one CUDA graph" % T,
+                   "state": "%.1f MB of state and conv history, resident in L2 across tokens"
+                            % ((Bt * Dn * (N * 4 + (K - 1) * 2)) / 1e6)},
+        "us_per_token_step": us_tok,
+        "eager_us_per_token_step": eager_ms * 1e3 / T,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "algorithmic_bytes": bytes_step, "kernel": "ssm_step_kernel",
+                     "traffic": ncu_traffic("ssm_step_kernel", "ssm_step.cu"), "peak_source": peaks.get("source")},
+        "gpu_launches": T * args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---- our arm ----------------------------------------------------------------------------------
 
 def main():
@@ -458,6 +568,12 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     from selective_state_space_34_b200 import workloads as wl
+    if args.workload in wl.DECODE_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the decode leg has no CPU reference "
+                              "arm; its parity is in tests/test_gpu_state.py"}))
+            return 0
+        return decode_bench(args, wl.DECODE_WORKLOADS[args.workload])
     if args.workload in wl.SSD_WORKLOADS:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the state-space-duality leg has no "

@@ -166,6 +166,11 @@ def generate_ssd(Bt: int, H: int, L: int, P: int, N: int, seed: int = 1008) -> D
 # Mamba-2-style layer on the 1.4B-shaped block: d_inner 4096 as 64 heads of 64, d_state 128.
 SSD_WORKLOADS = {"ssd_fwd": dict(Bt=4, H=64, L=4096, P=64, N=128, seed=1008)}
 
+# Token-by-token decode on the 1.4B-shaped block: 64 sequences x d_inner 4096, d_state 16, conv
+# width 4, 256 tokens (one decode step each); the token inputs are the columns of a scan workload
+# of that shape, so their distributions are the scan workloads'.
+DECODE_WORKLOADS = {"decode_1p4b": Workload("decode_1p4b", 64, 4096, 16, 256, seed=1009)}
+
 
 def shaped(base: str, **overrides) -> Workload:
     """A named workload with some fields replaced (e.g. smaller Bt/Dn/L for a parity case)."""

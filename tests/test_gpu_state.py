@@ -132,7 +132,7 @@ def test_decode_steps_match_oracle(T, dtype, euler):
     assert np.array_equal(to_np(hist), ex["conv_hist"])
 
 
-@pytest.mark.parametrize("N", [1, 4, 16, 64])
+@pytest.mark.parametrize("N", [1, 4, 16, 24, 32, 33, 64])
 def test_decode_step_state_sizes_and_bf16_out(N):
     w, a, t = _setup(2, 33, N, 1, "bf16", gate=False)
     h, hist = t["h0"].clone(), t["conv_hist"].clone()
