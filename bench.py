@@ -546,6 +546,73 @@ def decode_bench(args, w):
     return 0
 
 
+def conv_bench(args, w):
+    """The standalone causal conv1d + SiLU (ssm_conv1d_silu) through the C ABI: bf16 x in, bf16 u
+    out, inputs larger than L2; a pure stream, so the roofline is HBM."""
+    import ctypes
+    import torch
+    from selective_state_space_34_b200 import _abi
+    from selective_state_space_34_b200 import workloads as wl
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    a = wl.generate(w, seed=w.seed + rank)
+    x = torch.from_numpy(a["x"]).to(dev, torch.bfloat16)
+    cw = torch.from_numpy(a["conv_w"]).to(dev, torch.float32)
+    cb = torch.from_numpy(a["conv_b"]).to(dev, torch.float32)
+    u = torch.empty_like(x)
+    lib = _abi.load()
+    s = torch.cuda.current_stream(dev)
+
+    def run():
+        _abi.check("ssm_conv1d_silu", lib.ssm_conv1d_silu(
+            x.data_ptr(), u.data_ptr(), cw.data_ptr(), cb.data_ptr(), w.Bt, w.Dn, w.L, w.K,
+            _abi.SSM_BF16, _abi.SSM_BF16, s.cuda_stream))
+
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    e0, e1 = E(), E()
+    e0.record(s)
+    for _ in range(args.steps):
+        run()
+    e1.record(s)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    nbytes = w.Bt * w.Dn * w.L * 2 * 2 + w.Dn * (w.K + 1) * 4  # x in, u out (bf16), taps and bias
+    peaks = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "causal conv1d + SiLU elements/s, 1xB200", "value": w.Bt * w.Dn * w.L * world / (ms * 1e-3),
+        "unit": "elements/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "Bt": w.Bt, "Dn": w.Dn, "L": w.L, "K": w.K,
+                   "l2": "inputs larger than L2 (%.0f MB per call)" % (nbytes / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "algorithmic_bytes": nbytes, "kernel": "conv1d_silu_vec_kernel",
+                     "traffic": ncu_traffic("conv1d_silu_vec_kernel", "ssm_conv.cu"), "peak_source": peaks.get("source")},
+        "gpu_launches": args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---- our arm ----------------------------------------------------------------------------------
 
 def main():
@@ -568,6 +635,12 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     from selective_state_space_34_b200 import workloads as wl
+    if args.workload in wl.CONV_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the conv leg has no CPU reference "
+                              "arm; its parity is in tests/test_gpu_conv.py"}))
+            return 0
+        return conv_bench(args, wl.CONV_WORKLOADS[args.workload])
     if args.workload in wl.DECODE_WORKLOADS:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the decode leg has no CPU reference "

@@ -171,6 +171,9 @@ SSD_WORKLOADS = {"ssd_fwd": dict(Bt=4, H=64, L=4096, P=64, N=128, seed=1008)}
 # of that shape, so their distributions are the scan workloads'.
 DECODE_WORKLOADS = {"decode_1p4b": Workload("decode_1p4b", 64, 4096, 16, 256, seed=1009)}
 
+# The standalone causal conv1d + SiLU over the 1.4B-shaped activations (x only is used).
+CONV_WORKLOADS = {"conv_1p4b": Workload("conv_1p4b", 4, 4096, 16, 4096, seed=1010)}
+
 
 def shaped(base: str, **overrides) -> Workload:
     """A named workload with some fields replaced (e.g. smaller Bt/Dn/L for a parity case)."""

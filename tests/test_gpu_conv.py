@@ -12,7 +12,10 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("Bt,Dn,L,K", [(2, 33, 100, 4), (1, 4, 3, 4), (1, 5, 9, 1), (3, 7, 64, 2),
-                                       (1, 3, 1, 3)])
+                                       (1, 3, 1, 3),
+                                       # rows of whole 16-byte vectors: the vector path
+                                       (2, 9, 8, 4), (1, 6, 16, 3), (2, 5, 256, 1), (1, 3, 256, 2),
+                                       (2, 7, 24, 4)])
 @pytest.mark.parametrize("dtype,odt", [("bf16", "f32"), ("bf16", "bf16"), ("f32", "f32")])
 def test_conv1d_silu(Bt, Dn, L, K, dtype, odt):
     w = wl.shaped("mamba130m_fwd", Bt=Bt, Dn=Dn, L=L, K=K, in_dtype=dtype)

@@ -210,10 +210,12 @@ def test_ssd_guards(monkeypatch, H, L, P, N, od, form):
     _same(a, b)
 
 
+@pytest.mark.parametrize("L", [333, 336])
 @pytest.mark.parametrize("K", [1, 3, 4])
-def test_conv_guards(monkeypatch, K):
+def test_conv_guards(monkeypatch, K, L):
+    # L = 336: rows of whole 16-byte vectors (the vector path); 333: element by element
     gen = torch.Generator("cuda").manual_seed(K)
-    x = torch.randn(2, 70, 333, device="cuda", generator=gen).to(torch.bfloat16)
+    x = torch.randn(2, 70, L, device="cuda", generator=gen).to(torch.bfloat16)
     w = torch.randn(70, K, device="cuda", generator=gen) * 0.3
     b = torch.randn(70, device="cuda", generator=gen) * 0.1
 
