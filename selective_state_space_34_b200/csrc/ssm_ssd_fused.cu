@@ -18,9 +18,9 @@
 // decay coefficients, (2) copy H_{c-1} out of tensor memory as the bf16 operand of C H_{c-1},
 // scale H in place by e^{cum_end}, and write diag(w) X, (3) finish chunk c-1's output from its two
 // accumulators, and (4) turn G into G'. The MMA warp issues C H_{c-1} and the state product of
-// chunk c after step (2), then G of chunk c+1, then G' X of chunk c after step (4), so the tensor
-// core works on one chunk while the compute warps are on the other and the next chunk's G is
-// ready before the compute warps need it. G is double-buffered in tensor memory, C, B and X in
+// chunk c after step (2), then G of chunk c+1 if its tiles have landed (else right after G' X),
+// then G' X of chunk c after step (4), so the tensor core works on one chunk while the compute
+// warps are on the other and the next chunk's G is usually ready before they need it. G is double-buffered in tensor memory, C, B and X in
 // shared memory; the scaled X, the bf16 state and G' are single buffers whose reuse is ordered by
 // the barriers below. Every wait is bounded; a wait that runs out records the error word and an
 // abort flag, after which every role runs its loop to the end without issuing work, waits for its
