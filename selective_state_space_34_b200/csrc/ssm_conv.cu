@@ -48,6 +48,8 @@ conv1d_silu_kernel(const Tin *__restrict__ x, Tout *__restrict__ u, const float 
   }
 }
 
+namespace {  // helpers of this file only
+
 __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *v) {
   const uint4 r = *reinterpret_cast<const uint4 *>(p);
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
@@ -77,6 +79,8 @@ __device__ __forceinline__ void store8(float *p, const float *v) {
   reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
   reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
+
+}  // namespace
 
 // Rows of whole 8-element vectors, 16-byte aligned: R consecutive runs of 8 per thread, loaded and
 // stored with 16-byte accesses; the halo is the last 3 elements of the vector before them.
