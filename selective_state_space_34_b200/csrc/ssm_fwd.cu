@@ -12,12 +12,16 @@
 // nothing is computed twice; u and Delta reach the other lanes through shared memory and the G
 // partial readouts sum_n C h are combined through shared memory.
 //
-// Staging: each stage's x, dt, z rows and B, C rows are streamed global -> shared with 16-byte
-// cp.async (double-buffered, one stage in flight while the previous one is computed). The conv
-// halo of 3 steps is carried across stages in a prefix in front of each x row.
+// Staging: each stage's x, dt, z rows and B, C rows are streamed global -> shared (double-buffered,
+// one stage in flight while the previous one is computed). Where rows are 16-byte aligned, x, dt and
+// z arrive as one TMA box each (cp.async.bulk.tensor, issued by one thread, completion counted on
+// the buffer's mbarrier): the x box starts kPre steps early, so it also brings the conv halo in
+// front of each row. Otherwise every thread copies its share element by element and the halo of 3
+// steps is carried across stages in the prefix. B and C go through registers (transposed, fp32).
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
+#include "ssm_tc.cuh"
 
 namespace ssm {
 
@@ -37,14 +41,18 @@ template <int G, int NS, typename Tin, int NT> struct FwdSmem {
   static constexpr size_t cs_off = bs_off + sizeof(float) * 2 * kT * BS;
   static constexpr size_t ud_off = cs_off + sizeof(float) * 2 * kT * BS;
   static constexpr size_t yp_off = ud_off + sizeof(float2) * CH * US;
-  static constexpr size_t bytes = yp_off + sizeof(float) * CH * YC;
+  static constexpr size_t bar_off = (yp_off + sizeof(float) * CH * YC + 7) / 8 * 8;  // 2 mbarriers
+  static constexpr size_t bytes = bar_off + 16;
+  static_assert(dt_off % 128 == 0 && z_off % 128 == 0 && (sizeof(Tin) * CH * XS) % 128 == 0 &&
+                (sizeof(Tin) * CH * kT) % 128 == 0, "TMA destinations are 128-byte aligned");
 };
 
 // SUMMARY: pass 1 of the split-L forward -- the segment's recurrence from a zero state, keeping
 // only its end state and its sum of Delta (no readout, no outputs).
 template <int G, int NS, typename Tin, typename Tout, int NT, bool EULER, bool SUMMARY>
 __global__ void __launch_bounds__(NT, 512 / NT)
-ssm_fwd_kernel(const FwdParams p) {
+ssm_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap tmx,
+               const __grid_constant__ CUtensorMap tmdt, const __grid_constant__ CUtensorMap tmz) {
   using S = FwdSmem<G, NS, Tin, NT>;
   constexpr int CH = S::CH, NP = S::NP, EPL = kSub / G;
   constexpr bool PRECISE = sizeof(Tin) == 4;
@@ -56,6 +64,7 @@ ssm_fwd_kernel(const FwdParams p) {
   float *Cs = reinterpret_cast<float *>(smem + S::cs_off);
   float2 *ud = reinterpret_cast<float2 *>(smem + S::ud_off);
   float *yp = reinterpret_cast<float *>(smem + S::yp_off);
+  uint64_t *sbar = reinterpret_cast<uint64_t *>(smem + S::bar_off);
 
   const int64_t n_dtiles = (p.Dn + CH - 1) / CH;
   const int64_t per_seg = n_dtiles * p.Bt;
@@ -113,7 +122,12 @@ ssm_fwd_kernel(const FwdParams p) {
   // conv-halo prefixes of both x buffers: the kPre inputs before the first step -- from x itself
   // for a later segment, else the carried history (newest-first), zero where there is none
   const Tin *hist = (has_conv && p.conv_hist && p.K > 1) ? static_cast<const Tin *>(p.conv_hist) : nullptr;
-  for (int i = tid; i < 2 * CH * kPre; i += NT) {
+  const bool tma = p.tma && (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 127u) == 0;
+  if (tma && tid == 0) {
+    mbar_init(sbar, 1);
+    mbar_init(sbar + 1, 1);
+  }
+  for (int i = tid; !tma && i < 2 * CH * kPre; i += NT) {
     const int r = i / kPre, k = i % kPre, j = kPre - 1 - k;  // x_{ts-1-j}
     Tin v = zero_val<Tin>();
     if (r < rows_valid) {
@@ -128,6 +142,18 @@ ssm_fwd_kernel(const FwdParams p) {
   const int64_t n_stages = (te - ts + kT - 1) / kT;
   auto issue = [&](int64_t stage, int buf) {
     const int64_t t0 = ts + stage * kT;
+    if (tma) {
+      // x from kPre steps before the stage (its halo; a negative start reads zeros), dt, z: one box
+      // of (steps, channels) each; rows past Dn and steps past L read zeros
+      if (tid == 0) {
+        const uint32_t bytes = (uint32_t)(sizeof(Tin) * CH * (S::XS + kT * (has_z ? 2 : 1)));
+        mbar_expect_tx(sbar + buf, bytes);
+        tma_load_3d(xs + buf * CH * S::XS, &tmx, (int)(t0 - kPre), (int)d0, (int)b, sbar + buf);
+        tma_load_3d(dts + buf * CH * kT, &tmdt, (int)t0, (int)d0, (int)b, sbar + buf);
+        if (has_z) tma_load_3d(zs + buf * CH * kT, &tmz, (int)t0, (int)d0, (int)b, sbar + buf);
+      }
+      return;
+    }
     stage_rows<Tin, CH, kT, NT>(xs + buf * CH * S::XS + kPre, S::XS, gx, L, rows_valid, t0, L, vec);
     stage_rows<Tin, CH, kT, NT>(dts + buf * CH * kT, kT, gdt, L, rows_valid, t0, L, vec);
     if (has_z) stage_rows<Tin, CH, kT, NT>(zs + buf * CH * kT, kT, gz, L, rows_valid, t0, L, vec);
@@ -136,16 +162,30 @@ ssm_fwd_kernel(const FwdParams p) {
 
   BCStager<Tin, NP, NT> bc;
   float sdl = 0.0f;  // sum of Delta over the segment (SUMMARY)
+  if (tma) __syncthreads();  // the barriers are initialised before anyone polls them
   if (n_stages > 0) {
     issue(0, 0);
     bc.load(gB, gC, n_rows, ts, L, vec);
     bc.store(Bs, Cs, S::BS);
     if (n_stages > 1) bc.load(gB, gC, n_rows, ts + kT, L, vec);
+    if (tma && ts == 0 && hist) {
+      // the carried inputs before step 0 (newest-first) replace the zeros of the first box's halo,
+      // once it has landed (the wait at the top of stage 0 then returns at once)
+      mbar_wait(sbar, 0u);
+      for (int i = tid; i < CH * (p.K - 1); i += NT) {
+        const int r = i / (p.K - 1), j = i % (p.K - 1);
+        if (r < rows_valid) xs[r * S::XS + kPre - 1 - j] = hist[(b * p.Dn + d0 + r) * (p.K - 1) + j];
+      }
+    }
   }
   for (int64_t st = 0; st < n_stages; st++) {
     const int buf = (int)(st & 1), nbuf = buf ^ 1;
     const int64_t t0 = ts + st * kT;
-    cp_async_wait<0>();
+    if (tma) {
+      mbar_wait(sbar + buf, (uint32_t)((st >> 1) & 1));  // bounded; the copy completes on its own
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();  // stage st landed and Bs/Cs[buf] written; stage st-1's buffers are free
     if (st + 1 < n_stages) {
       issue(st + 1, nbuf);
@@ -191,7 +231,7 @@ ssm_fwd_kernel(const FwdParams p) {
         ud[c * S::US + g * EPL + j] = make_float2(dl, u);
         gate[j] = s;
         uown[j] = u;
-        if (t >= kT - 3)  // carry the conv halo into the next stage's prefix
+        if (!tma && t >= kT - 3)  // carry the conv halo into the next stage's prefix (TMA brings it)
           xs[(nbuf * CH + c) * S::XS + kPre + t - kT] = xrow[t];
       }
       if (!SUMMARY && p.u_out && live)
@@ -411,7 +451,18 @@ static cudaError_t launch_fwd_t(const FwdParams &p, int n_seg_launch, cudaStream
   const int64_t n_dtiles = (p.Dn + S::CH - 1) / S::CH;
   const int64_t grid = n_dtiles * p.Bt * n_seg_launch;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)grid, NT, S::bytes, stream>>>(p);
+  // TMA boxes for x (the stage plus its kPre-step halo), dt and z where the rows are 16-byte aligned
+  CUtensorMap mx, mdt, mz;
+  memset(&mx, 0, sizeof(mx));
+  memset(&mdt, 0, sizeof(mdt));
+  memset(&mz, 0, sizeof(mz));
+  FwdParams q = p;
+  constexpr bool bf = sizeof(Tin) == 2;
+  q.tma = p.vec && p.L <= 0x7fffffffLL && p.Dn <= 0x7fffffffLL &&
+          encode_tma_3d(&mx, bf, p.x, (uint64_t)p.L, (uint64_t)p.Dn, (uint64_t)p.Bt, kPre + kT, S::CH) &&
+          encode_tma_3d(&mdt, bf, p.dt, (uint64_t)p.L, (uint64_t)p.Dn, (uint64_t)p.Bt, kT, S::CH) &&
+          (!p.z || encode_tma_3d(&mz, bf, p.z, (uint64_t)p.L, (uint64_t)p.Dn, (uint64_t)p.Bt, kT, S::CH));
+  kern<<<(unsigned)grid, NT, S::bytes, stream>>>(q, mx, mdt, mz);
   return cudaGetLastError();
 }
 

@@ -2,6 +2,8 @@
 // the C-ABI layer. Host/device plain data only; no torch types anywhere in the library.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -35,6 +37,7 @@ struct FwdParams {
   int vec;  // 1: rows are 16-byte aligned, stage with cp.async and store with vector stores
   int euler;  // input discretisation: 0 exact ZOH, 1 Delta * B
   int chunked;  // one-pass scan layout: 0 states over lanes (ssm_fwd.cu), 1 chunked in time (ssm_fwd_tp.cu)
+  int tma;      // set by the launcher: stage x, dt, z with TMA boxes (the kernel's tensor maps are valid)
   const float *h0;        // (Bt, Dn, N) or null
   const void *conv_hist;  // (Bt, Dn, K-1) in-dtype or null
   float *h_last;          // (Bt, Dn, N) or null
@@ -64,6 +67,11 @@ struct SsdParams {
   int form;                    // ssm_ssd_form
 };
 cudaError_t launch_ssd(const SsdParams &p, int out_bf16, cudaStream_t stream);
+// A tensor map for TMA tile loads of a 3-D (d0 innermost, d1, d2) row-major bf16 or fp32 tensor, in
+// boxes of box0 x box1 x 1 elements with zero fill out of bounds (ssm_tma.cu); false when the driver
+// declines it.
+bool encode_tma_3d(CUtensorMap *m, bool bf16, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint32_t box0, uint32_t box1);
 // The fused one-launch form (ssm_ssd_fused.cu): P = 64, N = 64 or 128.
 bool ssd_fused_supported(const SsdParams &p);
 cudaError_t launch_ssd_fused(const SsdParams &p, int out_bf16, cudaStream_t stream);

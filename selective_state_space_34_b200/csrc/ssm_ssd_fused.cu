@@ -38,9 +38,6 @@
 //   X, XW [p/8][s][p%8]   -- MN-major B operands (N = p, K = s)
 //   SH    [p/8][n][p%8]   -- MN-major B operand (N = p, K = n)
 //   G'    [s/8][t][s%8]   -- K-major A operand (M = t, K = s)
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_tc.cuh"
@@ -95,23 +92,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(smem_u32(bar))
                : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n" ::"r"(
-                   smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// One 3-D tile load (no multicast) into this CTA's shared memory; completion is counted on bar.
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
-      "r"(smem_u32(bar))
-      : "memory");
 }
 
 __device__ __forceinline__ bool poll_once(uint64_t *bar, uint32_t parity) {
@@ -540,31 +520,10 @@ ssd_fused_kernel(const SsdParams p, const __grid_constant__ CUtensorMap tmX,
 
 namespace {
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }();
-  return fn;
-}
-
 // A (inner, rows, outer) bf16 tensor, row-major, loaded as boxes of 8 inner elements x 128 rows:
 // one box is one 8-column group of a tile, [row][8], 16 bytes a row. Rows past `rows` read zero.
 bool encode_rows_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t outer) {
-  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {inner, rows, outer};
-  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};  // bytes, of dims 1 and 2
-  cuuint32_t box[3] = {8, (cuuint32_t)kQ, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_tma_3d(m, true, base, inner, rows, outer, 8, (uint32_t)kQ);
 }
 
 }  // namespace
