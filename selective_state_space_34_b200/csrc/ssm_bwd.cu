@@ -29,6 +29,7 @@
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
+#include "ssm_tc.cuh"
 #include "ssm_tmem.cuh"
 
 namespace ssm {
@@ -93,7 +94,11 @@ template <int G, int NS, typename Tin> struct BwdSmem {
   // cluster exchange: every thread's 4-step sums of the stage, two rows (one per stage parity)
   static constexpr size_t cx_off = rb_off + (BFLY ? sizeof(float) * TS * WPT : sizeof(float) * 2 * RBW);
   static constexpr size_t slot_off = cx_off + (BFLY ? sizeof(float4) * 2 * kThreads : 0);
-  static constexpr size_t bytes = slot_off + 16;
+  static constexpr size_t bar_off = slot_off + 16;  // 2 mbarriers of the TMA stage copies
+  static constexpr size_t bytes = bar_off + 16;
+  static_assert(dt_off % 128 == 0 && z_off % 128 == 0 && do_off % 128 == 0 &&
+                (sizeof(Tin) * CH * XS) % 128 == 0 && (sizeof(Tin) * CH * TS) % 128 == 0,
+                "TMA destinations are 128-byte aligned");
   __host__ __device__ static constexpr int rb_index(int which, int tt, int c, int n) {
     return which * RBW + tt * RBT + (c / CHH) * RBC + (c % CHH) * NP + n;
   }
@@ -138,7 +143,9 @@ template <int NS> __device__ __forceinline__ void store_states(float *dst, const
 // the whole sequence and its bounds are compile-time constants of the one-pass kernel.
 template <int G, int NS, typename Tin, bool EULER, bool SEG>
 __global__ void __launch_bounds__(kThreads, SSM_BWD_MIN_CTAS)
-ssm_bwd_kernel(const BwdParams P) {
+ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
+               const __grid_constant__ CUtensorMap tmdt, const __grid_constant__ CUtensorMap tmz,
+               const __grid_constant__ CUtensorMap tmdo) {
   using S = BwdSmem<G, NS, Tin>;
   constexpr int CH = S::CH, NP = S::NP, TS = S::TS, EPL = TS / G, RH = S::RH;
   constexpr int GV = 4 * NS;  // TMEM columns of one quantity over a 4-step group
@@ -238,8 +245,28 @@ ssm_bwd_kernel(const BwdParams P) {
   for (int i = tid; i < CH * S::DCS; i += kThreads) dcs[i] = 0.f;
 
   const int64_t n_stages = (te - ts + TS - 1) / TS;
+  // TMA stage copies where the rows are 16-byte aligned: one box per tensor and stage, issued by
+  // one thread, counted on the buffer's mbarrier (x from kPre steps before the stage: its halo)
+  uint64_t *sbar = reinterpret_cast<uint64_t *>(smem + S::bar_off);
+  const bool tma = P.f.tma && (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 127u) == 0;
+  if (tma && tid == 0) {
+    mbar_init(sbar, 1);
+    mbar_init(sbar + 1, 1);
+  }
+  if (tma) __syncthreads();  // the barriers are initialised before anyone polls them
   auto issue = [&](int64_t stage, int buf) {
     const int64_t t0 = ts + stage * TS;
+    if (tma) {
+      if (tid == 0) {
+        const uint32_t bytes = (uint32_t)(sizeof(Tin) * CH * (S::XS + TS * (has_z ? 3 : 2)));
+        mbar_expect_tx(sbar + buf, bytes);
+        tma_load_3d(xs + buf * CH * S::XS, &tmx, (int)(t0 - kPre), (int)d0, (int)b, sbar + buf);
+        tma_load_3d(dts + buf * CH * TS, &tmdt, (int)t0, (int)d0, (int)b, sbar + buf);
+        if (has_z) tma_load_3d(zs + buf * CH * TS, &tmz, (int)t0, (int)d0, (int)b, sbar + buf);
+        tma_load_3d(dos + buf * CH * TS, &tmdo, (int)t0, (int)d0, (int)b, sbar + buf);
+      }
+      return;
+    }
     stage_rows<Tin, CH, kPre + TS>(xs + buf * CH * S::XS, S::XS, gx, L, rows_valid, t0 - kPre, L, vec);
     stage_rows<Tin, CH, TS>(dts + buf * CH * TS, TS, gdt, L, rows_valid, t0, L, vec);
     if (has_z) stage_rows<Tin, CH, TS>(zs + buf * CH * TS, TS, gz, L, rows_valid, t0, L, vec);
@@ -258,7 +285,10 @@ ssm_bwd_kernel(const BwdParams P) {
   for (int64_t st = n_stages - 1; st >= 0; st--) {
     const int buf = (int)(st & 1), pbuf = buf ^ 1;
     const int64_t t0 = ts + st * TS;
-    cp_async_wait<0>();
+    if (tma)  // buffers are used from the last stage down: use (n_stages - 1 - st) / 2 of buffer buf
+      mbar_wait(sbar + buf, (uint32_t)(((n_stages - 1 - st) >> 1) & 1));  // bounded
+    else
+      cp_async_wait<0>();
     __syncthreads();  // stage st landed; B/C rows of stage st written; stage st+1's buffers free
     if (st > 0) {
       issue(st - 1, pbuf);
@@ -1080,6 +1110,23 @@ static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int64_t grid = P.n_dtiles * P.f.Bt * P.n_seg;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  // TMA boxes for x (the stage plus its kPre-step halo), dt, z and dout where rows are 16-byte aligned
+  CUtensorMap mx, mdt, mz, mdo;
+  memset(&mx, 0, sizeof(mx));
+  memset(&mdt, 0, sizeof(mdt));
+  memset(&mz, 0, sizeof(mz));
+  memset(&mdo, 0, sizeof(mdo));
+  BwdParams Q = P;
+  {
+    constexpr bool bf = sizeof(Tin) == 2;
+    const FwdParams &f = P.f;
+    const uint64_t Lq = (uint64_t)f.L, Dq = (uint64_t)f.Dn, Bq = (uint64_t)f.Bt;
+    Q.f.tma = f.vec && f.L <= 0x7fffffffLL && f.Dn <= 0x7fffffffLL &&
+              encode_tma_3d(&mx, bf, f.x, Lq, Dq, Bq, kPre + S::TS, S::CH) &&
+              encode_tma_3d(&mdt, bf, f.dt, Lq, Dq, Bq, S::TS, S::CH) &&
+              (!f.z || encode_tma_3d(&mz, bf, f.z, Lq, Dq, Bq, S::TS, S::CH)) &&
+              encode_tma_3d(&mdo, bf, P.dout, Lq, Dq, Bq, S::TS, S::CH);
+  }
   if (P.cluster > 1) {
     // consecutive blocks are consecutive channel tiles of one (segment, batch element), and the
     // tile count is a multiple of the cluster size, so a cluster never straddles two of them
@@ -1095,11 +1142,11 @@ static cudaError_t launch_bwd_t(const BwdParams &P, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, P);
+    e = cudaLaunchKernelEx(&cfg, kern, Q, mx, mdt, mz, mdo);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(P);
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(Q, mx, mdt, mz, mdo);
   return cudaGetLastError();
 }
 
