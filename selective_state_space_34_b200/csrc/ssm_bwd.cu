@@ -43,10 +43,11 @@ namespace ssm {
 #define SSM_BWD_MIN_CTAS 4
 #endif
 // 1: the adjoint recomputes A_bar on the bf16 path instead of reading it back from TMEM (one
-// more exp per element-state on a pipe the backward keeps ~15% busy, 16 fewer live registers;
-// measured 2.63 -> 2.46 ms on 4x4096x16x4096, bit-identical gradients).
+// more exp per element-state, 16 fewer live registers). Measured on 4x4096x16x4096: 2.63 -> 2.46 ms
+// when the kernel spilled 60 bytes per thread; with the stages staged by TMA and the exp argument
+// formed as (Delta log2 e) A, reading A_bar back is the faster one (2.300 against 2.337 ms).
 #ifndef SSM_BWD_AREC
-#define SSM_BWD_AREC 1
+#define SSM_BWD_AREC 0
 #endif
 
 template <int G, int NS, typename Tin> struct BwdSmem {
@@ -190,11 +191,10 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
   const int64_t ts = SEG ? seg * P.seg_len : 0, te = SEG ? imin64(L, ts + P.seg_len) : L;
   const int64_t sbd = (seg * p.Bt + b) * p.Dn + d;  // row of the per-(segment, b, d) partials
 
-  // A, the exp coefficient (A, or A log2 e on the fast path) and -1/A per owned state
+  // A and -1/A per owned state (the fast path forms the exp argument as (Delta log2 e) A)
   constexpr int NH = (NS + 1) / 2;  // state pairs per lane
-  float2 A2[NH], Ac2[NH], nIA2[NH], lam2[NH], aN2[NH], dAl2[NH];
+  float2 A2[NH], nIA2[NH], lam2[NH], aN2[NH], dAl2[NH];
   float *A = reinterpret_cast<float *>(A2);
-  float *Acoef = reinterpret_cast<float *>(Ac2);
   float *nIA = reinterpret_cast<float *>(nIA2);
   float *lam = reinterpret_cast<float *>(lam2);
   float *aN = reinterpret_cast<float *>(aN2);
@@ -209,11 +209,9 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
     dAl[j] = 0.f;
     if (j < NS && live && n < N) {
       A[j] = -expf(p.A_log[d * N + n]);
-      Acoef[j] = PRECISE ? A[j] : A[j] * kLog2e;
       nIA[j] = -1.0f / A[j];
     } else {
       A[j] = 0.f;
-      Acoef[j] = 0.f;
       nIA[j] = 0.f;
     }
   }
@@ -411,10 +409,11 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
         for (int tt = 0; tt < 4; tt++) {
           if (PAIRS) {
             const float2 dl2 = make_float2(eq[tt].x, eq[tt].x), u2 = make_float2(eq[tt].y, eq[tt].y);
+            const float dlg = eq[tt].x * kLog2e;
             float2 y2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < NH; q++) {
-              const float2 x = __fmul2_rn(dl2, Ac2[q]);
+              const float2 x = __fmul2_rn(make_float2(dlg, dlg), A2[q]);
               float2 a;
               a.x = ex2_approx(x.x);
               a.y = ex2_approx(x.y);
@@ -439,12 +438,12 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
             for (int j = 0; j < NS; j++) {
               const float nw = Bt[j] * eq[tt].y * nIA[j];  // -B u / A
               if (PRECISE) {
-                const float em1 = expm1f(eq[tt].x * Acoef[j]);
+                const float em1 = expm1f(eq[tt].x * A[j]);
                 h[j] = EULER ? fmaf(em1, h[j], fmaf(eq[tt].x * Bt[j], eq[tt].y, h[j]))
                              : fmaf(em1, h[j] - nw, h[j]);
                 av[tt * NS + j] = em1;
               } else {
-                const float a = ex2_approx(eq[tt].x * Acoef[j]);
+                const float a = ex2_approx((eq[tt].x * kLog2e) * A[j]);
                 h[j] = EULER ? fmaf(a, h[j], eq[tt].x * Bt[j] * eq[tt].y) : fmaf(a, h[j] - nw, nw);
                 av[tt * NS + j] = a;
               }
@@ -516,7 +515,8 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
           for (int q = 0; q < NH; q++) {
             float2 a2;
             if constexpr (S::AREC) {
-              const float2 x = __fmul2_rn(dl2, Ac2[q]);  // as in the recompute: same bits
+              const float dlg = e.x * kLog2e;
+              const float2 x = __fmul2_rn(make_float2(dlg, dlg), A2[q]);  // as in the recompute: same bits
               a2 = make_float2(ex2_approx(x.x), ex2_approx(x.y));
             } else {
               a2 = make_float2(av[tt * NS + 2 * q], av[tt * NS + 2 * q + 1]);
@@ -548,7 +548,7 @@ ssm_bwd_kernel(const BwdParams P, const __grid_constant__ CUtensorMap tmx,
           const float *Ct = reinterpret_cast<const float *>(Cv);
 #pragma unroll
           for (int j = 0; j < NS; j++) {
-            const float aj = S::AREC ? ex2_approx(e.x * Acoef[j]) : av[tt * NS + j];
+            const float aj = S::AREC ? ex2_approx((e.x * kLog2e) * A[j]) : av[tt * NS + j];
             const float em1 = PRECISE ? aj : aj - 1.f;
             const float hs = hv[tt * NS + j];
             lam[j] = fmaf(aN[j], lam[j], Ct[j] * e.z);
@@ -880,9 +880,10 @@ __global__ void reduce_tiles_kernel(const float *__restrict__ pdB, const float *
 // per-channel parameters: add the (segment, batch) partials in order.
 // The same sum, 4 consecutive elements per thread with 16-byte accesses and 8 tiles' loads in
 // flight; the adds still run in tile order, so the result is bitwise that of the scalar kernel.
-__global__ void reduce_tiles_vec_kernel(const float4 *__restrict__ pdB, const float4 *__restrict__ pdC,
-                                        float4 *dB, float4 *dC, int64_t n_tiles, int64_t per_tile4) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// dB / dC: thread i adds 4 consecutive floats of the channel-tile partials in tile order.
+__device__ __forceinline__ void reduce_tiles_vec_at(const float4 *__restrict__ pdB, const float4 *__restrict__ pdC,
+                                                    float4 *dB, float4 *dC, int64_t n_tiles, int64_t per_tile4,
+                                                    int64_t i) {
   if (i >= per_tile4) return;
   float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
   constexpr int U = 8;
@@ -907,10 +908,18 @@ __global__ void reduce_tiles_vec_kernel(const float4 *__restrict__ pdB, const fl
   if (dC) dC[i] = sc;
 }
 
-__global__ void reduce_params_kernel(const BwdParams P) {
-  const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// per-channel parameters: thread j = d * N + n adds the (segment, batch) partials of dA_log[d, n]
+// in order, and the thread of state 0 those of the channel's D, dt_bias, conv bias and taps.
+__device__ __forceinline__ void reduce_params_at(const BwdParams &P, int64_t j) {
   const int64_t Dn = P.f.Dn, N = P.f.N, Bt = P.f.Bt * P.n_seg;
-  if (d >= Dn) return;
+  if (j >= Dn * N) return;
+  const int64_t d = j / N, n = j - d * N;
+  if (P.dA_log) {
+    float s = 0.f;
+    for (int64_t b = 0; b < Bt; b++) s += P.p_dA_log[b * Dn * N + j];
+    P.dA_log[j] = s;
+  }
+  if (n != 0) return;
   float sD = 0.f, sT = 0.f, sCb = 0.f, sW[4] = {0.f, 0.f, 0.f, 0.f};
   for (int64_t b = 0; b < Bt; b++) {
     sD += P.p_dD[b * Dn + d];
@@ -923,14 +932,23 @@ __global__ void reduce_params_kernel(const BwdParams P) {
   if (P.dconv_b) P.dconv_b[d] = sCb;
   if (P.dconv_w)
     for (int k = 0; k < P.f.K; k++) P.dconv_w[d * P.f.K + k] = sW[k];
-  if (P.dA_log)
-    for (int64_t n = 0; n < N; n++) {
-      float s = 0.f;
-      for (int64_t b = 0; b < Bt; b++) s += P.p_dA_log[(b * Dn + d) * N + n];
-      P.dA_log[d * N + n] = s;
-    }
 }
 
+// Both reductions in one launch where the dB / dC rows are whole 16-byte vectors: blocks
+// [0, n_tb) take the dB / dC tiles, the blocks after them the per-channel parameters.
+__global__ void reduce_all_vec_kernel(const BwdParams P, int64_t n_tb, int64_t per_tile4) {
+  if ((int64_t)blockIdx.x < n_tb) {
+    reduce_tiles_vec_at(reinterpret_cast<const float4 *>(P.p_dB), reinterpret_cast<const float4 *>(P.p_dC),
+                        reinterpret_cast<float4 *>(P.dB), reinterpret_cast<float4 *>(P.dC), P.n_ptiles,
+                        per_tile4, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    return;
+  }
+  reduce_params_at(P, ((int64_t)blockIdx.x - n_tb) * blockDim.x + threadIdx.x);
+}
+
+__global__ void reduce_params_kernel(const BwdParams P) {
+  reduce_params_at(P, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+}
 
 // Split-L pass 1: for every segment but the first, the adjoint run backwards from a zero arrival
 // -- lambda_t = dy_t C_t + A_bar_{t+1} lambda_{t+1} over [ts, te) -- needs only Delta, dy and C
@@ -1204,22 +1222,22 @@ cudaError_t launch_bwd(const BwdParams &P, int in_bf16, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   const int64_t per_tile = P.f.Bt * P.f.N * P.f.L;
+  const int64_t n_pb = (P.f.Dn * P.f.N + 255) / 256;  // blocks of the parameter reduction
   if (P.dB || P.dC) {
     const bool vec = per_tile % 4 == 0 && ((reinterpret_cast<uintptr_t>(P.p_dB) | reinterpret_cast<uintptr_t>(P.p_dC) |
                                              reinterpret_cast<uintptr_t>(P.dB) | reinterpret_cast<uintptr_t>(P.dC)) & 15) == 0;
     if (vec) {
-      const int64_t blocks = (per_tile / 4 + 255) / 256;
-      reduce_tiles_vec_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-          reinterpret_cast<const float4 *>(P.p_dB), reinterpret_cast<const float4 *>(P.p_dC),
-          reinterpret_cast<float4 *>(P.dB), reinterpret_cast<float4 *>(P.dC), P.n_ptiles, per_tile / 4);
-    } else {
-      const int64_t blocks = (per_tile + 255) / 256;
-      reduce_tiles_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P.p_dB, P.p_dC, P.dB, P.dC, P.n_ptiles, per_tile);
+      const int64_t n_tb = (per_tile / 4 + 255) / 256;
+      if (n_tb + n_pb > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+      reduce_all_vec_kernel<<<(unsigned)(n_tb + n_pb), 256, 0, stream>>>(P, n_tb, per_tile / 4);
+      return cudaGetLastError();
     }
+    const int64_t blocks = (per_tile + 255) / 256;
+    reduce_tiles_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P.p_dB, P.p_dC, P.dB, P.dC, P.n_ptiles, per_tile);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  reduce_params_kernel<<<(unsigned)((P.f.Dn + 127) / 128), 128, 0, stream>>>(P);
+  reduce_params_kernel<<<(unsigned)n_pb, 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
 
