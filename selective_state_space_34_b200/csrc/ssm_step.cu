@@ -1,12 +1,12 @@
 // ssm_step.cu -- one-token decode step ("Selective Mamba", step): every channel advances its
 // carried state by one token and emits one output, reading and rewriting the state in place.
 //
-// A warp takes 32 consecutive (batch, channel) rows. Lane c forms row c's per-channel scalars
-// (conv + SiLU, Delta, the gate) once, and owns its output and its conv history (read and
-// rewritten by that lane alone). The states are updated in P passes over the warp's rows, P lanes
-// per row and 4 states per lane (P = ceil(N / 4) rounded up to a power of two, 4 at N = 16): pass q
-// takes rows q R .. q R + R - 1 (R = 32 / P rows per pass) and lane l row q R + l / P, states
-// 4 (l % P) .. 4 (l % P) + 3. With N = 4 P the 16-byte state and A_log accesses of a pass then
+// A warp takes 32 kStepRows consecutive (batch, channel) rows, handled as kStepRows slots of 32.
+// Lane c forms the per-channel scalars (conv + SiLU, Delta, the gate) of row c of every slot once,
+// and owns those rows' outputs and conv histories (read and rewritten by that lane alone). The
+// states of a slot are updated in P passes, P lanes per row and 4 states per lane (P = ceil(N / 4)
+// rounded up to a power of two, 4 at N = 16): pass q takes the slot's rows q R .. q R + R - 1
+// (R = 32 / P rows per pass) and lane l row q R + l / P, states 4 (l % P) .. 4 (l % P) + 3. With N = 4 P the 16-byte state and A_log accesses of a pass then
 // cover one contiguous span of the warp (a row-per-lane layout puts 16 rows, 16 cache lines, under
 // every 16-byte access). A pass takes its row's u and Delta from the owning lane by shuffles, and
 // the P partial readouts sum_n C_n h_n are added by shuffles and handed to the owning lane. Each
@@ -20,6 +20,13 @@
 
 namespace ssm {
 
+// (batch, channel) rows per lane: 2 keeps the whole 64 x 4096 decode grid in one wave (1024 CTAs
+// of 128 threads at up to 8 per SM) where one row per lane needed 1.4 waves.
+#ifndef SSM_STEP_ROWS
+#define SSM_STEP_ROWS 2
+#endif
+constexpr int kStepRows = SSM_STEP_ROWS;
+
 template <typename Tin, typename Tout, bool EULER, int P>
 __global__ void __launch_bounds__(128) ssm_step_kernel(const StepParams p) {
   constexpr int R = 32 / P;  // rows per pass
@@ -27,65 +34,76 @@ __global__ void __launch_bounds__(128) ssm_step_kernel(const StepParams p) {
   constexpr unsigned kFull = 0xffffffffu;
   const int64_t rows = p.Bt * p.Dn;
   const int lane = threadIdx.x & 31;
-  const int64_t row0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x - lane;  // the warp's first row
-  const int64_t gi = row0 + lane;
-  const bool live = gi < rows;
-  const int64_t i = live ? gi : rows - 1;  // dead lanes compute on a valid row and store nothing
-  int64_t b, d;
-  if (rows <= 0x7fffffffLL) {  // 32-bit division where it fits (always, in practice)
-    const uint32_t i32 = (uint32_t)i, dn = (uint32_t)p.Dn;
-    b = i32 / dn;
-    d = i32 - (uint32_t)b * dn;
-  } else {
-    b = i / p.Dn;
-    d = i % p.Dn;
-  }
+  const int64_t row0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x - lane) * kStepRows;  // the warp's first row
   const int64_t N = p.N;
 
-  // -- this lane's row: the per-channel scalars
-  const Tin xin = static_cast<const Tin *>(p.x)[i];
-  float u;
-  if (p.conv_w) {
-    const int K = p.K;
-    float acc = (p.conv_b ? p.conv_b[d] : 0.f) + p.conv_w[d * K] * to_f32(xin);
-    if (K > 1) {
-      Tin *hist = static_cast<Tin *>(p.conv_hist) + i * (K - 1);
-      Tin old[3];
+  // -- this lane's rows row0 + 32 k + lane: the per-channel scalars
+  float u[kStepRows], dl[kStepRows];
+  int64_t bk[kStepRows], dk[kStepRows];
 #pragma unroll
-      for (int j = 0; j < 3; j++)
-        if (j < K - 1) old[j] = hist[j];
-#pragma unroll
-      for (int k = 1; k < 4; k++)
-        if (k < K) acc = fmaf(p.conv_w[d * K + k], to_f32(old[k - 1]), acc);
-      if (live) {  // the new token becomes the newest entry, the oldest one drops out
-        hist[0] = xin;
-#pragma unroll
-        for (int j = 1; j < 3; j++)
-          if (j < K - 1) hist[j] = old[j - 1];
-      }
+  for (int k = 0; k < kStepRows; k++) {
+    const int64_t gi = row0 + 32 * k + lane;
+    const bool live = gi < rows;
+    const int64_t i = live ? gi : rows - 1;  // dead rows are computed on a valid row and not stored
+    int64_t b, d;
+    if (rows <= 0x7fffffffLL) {  // 32-bit division where it fits (always, in practice)
+      const uint32_t i32 = (uint32_t)i, dn = (uint32_t)p.Dn;
+      b = i32 / dn;
+      d = i32 - (uint32_t)b * dn;
+    } else {
+      b = i / p.Dn;
+      d = i % p.Dn;
     }
-    u = acc * sigmoid<PRECISE>(acc);
-  } else {
-    u = to_f32(xin);
+    bk[k] = b;
+    dk[k] = d;
+    const Tin xin = static_cast<const Tin *>(p.x)[i];
+    float uk;
+    if (p.conv_w) {
+      const int K = p.K;
+      float acc = (p.conv_b ? p.conv_b[d] : 0.f) + p.conv_w[d * K] * to_f32(xin);
+      if (K > 1) {
+        Tin *hist = static_cast<Tin *>(p.conv_hist) + i * (K - 1);
+        Tin old[3];
+#pragma unroll
+        for (int j = 0; j < 3; j++)
+          if (j < K - 1) old[j] = hist[j];
+#pragma unroll
+        for (int kk = 1; kk < 4; kk++)
+          if (kk < K) acc = fmaf(p.conv_w[d * K + kk], to_f32(old[kk - 1]), acc);
+        if (live) {  // the new token becomes the newest entry, the oldest one drops out
+          hist[0] = xin;
+#pragma unroll
+          for (int j = 1; j < 3; j++)
+            if (j < K - 1) hist[j] = old[j - 1];
+        }
+      }
+      uk = acc * sigmoid<PRECISE>(acc);
+    } else {
+      uk = to_f32(xin);
+    }
+    u[k] = uk;
+    const float v = to_f32(static_cast<const Tin *>(p.dt)[i]) + (p.dt_bias ? p.dt_bias[d] : 0.f);
+    dl[k] = p.delta_softplus ? softplus<PRECISE>(v) : v;
   }
-  const float v = to_f32(static_cast<const Tin *>(p.dt)[i]) + (p.dt_bias ? p.dt_bias[d] : 0.f);
-  const float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
 
-  // -- the states, in P passes of 4 states per lane
+  // -- the states, in kStepRows * P passes of 4 states per lane
   const int sq = lane % P, rl = lane / P;
   const int64_t n0 = 4 * sq;
   const uintptr_t bc_align = PRECISE ? 15 : 7;  // 4 values of B_t / C_t as one access
   const bool vec = N == 4 * P && ((reinterpret_cast<uintptr_t>(p.h) | reinterpret_cast<uintptr_t>(p.A_log)) & 15) == 0 &&
                    ((reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & bc_align) == 0;
-  float yown = 0.f;  // this lane's row readout, collected from the pass that updates it
+  float yown[kStepRows];  // this lane's row readouts, collected from the passes that update them
 #pragma unroll
-  for (int q = 0; q < P; q++) {
-    const int src = q * R + rl;  // the lane that owns the row of this pass
-    const float ur = __shfl_sync(kFull, u, src);
-    const float dlr = __shfl_sync(kFull, dl, src);
-    const int64_t br = __shfl_sync(kFull, (long long)b, src);
-    const int64_t dr = __shfl_sync(kFull, (long long)d, src);
-    const int64_t r = row0 + src;
+  for (int k = 0; k < kStepRows; k++) yown[k] = 0.f;
+#pragma unroll
+  for (int q = 0; q < kStepRows * P; q++) {
+    const int k = q / P;                  // the slot of the pass's rows in their owners
+    const int src = (q % P) * R + rl;     // the lane that owns this lane's row of the pass
+    const float ur = __shfl_sync(kFull, u[k], src);
+    const float dlr = __shfl_sync(kFull, dl[k], src);
+    const int64_t br = __shfl_sync(kFull, (long long)bk[k], src);
+    const int64_t dr = __shfl_sync(kFull, (long long)dk[k], src);
+    const int64_t r = row0 + 32 * k + src;
     const bool rlive = r < rows;
     const int64_t rr = rlive ? r : rows - 1;
     float *h = p.h + rr * N + n0;
@@ -155,22 +173,26 @@ __global__ void __launch_bounds__(128) ssm_step_kernel(const StepParams p) {
 #pragma unroll
     for (int off = P / 2; off >= 1; off >>= 1) y += __shfl_xor_sync(kFull, y, off);
     const float yr = __shfl_sync(kFull, y, (lane % R) * P);
-    if (lane / R == q) yown = yr;
+    if (lane / R == q % P) yown[k] = yr;
   }
-  if (live) {
-    float y = fmaf(p.D ? p.D[d] : 0.f, u, yown);
-    if (p.z) {
-      const float zz = to_f32(static_cast<const Tin *>(p.z)[i]);
-      y *= zz * sigmoid<PRECISE>(zz);
+#pragma unroll
+  for (int k = 0; k < kStepRows; k++) {
+    const int64_t gi = row0 + 32 * k + lane;
+    if (gi < rows) {
+      float y = fmaf(p.D ? p.D[dk[k]] : 0.f, u[k], yown[k]);
+      if (p.z) {
+        const float zz = to_f32(static_cast<const Tin *>(p.z)[gi]);
+        y *= zz * sigmoid<PRECISE>(zz);
+      }
+      static_cast<Tout *>(p.out)[gi] = from_f32<Tout>(y);
     }
-    static_cast<Tout *>(p.out)[i] = from_f32<Tout>(y);
   }
 }
 
 template <typename Tin, typename Tout, int P>
 static cudaError_t step_p(const StepParams &p, cudaStream_t s) {
-  const int64_t n = p.Bt * p.Dn;  // one thread per (batch, channel) row
-  const int64_t blocks = (n + 127) / 128;
+  const int64_t warps = (p.Bt * p.Dn + 32 * kStepRows - 1) / (32 * kStepRows);  // 32 kStepRows rows each
+  const int64_t blocks = (warps + 3) / 4;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (p.euler)
     ssm_step_kernel<Tin, Tout, true, P><<<(unsigned)blocks, 128, 0, s>>>(p);
