@@ -18,14 +18,16 @@
 //
 // Decomposition mirrors the forward: a CTA owns CH = 128/G channels of one batch element, lanes
 // hold NS states each, and the sequence is walked backwards in stages of 16 steps (one saved-state
-// chunk each): recompute the stage forward from its saved start state, keeping h_t of every step
-// (and a_t on the precise path; the fast path recomputes it) in the thread's lane of tensor memory
-// (TMEM, otherwise idle here) instead of registers, then run the adjoint backwards through it one
-// 4-step group at a time. Moving that trajectory out of the register file is what lets four CTAs
+// chunk each): recompute the stage forward from its saved start state, keeping h_t and a_t of
+// every step (a_t - 1 on the precise path) in the thread's lane of tensor memory (TMEM, otherwise
+// idle here) instead of registers, then run the adjoint backwards through it one 4-step group at a
+// time. Moving that trajectory out of the register file is what lets four CTAs
 // share an SM. dB and dC are summed over the CTA's channels (a warp butterfly per step and one
 // cross-warp sum per stage, or a shared-memory sum after every 4 steps for the other lane layouts)
-// and written as per-tile partials; a second kernel adds the tiles (and the per-batch partials of
-// the per-channel parameter gradients) in a fixed order, so the result is deterministic.
+// and written as per-tile partials; one more launch adds the tiles (and the per-batch partials of
+// the per-channel parameter gradients) in a fixed order, so the result is deterministic. The
+// stage's x, dt, z and dout rows arrive by TMA boxes where rows are 16-byte aligned, else by
+// 16-byte cp.async.
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 #include "ssm_stage.cuh"
