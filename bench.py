@@ -65,17 +65,18 @@ def job_throughput(units_per_rank, world, steps, max_ms):
     return units_per_rank * world * steps / (max_ms * 1e-3)
 
 
-def ncu_traffic(kernel, source):
+def ncu_traffic(kernel, source, workload):
     """DRAM bytes per launch of `kernel` (dram__bytes_read.sum + dram__bytes_write.sum from one ncu
     capture, stored in profiles/ncu_traffic.json with the command that took it), or None when the
-    capture was taken on a different version of the kernel's source file."""
+    capture was taken on another workload (the entry lists the workloads that launch the kernel
+    on the captured shape and dtypes) or on a different version of the kernel's source file."""
     import hashlib
     try:
         sha = hashlib.sha256(open(os.path.join(ROOT, "selective_state_space_34_b200", "csrc", source),
                                   "rb").read()).hexdigest()[:16]
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             rec = json.load(f)["kernels"].get(kernel)
-        if rec and rec.get("source_sha256_16") == sha:
+        if rec and rec.get("source_sha256_16") == sha and workload in rec.get("workloads", []):
             return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
@@ -420,7 +421,7 @@ def ssd_bench(args, cfg, name):
                    "step": "ssd forward (1 launch, fused)" if fused else "ssd forward (3 launches)",
                    "form": "fused" if fused else "three_pass", "l2": "inputs larger than L2"},
         "roofline": {"bound": "hbm", "achieved": ob / (out_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                     "frac": ob / (out_ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic(kname, ksrc),
+                     "frac": ob / (out_ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic(kname, ksrc, name),
                      "algorithmic_bytes": ob, "kernel": kname, "ms": out_ms,
                      "peak_source": peaks.get("source")},
         "tensor": {"achieved": oflops / (out_ms * 1e-3) / 1e12, "peak": bf16, "unit": "TFLOP/s",
@@ -535,7 +536,7 @@ def decode_bench(args, w):
         "eager_us_per_token_step": eager_ms * 1e3 / T,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "algorithmic_bytes": bytes_step, "kernel": "ssm_step_kernel",
-                     "traffic": ncu_traffic("ssm_step_kernel", "ssm_step.cu"), "peak_source": peaks.get("source")},
+                     "traffic": ncu_traffic("ssm_step_kernel", "ssm_step.cu", w.name), "peak_source": peaks.get("source")},
         "gpu_launches": T * args.steps, "clocks": clk,
     }
     if rank == 0:
@@ -603,7 +604,7 @@ def conv_bench(args, w):
                    "l2": "inputs larger than L2 (%.0f MB per call)" % (nbytes / 1e6)},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "algorithmic_bytes": nbytes, "kernel": "conv1d_silu_vec_kernel",
-                     "traffic": ncu_traffic("conv1d_silu_vec_kernel", "ssm_conv.cu"), "peak_source": peaks.get("source")},
+                     "traffic": ncu_traffic("conv1d_silu_vec_kernel", "ssm_conv.cu", w.name), "peak_source": peaks.get("source")},
         "gpu_launches": args.steps, "clocks": clk,
     }
     if rank == 0:
@@ -821,7 +822,7 @@ def main():
     fb = fwd_bytes(Bt, Dn, N, L, s_in, s_out)
     fwd_roof = {"bound": "hbm", "achieved": fb / (fo_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": fb / (fo_ms * 1e-3) / 1e9 / hbm,
-                "traffic": ncu_traffic("ssm_fwd_kernel", "ssm_fwd.cu") if (s_out == 2 and s_in == 2) else None,
+                "traffic": ncu_traffic("ssm_fwd_kernel", "ssm_fwd.cu", w.name) if (s_out == 2 and s_in == 2) else None,
                 "algorithmic_bytes": fb, "kernel": "ssm_fwd_kernel", "ms": fo_ms,
                 "peak_source": peaks.get("source")}
     sm_hz = (clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6
@@ -843,7 +844,7 @@ def main():
         bb = bwd_bytes(Bt, Dn, N, L, s_in)
         roof = {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": bb / (bms * 1e-3) / 1e9 / hbm,
-                "traffic": ncu_traffic("ssm_bwd_kernel", "ssm_bwd.cu") if s_in == 2 else None,
+                "traffic": ncu_traffic("ssm_bwd_kernel", "ssm_bwd.cu", w.name) if s_in == 2 else None,
                 "algorithmic_bytes": bb, "kernel": "ssm_bwd_kernel", "ms": bms,
                 "peak_source": peaks.get("source"),
                 "overhead_bytes": bwd_overhead_bytes(Bt, Dn, N, n_ck)}

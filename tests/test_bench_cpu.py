@@ -51,3 +51,24 @@ def test_parity_report_flags_a_wrong_element():
 
 def bench_atol(ref):
     return 1e-4 * abs(ref).max()
+
+
+def test_measured_traffic_is_attached_only_to_its_workload_and_source(tmp_path, monkeypatch):
+    """A stored ncu capture counts for the workloads its entry lists and only while the kernel's
+    source file is the one it was taken on."""
+    import hashlib
+    import json
+    src = tmp_path / "selective_state_space_34_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k.cu").write_text("// kernel source\n")
+    sha = hashlib.sha256(b"// kernel source\n").hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps({"kernels": {"k": {
+        "source": "k.cu", "source_sha256_16": sha, "dram_bytes_per_launch": 1234,
+        "workloads": ["shape_a"]}}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("k", "k.cu", "shape_a") == 1234
+    assert bench.ncu_traffic("k", "k.cu", "shape_b") is None      # another workload
+    assert bench.ncu_traffic("other", "k.cu", "shape_a") is None  # no entry
+    (src / "k.cu").write_text("// kernel source, edited\n")
+    assert bench.ncu_traffic("k", "k.cu", "shape_a") is None      # the source changed
