@@ -850,10 +850,12 @@ def main():
                 "overhead_bytes": bwd_overhead_bytes(Bt, Dn, N, n_ck)}
     else:
         roof = dict(fwd_roof)
-    # a split forward is three launches (segment summaries, carry, segments); a split backward
-    # adds the adjoint summaries, their carry and the dx fix-up to its kernel and two reductions
+    # a split forward is three launches (segment summaries, carry, segments); the backward is its
+    # kernel and one reduction launch (dB / dC tiles and per-channel parameters, rows of whole
+    # 16-byte vectors as here), and a split backward adds the adjoint summaries, their carry and
+    # the dx fix-up
     split = ws_f is not None
-    launches_per_step = (3 if split else 1) + ((6 if split else 3) if backward else 0)
+    launches_per_step = (3 if split else 1) + ((5 if split else 2) if backward else 0)
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, compute, D2H results ----
     # Every step copies its inputs from pinned host memory and reads all of its results back (the
