@@ -148,6 +148,31 @@ def test_decode_step_state_sizes_and_bf16_out(N):
     assert_close("h", to_np(h), ex["h_last"], *TOL[("bf16", "f32")])
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_step_misaligned_rows_give_the_same_bits(dtype):
+    """State, A_log, B and C one element off a 16-byte boundary take the element-by-element path
+    of the state passes; the same values in aligned storage take the 16-byte path. Same bits."""
+    w, a, t = _setup(3, 45, 16, 1, dtype)
+    col = lambda v: v[..., 0].contiguous()
+
+    def shifted(v):  # the same values, starting one element into a fresh buffer
+        buf = torch.empty(v.numel() + 1, dtype=v.dtype, device=v.device)
+        out = buf[1:].view(v.shape)
+        out.copy_(v)
+        return out
+
+    kw = dict(D=t["D"], z=col(t["z"]), dt_bias=t["dt_bias"], conv_w=t["conv_w"], conv_b=t["conv_b"],
+              out_dtype=torch.float32)
+    h1, hist1 = t["h0"].clone(), t["conv_hist"].clone()
+    y1 = ssm.ssm_scan_step(col(t["x"]), col(t["dt"]), t["A_log"], col(t["B"]), col(t["C"]), h1, hist1, **kw)
+    h2, hist2 = shifted(t["h0"]), t["conv_hist"].clone()
+    y2 = ssm.ssm_scan_step(col(t["x"]), col(t["dt"]), shifted(t["A_log"]), shifted(col(t["B"])),
+                           shifted(col(t["C"])), h2, hist2, **kw)
+    torch.cuda.synchronize()
+    assert h2.data_ptr() % 16 != 0
+    assert torch.equal(y1, y2) and torch.equal(h1, h2) and torch.equal(hist1, hist2)
+
+
 def test_scan_then_step_continues_the_scan():
     """A scan over the first L-1 tokens followed by one decode step matches the scan over L."""
     L = 33
