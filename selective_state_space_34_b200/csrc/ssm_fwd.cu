@@ -207,7 +207,8 @@ ssm_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap tmx,
       load_window<Tin, EPL + 4>(xw, xrow + tb - 4);
       load_window<Tin, EPL>(dtw, dtrow + tb);
       if (has_z) load_window<Tin, EPL>(zw, zrow + tb);
-      float gate[EPL], uown[EPL];
+      float gate[EPL], uown[EPL], dlown[EPL];
+      const bool tail = t0 + kT > te;  // this stage runs past the end of the sequence
 #pragma unroll
       for (int j = 0; j < EPL; j++) {
         const int t = tb + j;
@@ -224,15 +225,21 @@ ssm_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap tmx,
         float dl = p.delta_softplus ? softplus<PRECISE>(v) : v;
         float s = 1.0f;
         if (has_z) s = zw[j] * sigmoid<PRECISE>(zw[j]);
-        if (t0 + t >= te) {  // padded tail: an identity step
+        if (tail && t0 + t >= te) {  // padded tail: an identity step
           u = 0.0f;
           dl = 0.0f;
         }
-        ud[c * S::US + g * EPL + j] = make_float2(dl, u);
+        if constexpr (EPL % 2 != 0) ud[c * S::US + g * EPL + j] = make_float2(dl, u);
+        dlown[j] = dl;
         gate[j] = s;
         uown[j] = u;
         if (!tma && t >= kT - 3)  // carry the conv halo into the next stage's prefix (TMA brings it)
           xs[(nbuf * CH + c) * S::XS + kPre + t - kT] = xrow[t];
+      }
+      if constexpr (EPL % 2 == 0) {
+#pragma unroll
+        for (int j = 0; j < EPL; j += 2)
+          *reinterpret_cast<float4 *>(ud + c * S::US + g * EPL + j) = make_float4(dlown[j], uown[j], dlown[j + 1], uown[j + 1]);
       }
       if (!SUMMARY && p.u_out && live)
         store_run<Tout, EPL>(static_cast<Tout *>(p.u_out) + row0 + (int64_t)c * L,
@@ -245,13 +252,17 @@ ssm_fwd_kernel(const FwdParams p, const __grid_constant__ CUtensorMap tmx,
 #pragma unroll
       for (int tq = 0; tq < kSub; tq += 4) {
         float dlq[4], uq[4], Bq[4][NS], Cq[4][NS];
+        {
+          // the group's (Delta, u) pairs as two 16-byte reads (rows and groups are 16-byte aligned)
+          const float4 d01 = *reinterpret_cast<const float4 *>(ud + c * S::US + tq);
+          const float4 d23 = *reinterpret_cast<const float4 *>(ud + c * S::US + tq + 2);
+          dlq[0] = d01.x; uq[0] = d01.y; dlq[1] = d01.z; uq[1] = d01.w;
+          dlq[2] = d23.x; uq[2] = d23.y; dlq[3] = d23.z; uq[3] = d23.w;
+        }
 #pragma unroll
         for (int tt = 0; tt < 4; tt++) {
           const int t = sb * kSub + tq + tt;
-          const float2 du = ud[c * S::US + tq + tt];
-          dlq[tt] = du.x;
-          uq[tt] = du.y;
-          if (SUMMARY) sdl += du.x;
+          if (SUMMARY) sdl += dlq[tt];
           load_states<NS>(Bq[tt], Bst + t * S::BS + g * NS);
           load_states<NS>(Cq[tt], Cst + t * S::BS + g * NS);
         }
